@@ -1,0 +1,185 @@
+"""Pins of the oracle's routing, permutation, FFN and combine (CPU only).
+
+Routing follows the pages "thinkingmachines/Inkling-2-Small" (Overview) and
+"Thinking Machines releases Inkling 2 Small weights under Apache 2.0"
+("NVFP4 and MXFP8 experts"): top-k of E routed experts, no shared expert.
+The checks compare with numpy's stable argsort and bincount (library
+routines), math.exp, a dense FFN written out directly, and a per-token loop.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+from oracle import formats as fm
+from oracle import moe
+from oracle import route as rt
+from fp8_moe_expert_top_b200 import inputs
+
+
+# ---------------------------------------------------------------- exp_own
+
+def test_exp_own_accuracy_against_math_exp():
+    x = np.concatenate([np.linspace(-80, 0, 200001), -np.exp2(np.linspace(-30, 6, 2000))]).astype(np.float32)
+    got = rt.exp_own(x).astype(np.float64)
+    ref = np.array([math.exp(float(v)) for v in x])
+    rel = np.abs(got - ref) / ref
+    assert rel.max() <= 3 * 2.0 ** -24, rel.max()
+    assert rt.exp_own(np.float32(0.0)) == np.float32(1.0)
+    assert rt.exp_own(np.float32(-80.5)) == 0.0
+
+
+# ---------------------------------------------------------------- top-k
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_topk_matches_stable_argsort(ties):
+    T, E, k = 300, 384, 8
+    if ties:
+        lg = inputs.make_logits_with_ties(T, E, seed=3).numpy()
+    else:
+        lg = np.random.default_rng(2).standard_normal((T, E)).astype(np.float32)
+    ids = rt.topk_select(lg, k)
+    ref = np.argsort(-lg, axis=1, kind="stable")[:, :k]
+    np.testing.assert_array_equal(ids, ref)
+
+
+def test_topk_signed_zero_ties_to_lower_index():
+    lg = np.full((1, 6), -1.0, dtype=np.float32)
+    lg[0, 4] = 0.0
+    lg[0, 1] = -0.0
+    ids = rt.topk_select(lg, 2)
+    assert ids.tolist() == [[1, 4]]
+
+
+def test_softmax_weights():
+    lg = np.random.default_rng(4).standard_normal((50, 16)).astype(np.float32)
+    ids = rt.topk_select(lg, 1)
+    assert np.all(rt.topk_softmax(lg, ids) == np.float32(1.0))
+    ids = rt.topk_select(lg, 4)
+    w = rt.topk_softmax(lg, ids)
+    sel = np.take_along_axis(lg.astype(np.float64), ids.astype(np.int64), axis=1)
+    ref = np.exp(sel - sel[:, :1])
+    ref /= ref.sum(1, keepdims=True)
+    np.testing.assert_allclose(w, ref, rtol=4e-7)
+    assert np.all(np.diff(w, axis=1) <= 0)             # rank order
+
+
+# ---------------------------------------------------------------- slot sort
+
+def test_sort_slots_matches_library_sort():
+    rng = np.random.default_rng(5)
+    T, E, k = 200, 24, 3
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    lg[:, 5] += 3.0                                     # one hot expert
+    lg[:, 7] -= 50.0                                    # one cold expert (no slots)
+    ids = rt.topk_select(lg, k)
+    counts, offsets, sorted_slots, slot_to_row = rt.sort_slots(ids, E)
+    flat = ids.reshape(-1)
+    np.testing.assert_array_equal(counts, np.bincount(flat, minlength=E))
+    assert counts[7] == 0
+    seg = np.diff(offsets)
+    assert np.all(offsets % 128 == 0)
+    np.testing.assert_array_equal(seg, (counts + 127) // 128 * 128)
+    # valid rows in (expert, token) order == a stable sort of the slots by expert
+    order = np.argsort(flat, kind="stable")
+    valid = sorted_slots[sorted_slots >= 0]
+    np.testing.assert_array_equal(valid, order)
+    # inverse map and padding
+    assert np.all(slot_to_row[sorted_slots[sorted_slots >= 0]] == np.nonzero(sorted_slots >= 0)[0])
+    for e in range(E):
+        lo = offsets[e]
+        assert np.all(sorted_slots[lo + counts[e]:offsets[e + 1]] == -1)
+        assert np.all(flat[sorted_slots[lo:lo + counts[e]]] == e)
+
+
+def test_combine_of_passthrough_is_identity():
+    """Permute x by the slot sort, combine with k=1 and w=1: y == x exactly."""
+    rng = np.random.default_rng(6)
+    T, E, H = 40, 6, 32
+    x = fm.bf16_round(rng.standard_normal((T, H)))
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    r = rt.route(lg, 1, E)
+    rows = np.zeros((r["sorted_slots"].shape[0], H))
+    valid = r["sorted_slots"] >= 0
+    rows[valid] = x[r["sorted_slots"][valid]]
+    y = moe.combine(rows, r["topk_w"], r["slot_to_row"])
+    np.testing.assert_array_equal(y, x)
+
+
+# ---------------------------------------------------------------- the layer
+
+def _small_case(fmt, T=24, H=64, I=32, E=4, k=2, seed=7):
+    rng = np.random.default_rng(seed)
+    x = fm.bf16_round(rng.standard_normal((T, H))).astype(np.float32)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    experts = {}
+    raw = {}
+    for e in range(E):
+        wg = (rng.standard_normal((I, H)) / math.sqrt(H)).astype(np.float32)
+        wu = (rng.standard_normal((I, H)) / math.sqrt(H)).astype(np.float32)
+        wd = (rng.standard_normal((H, I)) / math.sqrt(I)).astype(np.float32)
+        raw[e] = (wg, wu, wd)
+        experts[e] = moe.quantize_expert(wg, wu, wd, fmt)
+    return x, lg, experts, raw
+
+
+@pytest.mark.parametrize("fmt", [moe.NVFP4, moe.MXFP8])
+def test_one_expert_layer_equals_dense_ffn(fmt):
+    """E = 1, k = 1: the routed layer is exactly the dense FFN of that expert."""
+    x, lg, experts, raw = _small_case(fmt, T=16, H=64, I=32, E=1, k=1)
+    s_x, s_h = np.float32(8 / 2688), np.float32(24 / 2688)
+    res = moe.forward(x, lg, experts, 1, fmt, s_x, s_h)
+    # dense FFN written out: quantize x, dequantize, GEMM, SwiGLU, requantize, GEMM
+    if fmt == moe.NVFP4:
+        xc, xs = fm.nvfp4_quantize_rows(x, s_x)
+        xd = fm.nvfp4_dequantize_rows(xc, xs, s_x)
+    else:
+        xc, xs = fm.mxfp8_quantize_rows(x)
+        xd = fm.mxfp8_dequantize_rows(xc, xs)
+    q = experts[0]
+    deq = {}
+    for m, (c, s, ts) in q.items():
+        deq[m] = (fm.nvfp4_dequantize_rows(c, s, ts) if fmt == moe.NVFP4
+                  else fm.mxfp8_dequantize_rows(c, s))
+    g = xd @ deq["gate"].T
+    u = xd @ deq["up"].T
+    h = (g / (1.0 + np.exp(-g)) * u).astype(np.float32)
+    if fmt == moe.NVFP4:
+        hc, hs = fm.nvfp4_quantize_rows(h, s_h)
+        hd = fm.nvfp4_dequantize_rows(hc, hs, s_h)
+    else:
+        hc, hs = fm.mxfp8_quantize_rows(h)
+        hd = fm.mxfp8_dequantize_rows(hc, hs)
+    y = fm.bf16_round(hd @ deq["down"].T)
+    np.testing.assert_array_equal(res["y"], y)
+    np.testing.assert_array_equal(res["gate"][:16], g)
+    # and the quantized FFN is a close approximation of the float FFN
+    wg, wu, wd = raw[0]
+    gf = x.astype(np.float64) @ wg.T
+    uf = x.astype(np.float64) @ wu.T
+    yf = (gf / (1 + np.exp(-gf)) * uf) @ wd.T
+    rel = np.linalg.norm(res["y"] - yf) / np.linalg.norm(yf)
+    assert rel < (0.25 if fmt == moe.NVFP4 else 0.08), rel
+
+
+@pytest.mark.parametrize("fmt", [moe.NVFP4, moe.MXFP8])
+def test_layer_equals_per_token_loop(fmt):
+    """The permuted-matrix forward equals a token-by-token evaluation."""
+    x, lg, experts, _ = _small_case(fmt, T=24, E=5, k=2, seed=9)
+    s_x, s_h = np.float32(8 / 2688), np.float32(24 / 2688)
+    res = moe.forward(x, lg, experts, 2, fmt, s_x, s_h)
+    ref = moe.forward_tokens(x, lg, experts, 2, fmt, s_x, s_h)
+    np.testing.assert_array_equal(res["topk_ids"], ref["topk_ids"])
+    np.testing.assert_array_equal(res["topk_w"], ref["topk_w"])
+    np.testing.assert_allclose(res["y"], ref["y"], rtol=2 ** -7, atol=1e-6)
+    diff = np.mean(res["y"] != ref["y"])
+    assert diff < 0.02       # only float64 summation order differs, then bf16 rounding
+
+
+def test_swiglu_closed_form():
+    g = np.array([0.0, 1.0, -1.0, 10.0, -30.0])
+    u = np.array([2.0, 3.0, 1.0, 1.0, 1.0])
+    ref = np.array([0.0, 3.0 / (1 + math.exp(-1.0)), -1.0 / (1 + math.e), 10.0 / (1 + math.exp(-10.0)),
+                    -30.0 / (1 + math.exp(30.0))])
+    np.testing.assert_allclose(moe.swiglu(g, u), ref, rtol=1e-15)
