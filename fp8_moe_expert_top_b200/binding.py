@@ -1,0 +1,186 @@
+"""ctypes binding of libmoe_b200.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and takes
+PyTorch tensors where the C ABI takes device pointers; it passes their
+data_ptr() and the current CUDA stream, and raises MoeError on a non-OK
+status.  All arithmetic of the layer runs in the library's CUDA kernels;
+there is no fallback: if the shared library is missing, every call raises.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_NVFP4 = 0
+MOE_MXFP8 = 1
+FORMATS = {"nvfp4": MOE_NVFP4, "mxfp8": MOE_MXFP8}
+
+MOE_DEVICE_TIMEOUT_PRODUCER = 0x1
+MOE_DEVICE_TIMEOUT_MMA = 0x2
+MOE_DEVICE_TIMEOUT_EPILOGUE = 0x4
+
+
+class MoeError(RuntimeError):
+    def __init__(self, name, status, msg):
+        super().__init__(f"{name} failed: status {status} ({msg})")
+        self.status = status
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32), ("d_model", ctypes.c_int32),
+                ("d_ffn", ctypes.c_int32), ("fmt", ctypes.c_int32)]
+
+
+class moe_weights_layout(ctypes.Structure):
+    _fields_ = [("w13_codes", ctypes.c_int64), ("w13_sf", ctypes.c_int64), ("w2_codes", ctypes.c_int64),
+                ("w2_sf", ctypes.c_int64), ("scales", ctypes.c_int64), ("total_bytes", ctypes.c_int64)]
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_CFG = ctypes.POINTER(moe_config)
+
+# name -> (restype, argtypes)
+SIGNATURES = {
+    "moe_check_config": (ctypes.c_int, [_CFG]),
+    "moe_get_weights_layout": (ctypes.c_int, [_CFG, ctypes.POINTER(moe_weights_layout)]),
+    "moe_max_rows": (_I64, [_CFG, _I64]),
+    "moe_codes_bytes": (_I64, [_CFG, _I64, _I64]),
+    "moe_sf_bytes": (_I64, [_CFG, _I64, _I64]),
+    "moe_sf_offset": (_I64, [_I64, _I64, _I64]),
+    "moe_route_workspace_bytes": (_I64, [_CFG, _I64]),
+    "moe_quantize_weights": (ctypes.c_int, [_CFG, _I32, _I32, _P, _P, _P, _P, _P]),
+    "moe_route_topk": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P]),
+    "moe_permute": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P]),
+    "moe_forward": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_forward_gateup": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_forward_down": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_unpermute_combine": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P]),
+    "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+}
+
+_lib = None
+
+
+def lib():
+    """Load libmoe_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m fp8_moe_expert_top_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def make_config(num_experts, top_k, d_model, d_ffn, fmt):
+    if isinstance(fmt, str):
+        fmt = FORMATS[fmt]
+    return moe_config(int(num_experts), int(top_k), int(d_model), int(d_ffn), int(fmt))
+
+
+def _p(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(name, status):
+    if status != 0:
+        raise MoeError(name, status, lib().moe_status_string(status).decode())
+
+
+# ----------------------------------------------------------------- sizes
+
+def moe_check_config(cfg):
+    return lib().moe_check_config(ctypes.byref(cfg))
+
+
+def moe_get_weights_layout(cfg):
+    out = moe_weights_layout()
+    _check("moe_get_weights_layout", lib().moe_get_weights_layout(ctypes.byref(cfg), ctypes.byref(out)))
+    return out
+
+
+def moe_max_rows(cfg, T):
+    return lib().moe_max_rows(ctypes.byref(cfg), int(T))
+
+
+def moe_codes_bytes(cfg, rows, K):
+    return lib().moe_codes_bytes(ctypes.byref(cfg), int(rows), int(K))
+
+
+def moe_sf_bytes(cfg, rows, K):
+    return lib().moe_sf_bytes(ctypes.byref(cfg), int(rows), int(K))
+
+
+def moe_sf_offset(row, col, nsf):
+    return lib().moe_sf_offset(int(row), int(col), int(nsf))
+
+
+def moe_route_workspace_bytes(cfg, T):
+    return lib().moe_route_workspace_bytes(ctypes.byref(cfg), int(T))
+
+
+# ----------------------------------------------------------------- calls
+
+def moe_quantize_weights(cfg, expert_begin, expert_count, w_gate, w_up, w_down, packed, stream=None):
+    _check("moe_quantize_weights", lib().moe_quantize_weights(
+        ctypes.byref(cfg), int(expert_begin), int(expert_count), _p(w_gate), _p(w_up), _p(w_down), _p(packed),
+        _stream(stream)))
+
+
+def moe_route_topk(cfg, T, logits, topk_ids, topk_w, expert_counts, expert_offsets, sorted_slots, slot_to_row,
+                   workspace, stream=None):
+    _check("moe_route_topk", lib().moe_route_topk(
+        ctypes.byref(cfg), int(T), _p(logits), _p(topk_ids), _p(topk_w), _p(expert_counts), _p(expert_offsets),
+        _p(sorted_slots), _p(slot_to_row), _p(workspace), int(workspace.numel() * workspace.element_size()),
+        _stream(stream)))
+
+
+def moe_permute(cfg, T, x, act_scale, slot_to_row, a_codes, a_sf, stream=None):
+    _check("moe_permute", lib().moe_permute(
+        ctypes.byref(cfg), int(T), _p(x), _p(act_scale), _p(slot_to_row), _p(a_codes), _p(a_sf), _stream(stream)))
+
+
+def moe_forward(cfg, T, packed, a_codes, a_sf, act_scale, inter_scale, expert_offsets, expert_counts, h_codes, h_sf,
+                down_out, gateup_debug=None, status_word=None, stream=None):
+    _check("moe_forward", lib().moe_forward(
+        ctypes.byref(cfg), int(T), _p(packed), _p(a_codes), _p(a_sf), _p(act_scale), _p(inter_scale),
+        _p(expert_offsets), _p(expert_counts), _p(h_codes), _p(h_sf), _p(down_out), _p(gateup_debug),
+        _p(status_word), _stream(stream)))
+
+
+def moe_forward_gateup(cfg, T, packed, a_codes, a_sf, act_scale, inter_scale, expert_offsets, expert_counts,
+                       h_codes, h_sf, gateup_debug=None, status_word=None, stream=None):
+    _check("moe_forward_gateup", lib().moe_forward_gateup(
+        ctypes.byref(cfg), int(T), _p(packed), _p(a_codes), _p(a_sf), _p(act_scale), _p(inter_scale),
+        _p(expert_offsets), _p(expert_counts), _p(h_codes), _p(h_sf), _p(gateup_debug), _p(status_word),
+        _stream(stream)))
+
+
+def moe_forward_down(cfg, T, packed, h_codes, h_sf, inter_scale, expert_offsets, expert_counts, down_out,
+                     status_word=None, stream=None):
+    _check("moe_forward_down", lib().moe_forward_down(
+        ctypes.byref(cfg), int(T), _p(packed), _p(h_codes), _p(h_sf), _p(inter_scale), _p(expert_offsets),
+        _p(expert_counts), _p(down_out), _p(status_word), _stream(stream)))
+
+
+def moe_unpermute_combine(cfg, T, down_out, topk_w, slot_to_row, y, stream=None):
+    _check("moe_unpermute_combine", lib().moe_unpermute_combine(
+        ctypes.byref(cfg), int(T), _p(down_out), _p(topk_w), _p(slot_to_row), _p(y), _stream(stream)))

@@ -1,0 +1,436 @@
+// Persistent grouped block-scaled GEMMs of the expert FFN on tcgen05.
+//
+// Page "Thinking Machines releases Inkling 2 Small weights under Apache
+// 2.0", section "NVFP4 and MXFP8 experts": every token is processed by 8 of
+// 384 experts whose weights are NVFP4 (E2M1 with E4M3 block scales) or MXFP8
+// (E4M3 with E8M0 block scales), and the activations are quantized to that
+// format inside the kernel that produces them.  The gate/up GEMM therefore
+// ends in an epilogue that applies SwiGLU and requantizes h in registers
+// (NVFP4 with the 4-vs-6 pick of the section TL;DR), and the down GEMM reads
+// those codes directly.
+//
+// Tiling: a tile is 128 permuted rows (one expert's segment is a whole
+// number of 128-row blocks) x BN = 256 rows of that expert's weight matrix,
+// with K streamed in steps of 128 bytes per row (256 NVFP4 or 128 MXFP8
+// elements).  One CTA per SM walks the tile list (row block fastest-varying
+// over N tiles, so the tiles sharing an activation block run together and
+// the weight tiles of one expert are reused from L2 across its row blocks).
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: codes via 2-D tensor maps (128-byte swizzle),
+//               block scales via 1-D bulk copies, into a 4-stage ring
+//   warp 1      MMA issuer: TMEM allocation, scale atoms SMEM->TMEM with
+//               tcgen05.cp, tcgen05.mma block-scaled M=128 N=256, commits
+//   warps 2-5   epilogue: tcgen05.ld of the 128x256 fp32 accumulator, tensor
+//               scales, SwiGLU + requantization (gate/up) or bf16 store (down)
+// Every mbarrier wait is bounded; a wait that runs out raises a CTA-wide
+// abort flag, every role stops issuing, TMEM is freed and a status bit is
+// set.
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "quant.cuh"
+
+namespace moe {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kStages = 4;
+constexpr int kRowBytesPerStage = 128;  // K bytes of one row per stage
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+
+template <int FMT>
+struct GemmTraits {
+  static constexpr int kElemsPerStage = (FMT == MOE_NVFP4) ? 256 : 128;
+  static constexpr int kMmaK = (FMT == MOE_NVFP4) ? 64 : 32;
+  static constexpr int kSfVec = (FMT == MOE_NVFP4) ? 16 : 32;
+  // scale bytes of 128 rows for one stage: NVFP4 16 scales/row = 4 atoms,
+  // MXFP8 4 scales/row = 1 atom
+  static constexpr int kSfBytes128 = 128 * (kElemsPerStage / kSfVec);
+  static constexpr int kABytes = kBM * kRowBytesPerStage;
+  static constexpr int kBBytes = kBN * kRowBytesPerStage;
+  static constexpr int kSfaOff = kABytes + kBBytes;
+  static constexpr int kSfbOff = kSfaOff + kSfBytes128;
+  static constexpr int kStageRaw = kSfbOff + (kBN / 128) * kSfBytes128;
+  static constexpr int kStageBytes = (kStageRaw + 1023) / 1024 * 1024;
+  // TMEM columns: accumulator [0, kBN), scales of A, then scales of B
+  static constexpr int kTmemSfa = kBN;
+  static constexpr int kSfaCols = (FMT == MOE_NVFP4) ? 16 : 4;
+  static constexpr int kTmemSfb = kTmemSfa + kSfaCols;
+};
+
+struct GemmArgs {
+  const uint8_t* a_sf;
+  const uint8_t* b_sf;
+  const int32_t* offsets;
+  const int32_t* counts;
+  const float* a_scale;
+  const float* w_scales;
+  const float* h_scale;
+  uint8_t* h_codes;
+  uint8_t* h_sf;
+  float* dbg;
+  __nv_bfloat16* out;
+  uint32_t* status;
+  int E;
+  int K;            // reduction length in elements
+  int n_rows_b;     // weight rows per expert (2I for gate/up, H for down)
+  int64_t sf_rb_stride;       // scale bytes of one 128-row block (= K / sfvec * 128)
+  int64_t b_sf_expert_stride; // scale bytes of one expert's weight matrix
+};
+
+__device__ __forceinline__ int find_expert(const int32_t* offs, int E, int row) {
+  int lo = 0, hi = E;  // offs[lo] <= row < offs[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (offs[mid] <= row) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+template <int FMT, bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                    const GemmArgs args) {
+  using Tr = GemmTraits<FMT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kStages * Tr::kStageBytes);
+  uint64_t* empty_bar = full_bar + kStages;
+  uint64_t* tfull_bar = empty_bar + kStages;
+  uint64_t* tempty_bar = tfull_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* s_offsets = reinterpret_cast<int32_t*>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = args.E;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(tfull_bar, 1);
+    mbar_init(tempty_bar, 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&tmap_a);
+    prefetch_tensormap(&tmap_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i <= E; i += kThreads) s_offsets[i] = args.offsets[i];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int m_tiles = s_offsets[E] / kBM;
+  const int n_tiles = args.n_rows_b / kBN;
+  const int total = m_tiles * n_tiles;
+  const int k_tiles = (args.K + Tr::kElemsPerStage - 1) / Tr::kElemsPerStage;
+  uint32_t fail_bits = 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_a = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        const int mt = tile / n_tiles, nt = tile % n_tiles;
+        const int e = find_expert(s_offsets, E, mt * kBM);
+        const uint8_t* a_sf = args.a_sf + static_cast<int64_t>(mt) * args.sf_rb_stride;
+        const uint8_t* b_sf = args.b_sf + static_cast<int64_t>(e) * args.b_sf_expert_stride +
+                              static_cast<int64_t>(nt) * (kBN / 128) * args.sf_rb_stride;
+        const int b_row = e * args.n_rows_b + nt * kBN;
+        for (int kt = 0; kt < k_tiles; ++kt) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+            fail_bits |= MOE_DEVICE_TIMEOUT_PRODUCER;
+            break;
+          }
+          const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
+          const uint32_t sf_bytes = (FMT == MOE_NVFP4) ? 512u * kb_here : 512u;
+          uint8_t* st = smem + stage * Tr::kStageBytes;
+          mbar_arrive_expect_tx(&full_bar[stage], Tr::kABytes + Tr::kBBytes + sf_bytes * (1 + kBN / 128));
+          tma_load_2d(st, &tmap_a, kt * kRowBytesPerStage, mt * kBM, &full_bar[stage], pol_a);
+          tma_load_2d(st + Tr::kABytes, &tmap_b, kt * kRowBytesPerStage, b_row, &full_bar[stage], pol_w);
+          bulk_load(st + Tr::kSfaOff, a_sf + kt * Tr::kSfBytes128, sf_bytes, &full_bar[stage], pol_a);
+#pragma unroll
+          for (int h = 0; h < kBN / 128; ++h)
+            bulk_load(st + Tr::kSfbOff + h * Tr::kSfBytes128, b_sf + h * args.sf_rb_stride + kt * Tr::kSfBytes128,
+                      sf_bytes, &full_bar[stage], pol_w);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      const uint32_t d_tmem = tmem_base;
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        if (!mbar_wait(tempty_bar, acc_phase ^ 1u, abort_flag)) {
+          fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
+          break;
+        }
+        tc_fence_after();
+        bool ok = true;
+        for (int kt = 0; kt < k_tiles; ++kt) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+            fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
+          const uint32_t st = smem_u32(smem + stage * Tr::kStageBytes);
+          const uint64_t adesc = make_desc_sw128(st);
+          const uint64_t bdesc = make_desc_sw128(st + Tr::kABytes);
+          if (FMT == MOE_NVFP4) {
+            for (int kb = 0; kb < kb_here; ++kb) {
+              tc_cp_sf_atom(tmem_base + Tr::kTmemSfa + 4 * kb, make_desc_sf(st + Tr::kSfaOff + 512 * kb));
+#pragma unroll
+              for (int h = 0; h < kBN / 128; ++h)
+                tc_cp_sf_atom(tmem_base + Tr::kTmemSfb + (kBN / 32) * kb + 4 * h,
+                              make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
+            }
+            for (int kb = 0; kb < kb_here; ++kb) {
+              tc_mma_nvfp4(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_nvfp4(kBN),
+                           tmem_base + Tr::kTmemSfa + 4 * kb, tmem_base + Tr::kTmemSfb + (kBN / 32) * kb,
+                           (kt | kb) != 0 ? 1u : 0u);
+            }
+          } else {
+            tc_cp_sf_atom(tmem_base + Tr::kTmemSfa, make_desc_sf(st + Tr::kSfaOff));
+#pragma unroll
+            for (int h = 0; h < kBN / 128; ++h)
+              tc_cp_sf_atom(tmem_base + Tr::kTmemSfb + 4 * h, make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128));
+            for (int kb = 0; kb < kb_here; ++kb) {
+              const uint32_t sel = static_cast<uint32_t>(kb) << 30;
+              tc_mma_mxfp8(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_mxfp8(kBN, kb),
+                           (tmem_base + Tr::kTmemSfa) | sel, (tmem_base + Tr::kTmemSfb) | sel,
+                           (kt | kb) != 0 ? 1u : 0u);
+            }
+          }
+          tc_commit(&empty_bar[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar);
+        acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_l = q * 32 + lane;
+    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    uint32_t acc_phase = 0;
+    const int I = args.n_rows_b / 2;  // gate/up: channels; unused for down
+    const int H = args.n_rows_b;      // down: output channels
+    for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+      const int mt = tile / n_tiles, nt = tile % n_tiles;
+      const int e = find_expert(s_offsets, E, mt * kBM);
+      const int valid_rows = s_offsets[e] + __ldg(args.counts + e) - mt * kBM;
+      const bool valid = row_l < valid_rows;
+      const int64_t row = static_cast<int64_t>(mt) * kBM + row_l;
+      if (!mbar_wait(tfull_bar, acc_phase, abort_flag)) {
+        fail_bits |= MOE_DEVICE_TIMEOUT_EPILOGUE;
+        break;
+      }
+      tc_fence_after();
+      if (GATEUP) {
+        const float sa = (FMT == MOE_NVFP4) ? __ldg(args.a_scale) : 1.0f;
+        const float sg = (FMT == MOE_NVFP4) ? __fmul_rn(sa, __ldg(args.w_scales + 3 * e + 0)) : 1.0f;
+        const float su = (FMT == MOE_NVFP4) ? __fmul_rn(sa, __ldg(args.w_scales + 3 * e + 1)) : 1.0f;
+        const float sh = (FMT == MOE_NVFP4) ? __ldg(args.h_scale) : 1.0f;
+#pragma unroll 1
+        for (int j = 0; j < kBN / 64; ++j) {
+          float g[32], u[32];
+          tmem_ld32(t_row + 64 * j, g);
+          tmem_ld32(t_row + 64 * j + 32, u);
+          tmem_ld_wait();
+          if (valid) {
+            const int ch0 = nt * (kBN / 2) + 32 * j;
+            float h[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float gv = g[i] * sg;
+              const float uv = u[i] * su;
+              g[i] = gv;
+              u[i] = uv;
+              h[i] = gv * uv / (1.0f + expf(-gv));
+            }
+            if (args.dbg != nullptr) {
+              float4* dg = reinterpret_cast<float4*>(args.dbg + row * (2 * I) + ch0);
+              float4* du = reinterpret_cast<float4*>(args.dbg + row * (2 * I) + I + ch0);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                dg[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
+                du[i] = make_float4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
+              }
+            }
+            if (FMT == MOE_NVFP4) {
+              const Nvfp4Block b0 = nvfp4_quantize16(h, sh);
+              const Nvfp4Block b1 = nvfp4_quantize16(h + 16, sh);
+              *reinterpret_cast<uint4*>(args.h_codes + row * (I / 2) + ch0 / 2) =
+                  make_uint4(static_cast<uint32_t>(b0.codes), static_cast<uint32_t>(b0.codes >> 32),
+                             static_cast<uint32_t>(b1.codes), static_cast<uint32_t>(b1.codes >> 32));
+              *reinterpret_cast<uint16_t*>(args.h_sf + sf_offset(row, ch0 / 16, I / 16)) =
+                  static_cast<uint16_t>(b0.sf | (b1.sf << 8));
+            } else {
+              uint32_t w[8];
+              const uint32_t ex = mxfp8_quantize32(h, w);
+              uint4* dst = reinterpret_cast<uint4*>(args.h_codes + row * I + ch0);
+              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              args.h_sf[sf_offset(row, ch0 / 32, I / 32)] = static_cast<uint8_t>(ex);
+            }
+          }
+        }
+      } else {
+        const float s = (FMT == MOE_NVFP4) ? __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scales + 3 * e + 2)) : 1.0f;
+#pragma unroll 1
+        for (int j = 0; j < kBN / 32; ++j) {
+          float v[32];
+          tmem_ld32(t_row + 32 * j, v);
+          tmem_ld_wait();
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(args.out + row * H + nt * kBN + 32 * j);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint32_t p[4];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * i + 2 * c] * s, v[8 * i + 2 * c + 1] * s);
+                p[c] = *reinterpret_cast<const uint32_t*>(&b);
+              }
+              dst[i] = make_uint4(p[0], p[1], p[2], p[3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar);
+      acc_phase ^= 1u;
+    }
+  }
+
+  if (fail_bits != 0u && args.status != nullptr) atomicOr(args.status, fail_bits);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a [rows][row_bytes] byte matrix, box 128 bytes x box_rows,
+// 128-byte swizzle; columns past row_bytes read as zero.
+static bool make_map(CUtensorMap* map, const void* base, int64_t row_bytes, int64_t rows, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int FMT, bool GATEUP>
+static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& a, cudaStream_t stream) {
+  using Tr = GemmTraits<FMT>;
+  const size_t smem = 1024 + kStages * Tr::kStageBytes + (2 * kStages + 2) * 8 + 16 + (a.E + 1) * 4;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  static int configured[64] = {0};
+  if (dev >= 64 || !configured[dev]) {
+    // the largest size any supported E needs (E <= 1024)
+    const size_t smem_max = 1024 + kStages * Tr::kStageBytes + (2 * kStages + 2) * 8 + 16 + 1025 * 4;
+    err = cudaFuncSetAttribute(moe_gemm_kernel<FMT, GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_max));
+    if (err != cudaSuccess) return err;
+    if (dev < 64) configured[dev] = 1;
+  }
+  int sms = 0;
+  err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (err != cudaSuccess) return err;
+  moe_gemm_kernel<FMT, GATEUP><<<sms, kThreads, smem, stream>>>(ma, mb, a);
+  return cudaGetLastError();
+}
+
+size_t gemm_smem_bytes(int fmt, int E) {
+  const int sb = (fmt == MOE_NVFP4) ? GemmTraits<MOE_NVFP4>::kStageBytes : GemmTraits<MOE_MXFP8>::kStageBytes;
+  return 1024 + kStages * sb + (2 * kStages + 2) * 8 + 16 + (E + 1) * 4;
+}
+
+cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
+  const int bits = (g.fmt == MOE_NVFP4) ? 4 : 8;
+  const int sfvec = (g.fmt == MOE_NVFP4) ? 16 : 32;
+  const int64_t row_bytes = static_cast<int64_t>(g.K) * bits / 8;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, g.a_codes, row_bytes, g.R_max, kBM)) return cudaErrorInvalidValue;
+  if (!make_map(&mb, g.b_codes, row_bytes, static_cast<int64_t>(g.E) * g.n_rows_b, kBN)) return cudaErrorInvalidValue;
+  GemmArgs a;
+  a.a_sf = g.a_sf;
+  a.b_sf = g.b_sf;
+  a.offsets = g.offsets;
+  a.counts = g.counts;
+  a.a_scale = g.a_scale;
+  a.w_scales = g.w_scales;
+  a.h_scale = g.h_scale;
+  a.h_codes = g.h_codes;
+  a.h_sf = g.h_sf;
+  a.dbg = g.dbg;
+  a.out = static_cast<__nv_bfloat16*>(g.out);
+  a.status = g.status;
+  a.E = g.E;
+  a.K = g.K;
+  a.n_rows_b = g.n_rows_b;
+  a.sf_rb_stride = static_cast<int64_t>(g.K / sfvec) * 128;
+  a.b_sf_expert_stride = static_cast<int64_t>(g.n_rows_b) * (g.K / sfvec);
+  if (g.fmt == MOE_NVFP4)
+    return g.gateup ? launch_one<MOE_NVFP4, true>(ma, mb, a, stream) : launch_one<MOE_NVFP4, false>(ma, mb, a, stream);
+  return g.gateup ? launch_one<MOE_MXFP8, true>(ma, mb, a, stream) : launch_one<MOE_MXFP8, false>(ma, mb, a, stream);
+}
+
+}  // namespace moe

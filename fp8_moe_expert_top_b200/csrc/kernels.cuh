@@ -1,0 +1,48 @@
+// Host-side launchers of the library's kernels (internal).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+int64_t route_workspace_bytes(int E, int64_t T);
+cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w,
+                         int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
+                         int32_t* slot_to_row, int64_t R_max, void* workspace, cudaStream_t stream);
+
+cudaError_t launch_permute(int fmt, int T, int H, int k, const void* x, const float* act_scale,
+                           const int32_t* slot_to_row, uint8_t* a_codes, uint8_t* a_sf, cudaStream_t stream);
+
+cudaError_t launch_combine(int T, int H, int k, const void* down_out, const float* topk_w,
+                           const int32_t* slot_to_row, void* y, cudaStream_t stream);
+
+cudaError_t launch_quantize_weights(int fmt, int E, int H, int I, int expert_begin, int expert_count,
+                                    const float* w_gate, const float* w_up, const float* w_down, uint8_t* w13_codes,
+                                    uint8_t* w13_sf, uint8_t* w2_codes, uint8_t* w2_sf, float* scales,
+                                    cudaStream_t stream);
+
+struct GemmLaunch {
+  int fmt;
+  bool gateup;
+  int E, K, n_rows_b;     // K in elements, rows of B per expert (2I or H)
+  int64_t R_max;
+  const uint8_t* a_codes;
+  const uint8_t* a_sf;
+  const uint8_t* b_codes;
+  const uint8_t* b_sf;
+  const int32_t* offsets;
+  const int32_t* counts;
+  const float* a_scale;   // device scalar or null (MXFP8)
+  const float* w_scales;  // [E][3]
+  const float* h_scale;   // gate/up: tensor scale of h (NVFP4) or null
+  uint8_t* h_codes;
+  uint8_t* h_sf;
+  float* dbg;
+  void* out;              // down: bf16 [R_max][H]
+  uint32_t* status;
+};
+cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,150 @@
+// Permute-gather with fused activation quantization, and the weighted
+// un-permute / combine.
+//
+// Page "Thinking Machines releases Inkling 2 Small weights under Apache 2.0",
+// section "NVFP4 and MXFP8 experts": expert activations are quantized to the
+// layer's weight format inside the kernel that produces them, with no
+// separate quantization pass.  Here the producer of the GEMM1 operand is the
+// permute-gather: each token row is read once, quantized once (NVFP4 4-vs-6
+// or MXFP8) and written to each of its k expert rows.
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "quant.cuh"
+
+namespace moe {
+
+// 64 bf16 -> float
+__device__ __forceinline__ void load64_bf16(const __nv_bfloat16* p, float* f) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 u = __ldg(q + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+      f[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  }
+}
+
+// One warp per token; lane g handles 64-element groups g, g+32, ...
+template <int FMT>
+__global__ void __launch_bounds__(128) permute_kernel(int T, int H, int k, const __nv_bfloat16* __restrict__ x,
+                                                      const float* __restrict__ act_scale,
+                                                      const int32_t* __restrict__ slot_to_row,
+                                                      uint8_t* __restrict__ a_codes, uint8_t* __restrict__ a_sf) {
+  const int t = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const int groups = H / 64;
+  const float s_x = (FMT == MOE_NVFP4) ? __ldg(act_scale) : 1.0f;
+  int32_t rows[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) rows[j] = (j < k) ? __ldg(slot_to_row + static_cast<int64_t>(t) * k + j) : 0;
+  for (int g = lane; g < groups; g += 32) {
+    float f[64];
+    load64_bf16(x + static_cast<int64_t>(t) * H + 64 * g, f);
+    if (FMT == MOE_NVFP4) {
+      uint64_t c[4];
+      uint32_t sfw = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const Nvfp4Block q = nvfp4_quantize16(f + 16 * b, s_x);
+        c[b] = q.codes;
+        sfw |= q.sf << (8 * b);
+      }
+      const int64_t nsf = H / 16;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j >= k) break;
+        const int64_t r = rows[j];
+        uint4* dst = reinterpret_cast<uint4*>(a_codes + r * (H / 2) + 32 * g);
+        dst[0] = make_uint4(static_cast<uint32_t>(c[0]), static_cast<uint32_t>(c[0] >> 32),
+                            static_cast<uint32_t>(c[1]), static_cast<uint32_t>(c[1] >> 32));
+        dst[1] = make_uint4(static_cast<uint32_t>(c[2]), static_cast<uint32_t>(c[2] >> 32),
+                            static_cast<uint32_t>(c[3]), static_cast<uint32_t>(c[3] >> 32));
+        *reinterpret_cast<uint32_t*>(a_sf + sf_offset(r, 4 * g, nsf)) = sfw;
+      }
+    } else {
+      uint32_t w[16];
+      const uint32_t e0 = mxfp8_quantize32(f, w);
+      const uint32_t e1 = mxfp8_quantize32(f + 32, w + 8);
+      const int64_t nsf = H / 32;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j >= k) break;
+        const int64_t r = rows[j];
+        uint4* dst = reinterpret_cast<uint4*>(a_codes + r * H + 64 * g);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        *reinterpret_cast<uint16_t*>(a_sf + sf_offset(r, 2 * g, nsf)) = static_cast<uint16_t>(e0 | (e1 << 8));
+      }
+    }
+  }
+}
+
+cudaError_t launch_permute(int fmt, int T, int H, int k, const void* x, const float* act_scale,
+                           const int32_t* slot_to_row, uint8_t* a_codes, uint8_t* a_sf, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const dim3 grid((T + 3) / 4), block(128);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (fmt == MOE_NVFP4)
+    permute_kernel<MOE_NVFP4><<<grid, block, 0, stream>>>(T, H, k, xb, act_scale, slot_to_row, a_codes, a_sf);
+  else
+    permute_kernel<MOE_MXFP8><<<grid, block, 0, stream>>>(T, H, k, xb, act_scale, slot_to_row, a_codes, a_sf);
+  return cudaGetLastError();
+}
+
+// y[t] = sum_j w[t][j] * out[row(t, j)], float32 in rank order, then bf16.
+// One CTA per token; each thread owns 8 consecutive channels per step.
+__global__ void __launch_bounds__(256) combine_kernel(int H, int k, const __nv_bfloat16* __restrict__ down_out,
+                                                      const float* __restrict__ topk_w,
+                                                      const int32_t* __restrict__ slot_to_row,
+                                                      __nv_bfloat16* __restrict__ y) {
+  const int t = blockIdx.x;
+  float w[8];
+  int64_t rows[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    w[j] = (j < k) ? __ldg(topk_w + static_cast<int64_t>(t) * k + j) : 0.0f;
+    rows[j] = (j < k) ? __ldg(slot_to_row + static_cast<int64_t>(t) * k + j) : 0;
+  }
+  for (int c8 = threadIdx.x; c8 < H / 8; c8 += blockDim.x) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) break;
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(down_out + rows[j] * H) + c8);
+      const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(w[j], __uint_as_float(q[i] << 16)));
+        acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(w[j], __uint_as_float(q[i] & 0xFFFF0000u)));
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+      o[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    reinterpret_cast<uint4*>(y + static_cast<int64_t>(t) * H)[c8] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+cudaError_t launch_combine(int T, int H, int k, const void* down_out, const float* topk_w,
+                           const int32_t* slot_to_row, void* y, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  combine_kernel<<<T, 256, 0, stream>>>(H, k, static_cast<const __nv_bfloat16*>(down_out), topk_w, slot_to_row,
+                                        static_cast<__nv_bfloat16*>(y));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

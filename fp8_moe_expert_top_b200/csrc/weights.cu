@@ -1,0 +1,169 @@
+// Offline expert-weight quantization into the GEMM-ready packed layout.
+//
+// Pages: "thinkingmachines/Inkling-2-Small", section Overview (NVFP4 experts
+// in layers 0-39, MXFP8 in layers 40-47) and "Thinking Machines releases
+// Inkling 2 Small weights under Apache 2.0", section TL;DR (the 4-vs-6 block
+// scale pick of the NVFP4 quantizer).  NVFP4 tensor scale per (expert,
+// matrix): amax / 2688 (2688 = 6 * 448), 1 for an all-zero matrix.
+//
+// Four steps on the stream: zero the amax slots, reduce amax per matrix
+// (atomicMax on the float bits, exact and order-independent for values >= 0),
+// quantize every 64-element group, turn amax into the tensor scale.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "quant.cuh"
+
+namespace moe {
+
+// blockIdx.y = matrix (0 gate, 1 up, 2 down), blockIdx.z = expert in the slice
+__global__ void __launch_bounds__(256) weight_amax_kernel(int64_t n_per_matrix, const float* __restrict__ w_gate,
+                                                          const float* __restrict__ w_up,
+                                                          const float* __restrict__ w_down,
+                                                          float* __restrict__ amax_out) {
+  const int m = blockIdx.y, e = blockIdx.z;
+  const float* w = (m == 0 ? w_gate : (m == 1 ? w_up : w_down)) + static_cast<int64_t>(e) * n_per_matrix;
+  float a = 0.0f;
+  const int64_t n4 = n_per_matrix / 4;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(w) + i);
+    a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+  __shared__ float red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
+    atomicMax(reinterpret_cast<unsigned int*>(amax_out + e * 3 + m), __float_as_uint(a));
+  }
+}
+
+// One thread per 64-element group of one row.
+template <int FMT>
+__global__ void __launch_bounds__(256) weight_quant_kernel(int H, int I, const float* __restrict__ w_gate,
+                                                           const float* __restrict__ w_up,
+                                                           const float* __restrict__ w_down,
+                                                           const float* __restrict__ amax, uint8_t* __restrict__ w13_codes,
+                                                           uint8_t* __restrict__ w13_sf,
+                                                           uint8_t* __restrict__ w2_codes,
+                                                           uint8_t* __restrict__ w2_sf) {
+  const int m = blockIdx.y, e = blockIdx.z;  // e: index inside the slice (pointers are already offset)
+  const int64_t n_per_matrix = static_cast<int64_t>(I) * H;
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gid >= n_per_matrix / 64) return;
+  const int K = (m == 2) ? I : H;
+  const int G = K / 64;
+  const int64_t src_row = gid / G;
+  const int g = static_cast<int>(gid % G);
+  const float* src = (m == 0 ? w_gate : (m == 1 ? w_up : w_down)) + static_cast<int64_t>(e) * n_per_matrix +
+                     src_row * K + 64 * g;
+  float f[64];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(src) + i);
+    f[4 * i] = v.x;
+    f[4 * i + 1] = v.y;
+    f[4 * i + 2] = v.z;
+    f[4 * i + 3] = v.w;
+  }
+  // destination row: gate/up interleaved in groups of 32 rows inside w13
+  int64_t dst_row;
+  uint8_t *codes, *sfbuf;
+  int64_t rows_per_expert;
+  if (m == 2) {
+    dst_row = src_row;
+    rows_per_expert = H;
+    codes = w2_codes;
+    sfbuf = w2_sf;
+  } else {
+    dst_row = 64 * (src_row / 32) + (m == 1 ? 32 : 0) + (src_row % 32);
+    rows_per_expert = 2 * static_cast<int64_t>(I);
+    codes = w13_codes;
+    sfbuf = w13_sf;
+  }
+  if (FMT == MOE_NVFP4) {
+    const float a = amax[e * 3 + m];
+    const float s_g = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);
+    uint64_t c[4];
+    uint32_t sfw = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const Nvfp4Block q = nvfp4_quantize16(f + 16 * b, s_g);
+      c[b] = q.codes;
+      sfw |= q.sf << (8 * b);
+    }
+    const int64_t row_bytes = K / 2;
+    uint8_t* dst = codes + (static_cast<int64_t>(e) * rows_per_expert + dst_row) * row_bytes + 32 * g;
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(static_cast<uint32_t>(c[0]), static_cast<uint32_t>(c[0] >> 32),
+                                                  static_cast<uint32_t>(c[1]), static_cast<uint32_t>(c[1] >> 32));
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(static_cast<uint32_t>(c[2]), static_cast<uint32_t>(c[2] >> 32),
+                                                  static_cast<uint32_t>(c[3]), static_cast<uint32_t>(c[3] >> 32));
+    const int64_t nsf = K / 16;
+    uint8_t* sfe = sfbuf + static_cast<int64_t>(e) * rows_per_expert * nsf;
+    *reinterpret_cast<uint32_t*>(sfe + sf_offset(dst_row, 4 * g, nsf)) = sfw;
+  } else {
+    uint32_t w[16];
+    const uint32_t e0 = mxfp8_quantize32(f, w);
+    const uint32_t e1 = mxfp8_quantize32(f + 32, w + 8);
+    uint8_t* dst = codes + (static_cast<int64_t>(e) * rows_per_expert + dst_row) * K + 64 * g;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    const int64_t nsf = K / 32;
+    uint8_t* sfe = sfbuf + static_cast<int64_t>(e) * rows_per_expert * nsf;
+    *reinterpret_cast<uint16_t*>(sfe + sf_offset(dst_row, 2 * g, nsf)) = static_cast<uint16_t>(e0 | (e1 << 8));
+  }
+}
+
+__global__ void weight_scale_finalize_kernel(int n, int fmt, float* __restrict__ scales) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  if (fmt == MOE_NVFP4) {
+    const float a = scales[i];
+    scales[i] = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);
+  } else {
+    scales[i] = 1.0f;
+  }
+}
+
+cudaError_t launch_quantize_weights(int fmt, int E, int H, int I, int expert_begin, int expert_count,
+                                    const float* w_gate, const float* w_up, const float* w_down, uint8_t* w13_codes,
+                                    uint8_t* w13_sf, uint8_t* w2_codes, uint8_t* w2_sf, float* scales,
+                                    cudaStream_t stream) {
+  (void)E;
+  if (expert_count == 0) return cudaSuccess;
+  const int bits = (fmt == MOE_NVFP4) ? 4 : 8;
+  const int sfvec = (fmt == MOE_NVFP4) ? 16 : 32;
+  const int64_t rows13 = 2 * static_cast<int64_t>(I);
+  // offset every output by the slice start so the kernels index experts 0..count-1
+  uint8_t* c13 = w13_codes + static_cast<int64_t>(expert_begin) * rows13 * H * bits / 8;
+  uint8_t* s13 = w13_sf + static_cast<int64_t>(expert_begin) * rows13 * H / sfvec;
+  uint8_t* c2 = w2_codes + static_cast<int64_t>(expert_begin) * H * static_cast<int64_t>(I) * bits / 8;
+  uint8_t* s2 = w2_sf + static_cast<int64_t>(expert_begin) * H * static_cast<int64_t>(I) / sfvec;
+  float* sc = scales + static_cast<int64_t>(expert_begin) * 3;
+  cudaError_t err = cudaMemsetAsync(sc, 0, sizeof(float) * 3 * expert_count, stream);
+  if (err != cudaSuccess) return err;
+  const int64_t n = static_cast<int64_t>(I) * H;
+  if (fmt == MOE_NVFP4) {
+    const int bx = static_cast<int>((n / 4 + 255) / 256 < 512 ? (n / 4 + 255) / 256 : 512);
+    weight_amax_kernel<<<dim3(bx, 3, expert_count), 256, 0, stream>>>(n, w_gate, w_up, w_down, sc);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  const dim3 grid(static_cast<unsigned>((n / 64 + 255) / 256), 3, expert_count);
+  if (fmt == MOE_NVFP4)
+    weight_quant_kernel<MOE_NVFP4><<<grid, 256, 0, stream>>>(H, I, w_gate, w_up, w_down, sc, c13, s13, c2, s2);
+  else
+    weight_quant_kernel<MOE_MXFP8><<<grid, 256, 0, stream>>>(H, I, w_gate, w_up, w_down, sc, c13, s13, c2, s2);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  weight_scale_finalize_kernel<<<(3 * expert_count + 255) / 256, 256, 0, stream>>>(3 * expert_count, fmt, sc);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

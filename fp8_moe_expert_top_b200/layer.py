@@ -1,0 +1,103 @@
+"""ExpertLayer: device buffers plus the four calls of one routed-expert layer.
+
+This is the public Python entry point a user calls: it owns PyTorch-allocated
+device buffers sized for up to T_max tokens and runs, on the current stream,
+
+    moe_route_topk -> moe_permute -> moe_forward -> moe_unpermute_combine
+
+through the C ABI.  Nothing here computes any part of the layer.
+"""
+
+import torch
+
+from . import binding as B
+
+
+class ExpertLayer:
+    def __init__(self, num_experts, top_k, d_model, d_ffn, fmt, T_max, device, s_x=None, s_h=None,
+                 debug=False):
+        self.cfg = B.make_config(num_experts, top_k, d_model, d_ffn, fmt)
+        st = B.moe_check_config(self.cfg)
+        if st != 0:
+            raise B.MoeError("moe_check_config", st, B.lib().moe_status_string(st).decode())
+        self.E, self.k, self.H, self.I = num_experts, top_k, d_model, d_ffn
+        self.fmt = self.cfg.fmt
+        self.T_max = int(T_max)
+        self.device = torch.device(device)
+        dev = self.device
+        self.layout = B.moe_get_weights_layout(self.cfg)
+        self.packed = torch.empty(self.layout.total_bytes, dtype=torch.uint8, device=dev)
+        self.R_max = B.moe_max_rows(self.cfg, self.T_max)
+        R, T, k, E, H, I = self.R_max, self.T_max, top_k, num_experts, d_model, d_ffn
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.topk_ids = torch.empty(T, k, **i32)
+        self.topk_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+        self.expert_counts = torch.empty(E, **i32)
+        self.expert_offsets = torch.empty(E + 1, **i32)
+        self.sorted_slots = torch.empty(R, **i32)
+        self.slot_to_row = torch.empty(T * k, **i32)
+        self.route_ws = torch.empty(B.moe_route_workspace_bytes(self.cfg, T), dtype=torch.uint8, device=dev)
+        u8 = dict(dtype=torch.uint8, device=dev)
+        self.a_codes = torch.empty(B.moe_codes_bytes(self.cfg, R, H), **u8)
+        self.a_sf = torch.empty(B.moe_sf_bytes(self.cfg, R, H), **u8)
+        self.h_codes = torch.empty(B.moe_codes_bytes(self.cfg, R, I), **u8)
+        self.h_sf = torch.empty(B.moe_sf_bytes(self.cfg, R, I), **u8)
+        self.down_out = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        self.status = torch.zeros(1, **i32)
+        self.gateup_debug = torch.empty(R, 2 * I, dtype=torch.float32, device=dev) if debug else None
+        f32 = dict(dtype=torch.float32, device=dev)
+        if self.fmt == B.MOE_NVFP4:
+            if s_x is None or s_h is None:
+                raise ValueError("NVFP4 needs the static activation scales s_x and s_h")
+            self.act_scale = torch.tensor([float(s_x)], **f32)
+            self.inter_scale = torch.tensor([float(s_h)], **f32)
+        else:
+            self.act_scale = None
+            self.inter_scale = None
+
+    # ------------------------------------------------------------- weights
+    def quantize_experts(self, expert_begin, w_gate, w_up, w_down):
+        """Quantize float32 weights of experts [begin, begin + n) into self.packed."""
+        n = w_gate.shape[0]
+        for t in (w_gate, w_up, w_down):
+            assert t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+        B.moe_quantize_weights(self.cfg, expert_begin, n, w_gate, w_up, w_down, self.packed)
+
+    # ------------------------------------------------------------- steps
+    def route(self, logits, T):
+        B.moe_route_topk(self.cfg, T, logits, self.topk_ids, self.topk_w, self.expert_counts,
+                         self.expert_offsets, self.sorted_slots, self.slot_to_row, self.route_ws)
+
+    def permute(self, x, T):
+        B.moe_permute(self.cfg, T, x, self.act_scale, self.slot_to_row, self.a_codes, self.a_sf)
+
+    def experts(self, T):
+        B.moe_forward(self.cfg, T, self.packed, self.a_codes, self.a_sf, self.act_scale, self.inter_scale,
+                      self.expert_offsets, self.expert_counts, self.h_codes, self.h_sf, self.down_out,
+                      self.gateup_debug, self.status)
+
+    def gateup(self, T):
+        B.moe_forward_gateup(self.cfg, T, self.packed, self.a_codes, self.a_sf, self.act_scale, self.inter_scale,
+                             self.expert_offsets, self.expert_counts, self.h_codes, self.h_sf, self.gateup_debug,
+                             self.status)
+
+    def down(self, T):
+        B.moe_forward_down(self.cfg, T, self.packed, self.h_codes, self.h_sf, self.inter_scale,
+                           self.expert_offsets, self.expert_counts, self.down_out, self.status)
+
+    def combine(self, T):
+        B.moe_unpermute_combine(self.cfg, T, self.down_out, self.topk_w, self.slot_to_row, self.y)
+
+    def forward(self, x, logits):
+        """y[:T] for bf16 x [T, H] and float32 logits [T, E] already on the device."""
+        T = x.shape[0]
+        assert T <= self.T_max and logits.shape == (T, self.E)
+        assert x.dtype == torch.bfloat16 and logits.dtype == torch.float32
+        assert x.is_contiguous() and logits.is_contiguous()
+        self.route(logits, T)
+        self.permute(x, T)
+        self.gateup(T)
+        self.down(T)
+        self.combine(T)
+        return self.y[:T]

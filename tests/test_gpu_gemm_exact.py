@@ -1,0 +1,149 @@
+"""Integer-exact check of the tcgen05 block-scaled GEMMs (GPU).
+
+Codes are drawn from the E2M1 value grid {0, +-0.5, ..., +-6} (for MXFP8 the
+same values as E4M3 codes) and block scales from {0.5, 1, 2}; tensor scales
+are 1.  Every product is a multiple of 1/16 and every partial sum stays far
+below 2^24 / 16, so any summation order gives the exact result in float32:
+the kernel's gate/up output must equal the float64 product bit for bit, and
+its bf16 down output must equal the correctly rounded exact value.  This
+pins the operand layouts, the scale-atom layout, the nibble order and the
+gate/up interleave with no tolerance.  Padding rows carry random bytes,
+including NaN scale codes, and must not leak into valid rows.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from fp8_moe_expert_top_b200 import binding as B
+from oracle import formats as fm
+
+from helpers import encode_expert_into, pack_nvfp4, swizzle_sf, sfvec, w13_row
+
+GRID_E2M1 = np.array([0, 1, 2, 3, 4, 5, 6, 7, 9, 10, 11, 12, 13, 14, 15], dtype=np.uint8)   # no -0
+GRID_E4M3 = np.array([0x00, 0x30, 0x38, 0x3C, 0x40, 0x44, 0x48, 0x4C,
+                      0xB0, 0xB8, 0xBC, 0xC0, 0xC4, 0xC8, 0xCC], dtype=np.uint8)
+SF_E4M3 = np.array([0x30, 0x38, 0x40], dtype=np.uint8)       # 0.5, 1, 2
+SF_E8M0 = np.array([126, 127, 128], dtype=np.uint8)          # 0.5, 1, 2
+
+
+def rand_codes(rng, fmt, shape):
+    g = GRID_E2M1 if fmt == "nvfp4" else GRID_E4M3
+    return rng.choice(g, size=shape).astype(np.uint8)
+
+
+def rand_sf(rng, fmt, shape):
+    return rng.choice(SF_E4M3 if fmt == "nvfp4" else SF_E8M0, size=shape).astype(np.uint8)
+
+
+def decode(fmt, codes, sf):
+    v = sfvec(fmt)
+    rows, K = codes.shape
+    if fmt == "nvfp4":
+        val = fm.e2m1_decode(codes).reshape(rows, K // v, v) * fm.e4m3_decode(sf)[..., None]
+    else:
+        val = fm.e4m3_decode(codes).reshape(rows, K // v, v) * fm.e8m0_decode(sf)[..., None]
+    return val.reshape(rows, K)
+
+
+def to_rows_bytes(fmt, codes):
+    return pack_nvfp4(codes) if fmt == "nvfp4" else codes
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp8"])
+@pytest.mark.parametrize("H,I", [(256, 128), (512, 256), (1024, 384)])
+def test_gemm_integer_exact(cuda_device, fmt, H, I):
+    rng = np.random.default_rng(H * 7 + I + (1 if fmt == "mxfp8" else 0))
+    E, k = 4, 1
+    counts = np.array([130, 0, 5, 256], dtype=np.int32)
+    offsets = np.concatenate([[0], np.cumsum((counts + 127) // 128 * 128)]).astype(np.int32)
+    T = 391                                      # R_max(T) >= offsets[E] for k = 1
+    cfg = B.make_config(E, k, H, I, fmt)
+    R = B.moe_max_rows(cfg, T)
+    assert R >= offsets[-1]
+    v = sfvec(fmt)
+    dev = cuda_device
+
+    # weights written directly in the packed layout, tensor scales 1
+    layout = B.moe_get_weights_layout(cfg)
+    packed = np.zeros(layout.total_bytes, dtype=np.uint8)
+    W = {}
+    for e in range(E):
+        q = {}
+        for m, (rows, K) in (("gate", (I, H)), ("up", (I, H)), ("down", (H, I))):
+            q[m] = (rand_codes(rng, fmt, (rows, K)), rand_sf(rng, fmt, (rows, K // v)), np.float32(1.0))
+        encode_expert_into(packed, layout, fmt, e, H, I, q)
+        W[e] = {m: decode(fmt, q[m][0], q[m][1]) for m in q}
+
+    # activations: valid rows from the grid, padding rows random bytes
+    bpe = 4 if fmt == "nvfp4" else 8
+    a_codes = rng.integers(0, 256, (R, H * bpe // 8), dtype=np.uint8)
+    a_sf = rng.integers(0, 256, (R, H // v), dtype=np.uint8)
+    A = np.zeros((R, H))
+    for e in range(E):
+        lo, c = offsets[e], counts[e]
+        if c == 0:
+            continue
+        codes = rand_codes(rng, fmt, (c, H))
+        sf = rand_sf(rng, fmt, (c, H // v))
+        a_codes[lo:lo + c] = to_rows_bytes(fmt, codes)
+        a_sf[lo:lo + c] = sf
+        A[lo:lo + c] = decode(fmt, codes, sf)
+
+    t = lambda a, dt=torch.uint8: torch.from_numpy(np.ascontiguousarray(a)).to(dt).to(dev)
+    d_packed = t(packed)
+    d_a = t(a_codes)
+    d_asf = t(swizzle_sf(a_sf))
+    d_off = t(offsets, torch.int32)
+    d_cnt = t(counts, torch.int32)
+    one = torch.ones(1, dtype=torch.float32, device=dev)
+    scale = one if fmt == "nvfp4" else None
+    h_codes = torch.zeros(B.moe_codes_bytes(cfg, R, I), dtype=torch.uint8, device=dev)
+    h_sf = torch.zeros(B.moe_sf_bytes(cfg, R, I), dtype=torch.uint8, device=dev)
+    dbg = torch.full((R, 2 * I), float("nan"), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    B.moe_forward_gateup(cfg, T, d_packed, d_a, d_asf, scale, scale, d_off, d_cnt, h_codes, h_sf, dbg, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = dbg.cpu().numpy()
+    for e in range(E):
+        lo, c = offsets[e], counts[e]
+        if c == 0:
+            continue
+        g = A[lo:lo + c] @ W[e]["gate"].T
+        u = A[lo:lo + c] @ W[e]["up"].T
+        assert np.all(np.abs(g) < 2 ** 20)
+        np.testing.assert_array_equal(got[lo:lo + c, :I], g.astype(np.float32), err_msg=f"gate e={e}")
+        np.testing.assert_array_equal(got[lo:lo + c, I:], u.astype(np.float32), err_msg=f"up e={e}")
+    # rows without a slot are never written
+    valid = np.zeros(R, dtype=bool)
+    for e in range(E):
+        valid[offsets[e]:offsets[e] + counts[e]] = True
+    assert np.all(np.isnan(got[~valid]))
+
+    # down GEMM on intermediate codes chosen the same way
+    hc = rng.integers(0, 256, (R, I * bpe // 8), dtype=np.uint8)
+    hs = rng.integers(0, 256, (R, I // v), dtype=np.uint8)
+    Hm = np.zeros((R, I))
+    for e in range(E):
+        lo, c = offsets[e], counts[e]
+        if c == 0:
+            continue
+        codes = rand_codes(rng, fmt, (c, I))
+        sf = rand_sf(rng, fmt, (c, I // v))
+        hc[lo:lo + c] = to_rows_bytes(fmt, codes)
+        hs[lo:lo + c] = sf
+        Hm[lo:lo + c] = decode(fmt, codes, sf)
+    out = torch.full((R, H), float("nan"), dtype=torch.bfloat16, device=dev)
+    B.moe_forward_down(cfg, T, d_packed, t(hc), t(swizzle_sf(hs)), scale, d_off, d_cnt, out, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    o = out.float().cpu().numpy().astype(np.float64)
+    for e in range(E):
+        lo, c = offsets[e], counts[e]
+        if c == 0:
+            continue
+        ref = fm.bf16_round(Hm[lo:lo + c] @ W[e]["down"].T)
+        np.testing.assert_array_equal(o[lo:lo + c], ref, err_msg=f"down e={e}")
+    assert np.all(np.isnan(o[~valid]))

@@ -1,0 +1,137 @@
+"""GPU parity on small layers, every step against the oracle (GPU).
+
+Workload "tiny": T = 64 tokens, d_model 256, expert ffn 128, 8 experts,
+top-2, bf16 x ~ N(0, 1), float32 logits ~ N(0, 1), weights N(0, 1/fan_in)
+quantized by the library (NVFP4 with the 4-vs-6 pick, or MXFP8).  Bars:
+weight codes, routing, permutation and activation codes bit-exact; gate/up
+float32 relative Frobenius error <= 1e-4; at most 1e-3 of the requantized
+intermediate (code, block scale) pairs differ; bf16 output relative
+Frobenius error <= 1e-2.  Edge cases: a single token, routing that leaves
+experts empty or sends every token to the same experts, tied logits.
+"""
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from fp8_moe_expert_top_b200 import inputs
+from oracle import moe as omoe
+
+from gpu_common import assert_expert_equal, build_layer, gpu_expert, oracle_expert
+from helpers import rel_fro, sfvec, unpack_codes, unswizzle_sf
+
+TINY = inputs.WORKLOADS["tiny_nvfp4"]
+TINY_MX = dataclasses.replace(TINY, name="tiny_mxfp8", fmt=inputs.MXFP8)
+
+_layers = {}
+
+
+def get_layer(wl, dev):
+    key = (wl.name, wl.T)
+    if key not in _layers:
+        _layers[key] = build_layer(wl, dev)
+    return _layers[key]
+
+
+def oracle_experts(wl):
+    return {e: oracle_expert(wl, e, "cpu") for e in range(wl.num_experts)}
+
+
+def run_and_compare(layer, wl, x, logits, experts_q):
+    dev = layer.device
+    T = x.shape[0]
+    layer.status.zero_()
+    layer.gateup_debug.fill_(float("nan"))
+    y = layer.forward(x.to(dev), logits.to(dev))
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0
+    ref = omoe.forward(x.float().numpy(), logits.numpy(), experts_q, wl.top_k, wl.fmt,
+                       inputs.S_X, inputs.S_H, wl.num_experts)
+    # routing: bit-exact
+    np.testing.assert_array_equal(layer.topk_ids[:T].cpu().numpy(), ref["topk_ids"])
+    np.testing.assert_array_equal(layer.topk_w[:T].cpu().numpy().view(np.uint32), ref["topk_w"].view(np.uint32))
+    np.testing.assert_array_equal(layer.expert_counts.cpu().numpy(), ref["counts"])
+    np.testing.assert_array_equal(layer.expert_offsets.cpu().numpy(), ref["offsets"])
+    R = int(ref["offsets"][-1])
+    ss = layer.sorted_slots.cpu().numpy()
+    np.testing.assert_array_equal(ss[:R], ref["sorted_slots"])
+    assert np.all(ss[R:] == -1)
+    np.testing.assert_array_equal(layer.slot_to_row[:T * wl.top_k].cpu().numpy(), ref["slot_to_row"])
+    valid = ref["valid"]
+    H, I, v = wl.d_model, wl.d_ffn, sfvec(wl.fmt)
+    Rb = layer.R_max
+    # activation codes: bit-exact on valid rows
+    a_codes = unpack_codes(wl.fmt, layer.a_codes.cpu().numpy(), Rb, H)[:R]
+    a_sf = unswizzle_sf(layer.a_sf.cpu().numpy(), Rb, H // v)[:R]
+    np.testing.assert_array_equal(a_codes[valid], ref["a_codes"][valid])
+    np.testing.assert_array_equal(a_sf[valid], ref["a_sf"][valid])
+    # gate/up float32
+    dbg = layer.gateup_debug.cpu().numpy()[:R]
+    err_g = rel_fro(dbg[valid, :I], ref["gate"][valid])
+    err_u = rel_fro(dbg[valid, I:], ref["up"][valid])
+    assert err_g <= 1e-4 and err_u <= 1e-4, (err_g, err_u)
+    assert np.all(np.isnan(dbg[~valid]))
+    # requantized intermediate
+    hc = unpack_codes(wl.fmt, layer.h_codes.cpu().numpy(), Rb, I)[:R]
+    hs = unswizzle_sf(layer.h_sf.cpu().numpy(), Rb, I // v)[:R]
+    rc, rs = ref["h_codes"], ref["h_sf"]
+    differ = (hc != rc) | (np.repeat(hs, v, axis=1) != np.repeat(rs, v, axis=1))
+    frac = float(differ[valid].mean())
+    assert frac <= 1e-3, frac
+    # layer output
+    yr = ref["y"]
+    err_y = rel_fro(y.float().cpu().numpy(), yr)
+    assert err_y <= 1e-2, err_y
+    return dict(err_g=err_g, err_u=err_u, h_frac=frac, err_y=err_y)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl", [TINY, TINY_MX], ids=lambda w: w.name)
+def test_weights_bit_exact(cuda_device, wl):
+    layer = get_layer(wl, cuda_device)
+    for e in range(wl.num_experts):
+        assert_expert_equal(gpu_expert(layer, wl, e), oracle_expert(wl, e, "cpu"), e)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl", [TINY, TINY_MX], ids=lambda w: w.name)
+def test_layer_seeded_inputs(cuda_device, wl):
+    layer = get_layer(wl, cuda_device)
+    x, lg = inputs.make_x(wl), inputs.make_logits(wl)
+    run_and_compare(layer, wl, x, lg, oracle_experts(wl))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl", [TINY, TINY_MX], ids=lambda w: w.name)
+@pytest.mark.parametrize("case", ["one_token", "hot_experts", "ties", "empty_experts", "ragged"])
+def test_layer_edge_cases(cuda_device, wl, case):
+    layer = get_layer(wl, cuda_device)
+    E = wl.num_experts
+    if case == "one_token":
+        x, lg = inputs.make_x(wl, T=1, seed=11), inputs.make_logits(wl, T=1, seed=12)
+    elif case == "hot_experts":          # every token picks experts 3 and 5
+        x, lg = inputs.make_x(wl, seed=13), inputs.make_logits(wl, seed=14)
+        lg[:, 3] += 50.0
+        lg[:, 5] += 40.0
+    elif case == "ties":                 # many equal logits, ties go to the lower index
+        x = inputs.make_x(wl, seed=15)
+        lg = inputs.make_logits_with_ties(wl.T, E, seed=16)
+    elif case == "empty_experts":        # experts 0, 1 and 6 never chosen
+        x, lg = inputs.make_x(wl, seed=17), inputs.make_logits(wl, seed=18)
+        lg[:, [0, 1, 6]] -= 100.0
+    else:                                # T not a multiple of anything
+        x, lg = inputs.make_x(wl, T=37, seed=19), inputs.make_logits(wl, T=37, seed=20)
+    run_and_compare(layer, wl, x, lg, oracle_experts(wl))
+
+
+@pytest.mark.gpu
+def test_empty_batch(cuda_device):
+    layer = get_layer(TINY, cuda_device)
+    x = torch.zeros(0, TINY.d_model, dtype=torch.bfloat16, device=cuda_device)
+    lg = torch.zeros(0, TINY.num_experts, dtype=torch.float32, device=cuda_device)
+    y = layer.forward(x, lg)
+    torch.cuda.synchronize()
+    assert y.shape == (0, TINY.d_model)
+    assert int(layer.expert_offsets[-1].item()) == 0
