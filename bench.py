@@ -1,0 +1,456 @@
+"""Benchmark of the routed MoE expert layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the whole layer over one batch of synthetic inputs
+already resident in HBM: route -> permute+quantize -> gate/up GEMM (SwiGLU +
+requantization) -> down GEMM -> weighted combine.  Default workload: the
+decode NVFP4 layer (64 tokens, d_model 4096, expert ffn 2560, 384 experts,
+top-8).  Weights are random-init of that architecture, quantized once by the
+library before timing.  Every timed step is bracketed by CUDA events on the
+launching stream; L2 is flushed (a 512 MiB write) between timed steps,
+outside the events.  With --gpus N > 1 (launched by torchrun) every rank runs
+an independent replica of the same workload (the layer has no data-path
+exchange on one node: "replicas only"), the times are max-reduced over ranks
+and `value` counts the tokens of all ranks.
+
+--impl reference times the CPU oracle (oracle/, numpy) on a bounded sample of
+the same workload on the host cores; under torchrun only rank 0 runs it.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fp8_moe_expert_top_b200 import inputs  # noqa: E402
+
+METRIC = "MoE layer tokens/s on 1 B200; % of HBM or NVFP4/FP8 tensor roofline"
+UNIT = "tokens/s"
+
+
+# --------------------------------------------------------------------------- helpers
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(values, world_size, device=None):
+    """Element-wise max of a list of floats over all ranks (identity for one rank)."""
+    if world_size <= 1:
+        return list(values)
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def barrier(world_size):
+    if world_size > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sms.append(float(parts[1]))
+                    maxs.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+# --------------------------------------------------------------------------- workload
+
+def build_layer(wl, device, T):
+    from fp8_moe_expert_top_b200.layer import ExpertLayer
+    layer = ExpertLayer(wl.num_experts, wl.top_k, wl.d_model, wl.d_ffn, wl.fmt, T, device,
+                        s_x=inputs.S_X, s_h=inputs.S_H)
+    chunk = 16
+    for e0 in range(0, wl.num_experts, chunk):
+        n = min(chunk, wl.num_experts - e0)
+        ws = [inputs.make_expert_weights(wl, e, device=device) for e in range(e0, e0 + n)]
+        wg = torch.stack([w[0] for w in ws]).contiguous()
+        wu = torch.stack([w[1] for w in ws]).contiguous()
+        wd = torch.stack([w[2] for w in ws]).contiguous()
+        layer.quantize_experts(e0, wg, wu, wd)
+        del ws, wg, wu, wd
+    torch.cuda.synchronize()
+    return layer
+
+
+def phase_bytes(wl, n_touched, slots):
+    """Algorithmic HBM bytes of each phase (compulsory traffic, no re-reads)."""
+    H, I, E, T = wl.d_model, wl.d_ffn, wl.num_experts, wl.T
+    bpe = 0.5 if wl.fmt == inputs.NVFP4 else 1.0
+    sf = 1.0 / (16 if wl.fmt == inputs.NVFP4 else 32)
+    q = bpe + sf                                  # bytes per quantized element (codes + block scales)
+    w13 = n_touched * 2 * I * H * q
+    w2 = n_touched * H * I * q
+    return {
+        "route": T * E * 4 + T * wl.top_k * 8,
+        "permute": T * H * 2 + slots * H * q,
+        "gateup": w13 + slots * H * q + slots * I * q,
+        "down": w2 + slots * I * q + slots * H * 2,
+        "combine": slots * H * 2 + T * H * 2 + T * wl.top_k * 8,
+        "layer": w13 + w2 + T * H * 2 + T * E * 4 + T * H * 2,
+    }
+
+
+PHASES = ("route", "permute", "gateup", "down", "combine")
+
+
+def run_ours(args, wl, ws, rank, local):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    T = wl.T
+    layer = build_layer(wl, device, T)
+    x_h = inputs.make_x(wl)
+    lg_h = inputs.make_logits(wl)
+    x = x_h.to(device)
+    lg = lg_h.to(device)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        layer.route(lg, T)
+        if ev is not None:
+            ev[1].record(stream)
+        layer.permute(x, T)
+        if ev is not None:
+            ev[2].record(stream)
+        layer.gateup(T)
+        if ev is not None:
+            ev[3].record(stream)
+        layer.down(T)
+        if ev is not None:
+            ev[4].record(stream)
+        layer.combine(T)
+        if ev is not None:
+            ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    counts = layer.expert_counts.cpu().numpy()
+    n_touched = int((counts > 0).sum())
+    slots = T * wl.top_k
+    status = int(layer.status.item())
+    if status != 0:
+        raise RuntimeError(f"device status word {status:#x} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(ws)
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()                      # L2 flush, outside the events
+        step(evs[i])
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    per_phase = {p: [] for p in PHASES}
+    step_ms = []
+    for ev in evs:
+        for j, p in enumerate(PHASES):
+            per_phase[p].append(ev[j].elapsed_time(ev[j + 1]))
+        step_ms.append(ev[0].elapsed_time(ev[5]))
+    total_ms = sum(step_ms)
+    total_ms = max_over_ranks([total_ms], ws, device)[0]
+
+    # end to end through the public API: pinned host inputs in, host output back
+    x_pin = x_h.pin_memory()
+    lg_pin = lg_h.pin_memory()
+    y_pin = torch.empty(T, wl.d_model, dtype=torch.bfloat16).pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for _ in range(max(1, args.warmup)):
+        x_d = x_pin.to(device, non_blocking=True)
+        lg_d = lg_pin.to(device, non_blocking=True)
+        y_pin.copy_(layer.forward(x_d, lg_d), non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(ws)
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        x_d = x_pin.to(device, non_blocking=True)
+        lg_d = lg_pin.to(device, non_blocking=True)
+        y = layer.forward(x_d, lg_d)
+        y_pin.copy_(y, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e2e_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in e2e_ev)], ws, device)[0]
+
+    # roofline of the dominant kernel
+    peaks, peak_kind = load_peaks()
+    bytes_ = phase_bytes(wl, n_touched, slots)
+    mean_ms = {p: statistics.mean(v) for p, v in per_phase.items()}
+    dom = max(("gateup", "down"), key=lambda p: mean_ms[p])
+    flops_slot = 6.0 * wl.d_model * wl.d_ffn
+    dom_flops = slots * flops_slot * (2.0 / 3.0 if dom == "gateup" else 1.0 / 3.0)
+    t_dom = mean_ms[dom] * 1e-3
+    bf16 = peaks.get("bf16_tflops", 1590.0)
+    tensor_peak = bf16 * (4.0 if wl.fmt == inputs.NVFP4 else 2.0)     # nominal fp4 / fp8 : bf16 ratios
+    t_hbm = bytes_[dom] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = dom_flops / (tensor_peak * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": bytes_[dom] / t_dom / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": dom_flops / t_dom / 1e12, "peak": tensor_peak, "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = f"moe_gemm_kernel ({dom})"
+    roof["peak_source"] = peak_kind + (" hbm_gbs" if roof["bound"] == "hbm" else
+                                       f" bf16_tflops x {4 if wl.fmt == inputs.NVFP4 else 2} (nominal ratio)")
+    roof["traffic"] = measured_traffic(wl.name, dom)
+    # whole-layer roofline (slower of bytes at HBM peak and FLOPs at tensor peak)
+    layer_t = max(bytes_["layer"] / (peaks["hbm_gbs"] * 1e9), slots * flops_slot / (tensor_peak * 1e12))
+    value = ws * T * args.steps / (total_ms * 1e-3)
+    out = {
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": wl.fmt,
+        "data": "synthetic (seeded N(0,1) x and logits, N(0,1/fan_in) weights, random init)",
+        "config": {"workload": wl.name, "T": T, "d_model": wl.d_model, "d_ffn": wl.d_ffn,
+                   "num_experts": wl.num_experts, "top_k": wl.top_k, "format": wl.fmt,
+                   "experts_touched": n_touched, "l2": "flushed between timed steps (512 MiB write)",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+        "roofline": roof,
+        "layer_roofline_frac": layer_t / (total_ms * 1e-3 / args.steps),
+        "phase_ms": {p: round(mean_ms[p], 4) for p in PHASES},
+        "e2e": {"value": ws * T * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": int(x_h.numel() * 2 + lg_h.numel() * 4),
+                "d2h_bytes_per_step": int(T * wl.d_model * 2)},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk,
+    }
+    return out, layer
+
+
+def measured_traffic(workload, phase):
+    """Per-launch DRAM bytes from the committed ncu summary, if the kernel source
+    has not changed since it was captured (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(workload, {}).get(phase)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "fp8_moe_expert_top_b200", "csrc", "gemm.cu")
+    if ent.get("gemm_sha") != file_sha(src):
+        return None
+    return ent.get("bytes")
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def _oracle_quantize(args_):
+    e, fmt, wg, wu, wd = args_
+    from oracle import moe as omoe
+    return e, omoe.quantize_expert(wg, wu, wd, fmt)
+
+
+def oracle_sample(wl, n_tokens):
+    """Inputs of the bounded oracle sample: the first n_tokens tokens and the
+    quantized weights of every expert they select (prepared outside timing,
+    in a spawn pool).  Weights are drawn on the GPU when there is one, as the
+    library's benchmark does, else on the CPU."""
+    import multiprocessing as mp
+    from oracle import route as ort
+    x = inputs.make_x(wl)[:n_tokens].float().numpy()
+    lg = inputs.make_logits(wl)[:n_tokens].numpy()
+    ids = ort.topk_select(lg, wl.top_k)
+    need = sorted(set(int(e) for e in ids.reshape(-1)))
+    wdev = "cuda" if torch.cuda.is_available() else "cpu"
+    jobs = []
+    for e in need:
+        wg, wu, wd = (w.cpu().numpy() for w in inputs.make_expert_weights(wl, e, device=wdev))
+        jobs.append((e, wl.fmt, wg, wu, wd))
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(min(len(need), max(1, os.cpu_count() or 1))) as pool:
+        experts = dict(pool.map(_oracle_quantize, jobs))
+    return x, lg, experts
+
+
+def time_oracle(wl, x, lg, experts):
+    from oracle import moe as omoe
+    t0 = time.perf_counter()
+    omoe.forward_tokens(x, lg, experts, wl.top_k, wl.fmt, inputs.S_X, inputs.S_H)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return 1
+
+
+def default_sample_tokens(wl):
+    return 2 if wl.d_model * wl.d_ffn > (1 << 20) else min(wl.T, 64)
+
+
+def cpu_baseline(wl, n_tokens=None):
+    n = n_tokens or default_sample_tokens(wl)
+    x, lg, experts = oracle_sample(wl, n)
+    dt = time_oracle(wl, x, lg, experts)
+    return {"value": n / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} tokens of {wl.name} (their {len(experts)} experts' weights quantized by the "
+                      f"oracle beforehand, untimed); numpy float64, host cpu_count={os.cpu_count()}"}
+
+
+def run_reference(args, wl, ws, rank):
+    if rank != 0:
+        return None
+    n = default_sample_tokens(wl)
+    x, lg, experts = oracle_sample(wl, n)
+    for _ in range(args.warmup):
+        time_oracle(wl, x, lg, experts)
+    times = [time_oracle(wl, x, lg, experts) for _ in range(args.steps)]
+    total = sum(times)
+    value = n * args.steps / total
+    cores = blas_threads()
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) x and logits, N(0,1/fan_in) weights, random init)",
+        "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "d_ffn": wl.d_ffn,
+                   "num_experts": wl.num_experts, "top_k": wl.top_k, "format": wl.fmt,
+                   "sample_tokens_per_step": n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{n} tokens of {wl.name} per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# --------------------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode_nvfp4", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = inputs.WORKLOADS[args.workload]
+    ws, rank, local = dist_env()
+    if ws != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {ws}", file=sys.stderr)
+    if args.impl == "reference":
+        out = run_reference(args, wl, ws, rank)
+        if out is not None:
+            print(json.dumps(out))
+        return 0
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        out, layer = run_ours(args, wl, ws, rank, local)
+        del layer
+        torch.cuda.empty_cache()
+        if rank == 0:
+            if ws == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(wl)
+            print(json.dumps(out))
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -16,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+from fp8_moe_expert_top_b200 import binding as B
 from fp8_moe_expert_top_b200 import inputs
 from oracle import moe as omoe
 
@@ -57,7 +58,8 @@ def run_and_compare(layer, wl, x, logits, experts_q):
     R = int(ref["offsets"][-1])
     ss = layer.sorted_slots.cpu().numpy()
     np.testing.assert_array_equal(ss[:R], ref["sorted_slots"])
-    assert np.all(ss[R:] == -1)
+    R_call = B.moe_max_rows(layer.cfg, T)          # rows this call owns
+    assert np.all(ss[R:R_call] == -1)
     np.testing.assert_array_equal(layer.slot_to_row[:T * wl.top_k].cpu().numpy(), ref["slot_to_row"])
     valid = ref["valid"]
     H, I, v = wl.d_model, wl.d_ffn, sfvec(wl.fmt)
