@@ -420,10 +420,15 @@ def main(argv=None):
     ap.add_argument("--workload", default="decode_nvfp4", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="profiling only: override the number of experts (smaller device footprint for ncu)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = inputs.WORKLOADS[args.workload]
+    if args.experts is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, name=f"{wl.name}_e{args.experts}", num_experts=args.experts)
     ws, rank, local = dist_env()
     if ws != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {ws}", file=sys.stderr)

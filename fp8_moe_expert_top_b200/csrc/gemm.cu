@@ -40,7 +40,8 @@ constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kStages = 4;
 constexpr int kRowBytesPerStage = 128;  // K bytes of one row per stage
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;             // two warps per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 
 template <int FMT>
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(tfull_bar, 1);
-    mbar_init(tempty_bar, 128);
+    mbar_init(tempty_bar, 32 * kEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmap_a);
@@ -238,9 +239,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // Warps 2..9: quarter q = warp % 4 of the TMEM lanes (rows), half of the
+    // accumulator columns.  Each thread copies its 128 columns to registers,
+    // hands the accumulator back to the MMA warp at once, and then does the
+    // epilogue math while the next tile's MMAs run.
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row_l = q * 32 + lane;
-    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + half * (kBN / 2);
     uint32_t acc_phase = 0;
     const int I = args.n_rows_b / 2;  // gate/up: channels; unused for down
     const int H = args.n_rows_b;      // down: output channels
@@ -255,80 +261,87 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      float acc[kBN / 2];
+#pragma unroll
+      for (int j = 0; j < kBN / 64; ++j) tmem_ld32(t_row + 32 * j, acc + 32 * j);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(tempty_bar);
+      acc_phase ^= 1u;
+      if (!valid) continue;
       if (GATEUP) {
+        // columns of this half: [gate 32 | up 32] x 2, channels ch0 + [0, 64)
+        const int ch0 = nt * (kBN / 2) + half * (kBN / 4);
         const float sa = (FMT == MOE_NVFP4) ? __ldg(args.a_scale) : 1.0f;
         const float sg = (FMT == MOE_NVFP4) ? __fmul_rn(sa, __ldg(args.w_scales + 3 * e + 0)) : 1.0f;
         const float su = (FMT == MOE_NVFP4) ? __fmul_rn(sa, __ldg(args.w_scales + 3 * e + 1)) : 1.0f;
         const float sh = (FMT == MOE_NVFP4) ? __ldg(args.h_scale) : 1.0f;
+#pragma unroll
+        for (int j = 0; j < kBN / 128; ++j) {
+          float* g = acc + 64 * j;
+          float* u = acc + 64 * j + 32;
+          const int ch = ch0 + 32 * j;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            g[i] *= sg;
+            u[i] *= su;
+          }
+          if (args.dbg != nullptr) {
+            float4* dg = reinterpret_cast<float4*>(args.dbg + row * (2 * I) + ch);
+            float4* du = reinterpret_cast<float4*>(args.dbg + row * (2 * I) + I + ch);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              dg[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
+              du[i] = make_float4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
+            }
+          }
+          // h = silu(g) * u, written over g
+#pragma unroll
+          for (int i = 0; i < 32; ++i) g[i] = __fdividef(g[i] * u[i], 1.0f + __expf(-g[i]));
+        }
+        // h of this thread: acc[0..32) channels ch0 + [0, 32), acc[64..96) ch0 + [32, 64)
+        if (FMT == MOE_NVFP4) {
 #pragma unroll 1
-        for (int j = 0; j < kBN / 64; ++j) {
-          float g[32], u[32];
-          tmem_ld32(t_row + 64 * j, g);
-          tmem_ld32(t_row + 64 * j + 32, u);
-          tmem_ld_wait();
-          if (valid) {
-            const int ch0 = nt * (kBN / 2) + 32 * j;
-            float h[32];
+          for (int b = 0; b < 4; ++b) {
+            float blk[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float gv = g[i] * sg;
-              const float uv = u[i] * su;
-              g[i] = gv;
-              u[i] = uv;
-              h[i] = gv * uv / (1.0f + expf(-gv));
-            }
-            if (args.dbg != nullptr) {
-              float4* dg = reinterpret_cast<float4*>(args.dbg + row * (2 * I) + ch0);
-              float4* du = reinterpret_cast<float4*>(args.dbg + row * (2 * I) + I + ch0);
+            for (int i = 0; i < 16; ++i)
+              blk[i] = (b == 0) ? acc[i] : (b == 1) ? acc[16 + i] : (b == 2) ? acc[64 + i] : acc[80 + i];
+            const Nvfp4Block qb = nvfp4_quantize16(blk, sh);
+            const int ch = ch0 + 16 * b;
+            *reinterpret_cast<uint2*>(args.h_codes + row * (I / 2) + ch / 2) =
+                make_uint2(static_cast<uint32_t>(qb.codes), static_cast<uint32_t>(qb.codes >> 32));
+            args.h_sf[sf_offset(row, ch / 16, I / 16)] = static_cast<uint8_t>(qb.sf);
+          }
+        } else {
+#pragma unroll 1
+          for (int b = 0; b < 2; ++b) {
+            float blk[32];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                dg[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
-                du[i] = make_float4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
-              }
-            }
-            if (FMT == MOE_NVFP4) {
-              const Nvfp4Block b0 = nvfp4_quantize16(h, sh);
-              const Nvfp4Block b1 = nvfp4_quantize16(h + 16, sh);
-              *reinterpret_cast<uint4*>(args.h_codes + row * (I / 2) + ch0 / 2) =
-                  make_uint4(static_cast<uint32_t>(b0.codes), static_cast<uint32_t>(b0.codes >> 32),
-                             static_cast<uint32_t>(b1.codes), static_cast<uint32_t>(b1.codes >> 32));
-              *reinterpret_cast<uint16_t*>(args.h_sf + sf_offset(row, ch0 / 16, I / 16)) =
-                  static_cast<uint16_t>(b0.sf | (b1.sf << 8));
-            } else {
-              uint32_t w[8];
-              const uint32_t ex = mxfp8_quantize32(h, w);
-              uint4* dst = reinterpret_cast<uint4*>(args.h_codes + row * I + ch0);
-              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-              args.h_sf[sf_offset(row, ch0 / 32, I / 32)] = static_cast<uint8_t>(ex);
-            }
+            for (int i = 0; i < 32; ++i) blk[i] = (b == 0) ? acc[i] : acc[64 + i];
+            uint32_t w[8];
+            const uint32_t ex = mxfp8_quantize32(blk, w);
+            const int ch = ch0 + 32 * b;
+            uint4* dst = reinterpret_cast<uint4*>(args.h_codes + row * I + ch);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            args.h_sf[sf_offset(row, ch / 32, I / 32)] = static_cast<uint8_t>(ex);
           }
         }
       } else {
         const float s = (FMT == MOE_NVFP4) ? __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scales + 3 * e + 2)) : 1.0f;
-#pragma unroll 1
-        for (int j = 0; j < kBN / 32; ++j) {
-          float v[32];
-          tmem_ld32(t_row + 32 * j, v);
-          tmem_ld_wait();
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(args.out + row * H + nt * kBN + 32 * j);
+        uint4* dst = reinterpret_cast<uint4*>(args.out + row * H + nt * kBN + half * (kBN / 2));
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint32_t p[4];
+        for (int i = 0; i < kBN / 16; ++i) {
+          uint32_t p[4];
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * i + 2 * c] * s, v[8 * i + 2 * c + 1] * s);
-                p[c] = *reinterpret_cast<const uint32_t*>(&b);
-              }
-              dst[i] = make_uint4(p[0], p[1], p[2], p[3]);
-            }
+          for (int c = 0; c < 4; ++c) {
+            const __nv_bfloat162 b = __floats2bfloat162_rn(acc[8 * i + 2 * c] * s, acc[8 * i + 2 * c + 1] * s);
+            p[c] = *reinterpret_cast<const uint32_t*>(&b);
           }
+          dst[i] = make_uint4(p[0], p[1], p[2], p[3]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(tempty_bar);
-      acc_phase ^= 1u;
     }
   }
 

@@ -17,11 +17,11 @@
 
 namespace moe {
 
-// 64 bf16 -> float
-__device__ __forceinline__ void load64_bf16(const __nv_bfloat16* p, float* f) {
+// 16 bf16 -> float
+__device__ __forceinline__ void load16_bf16(const __nv_bfloat16* p, float* f) {
   const uint4* q = reinterpret_cast<const uint4*>(p);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < 2; ++i) {
     const uint4 u = __ldg(q + i);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -47,42 +47,50 @@ __global__ void __launch_bounds__(128) permute_kernel(int T, int H, int k, const
 #pragma unroll
   for (int j = 0; j < 8; ++j) rows[j] = (j < k) ? __ldg(slot_to_row + static_cast<int64_t>(t) * k + j) : 0;
   for (int g = lane; g < groups; g += 32) {
-    float f[64];
-    load64_bf16(x + static_cast<int64_t>(t) * H + 64 * g, f);
+    const __nv_bfloat16* src = x + static_cast<int64_t>(t) * H + 64 * g;
     if (FMT == MOE_NVFP4) {
-      uint64_t c[4];
-      uint32_t sfw = 0;
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const Nvfp4Block q = nvfp4_quantize16(f + 16 * b, s_x);
-        c[b] = q.codes;
-        sfw |= q.sf << (8 * b);
-      }
       const int64_t nsf = H / 16;
+      uint32_t sfw = 0;
+#pragma unroll 1
+      for (int b = 0; b < 4; ++b) {
+        float f[16];
+        load16_bf16(src + 16 * b, f);
+        const Nvfp4Block q = nvfp4_quantize16(f, s_x);
+        sfw |= q.sf << (8 * b);
+        const uint2 c = make_uint2(static_cast<uint32_t>(q.codes), static_cast<uint32_t>(q.codes >> 32));
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j >= k) break;
+          *reinterpret_cast<uint2*>(a_codes + static_cast<int64_t>(rows[j]) * (H / 2) + 32 * g + 8 * b) = c;
+        }
+      }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j >= k) break;
-        const int64_t r = rows[j];
-        uint4* dst = reinterpret_cast<uint4*>(a_codes + r * (H / 2) + 32 * g);
-        dst[0] = make_uint4(static_cast<uint32_t>(c[0]), static_cast<uint32_t>(c[0] >> 32),
-                            static_cast<uint32_t>(c[1]), static_cast<uint32_t>(c[1] >> 32));
-        dst[1] = make_uint4(static_cast<uint32_t>(c[2]), static_cast<uint32_t>(c[2] >> 32),
-                            static_cast<uint32_t>(c[3]), static_cast<uint32_t>(c[3] >> 32));
-        *reinterpret_cast<uint32_t*>(a_sf + sf_offset(r, 4 * g, nsf)) = sfw;
+        *reinterpret_cast<uint32_t*>(a_sf + sf_offset(rows[j], 4 * g, nsf)) = sfw;
       }
     } else {
-      uint32_t w[16];
-      const uint32_t e0 = mxfp8_quantize32(f, w);
-      const uint32_t e1 = mxfp8_quantize32(f + 32, w + 8);
       const int64_t nsf = H / 32;
+      uint32_t sfw = 0;
+#pragma unroll 1
+      for (int b = 0; b < 2; ++b) {
+        float f[32];
+        load16_bf16(src + 32 * b, f);
+        load16_bf16(src + 32 * b + 16, f + 16);
+        uint32_t w[8];
+        sfw |= mxfp8_quantize32(f, w) << (8 * b);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j >= k) break;
+          uint4* dst = reinterpret_cast<uint4*>(a_codes + static_cast<int64_t>(rows[j]) * H + 64 * g + 32 * b);
+          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+      }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j >= k) break;
-        const int64_t r = rows[j];
-        uint4* dst = reinterpret_cast<uint4*>(a_codes + r * H + 64 * g);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-        *reinterpret_cast<uint16_t*>(a_sf + sf_offset(r, 2 * g, nsf)) = static_cast<uint16_t>(e0 | (e1 << 8));
+        *reinterpret_cast<uint16_t*>(a_sf + sf_offset(rows[j], 2 * g, nsf)) = static_cast<uint16_t>(sfw);
       }
     }
   }

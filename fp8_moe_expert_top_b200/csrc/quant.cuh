@@ -58,32 +58,90 @@ struct Nvfp4Block {
   uint32_t sf;     // E4M3 block-scale code
 };
 
-// Quantize one candidate: the block maximum a is mapped to c (4 or 6).
-__device__ __forceinline__ float nvfp4_candidate(const float* x, float a, float s_g, float c, uint64_t& codes,
+// Hardware round-to-nearest-even conversions of two floats at once (lo goes
+// to the low nibble / byte).
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tmov.b16 %0, {t, 0};\n\t}"
+      : "=h"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Relative width of the bracket around an approximate quotient.  The
+// approximation |x| * RN(1/S) is within 2^-23 (relative) of the exact
+// quotient, so the exact quotient and its float32 rounding both lie strictly
+// inside [q(1 - 2^-21), q(1 + 2^-21)].  When both ends of the bracket encode
+// to the same code, so does RN(|x| / S) (the encoders are monotone); only
+// otherwise is the exact division needed.  The results are therefore those
+// of the plain definition, bit for bit.
+constexpr float kBracketLo = 1.0f - 0x1p-21f;
+constexpr float kBracketHi = 1.0f + 0x1p-21f;
+
+// Exact slow paths, kept out of line so the common path stays small.
+static __device__ __noinline__ uint32_t e2m1_code_exact(float num, float den) {
+  return e2m1_mag_code(__fdiv_rn(num, den));
+}
+static __device__ __noinline__ uint32_t e4m3_code_exact(float num, float den) {
+  return e4m3_encode(__fdiv_rn(num, den));
+}
+
+// E2M1 magnitude code of RN(num / den), num >= 0, den > 0, with 1/den given.
+__device__ __forceinline__ uint32_t e2m1_code_of_quotient(float num, float den, float rden) {
+  const float q = __fmul_rn(num, rden);
+  const uint32_t pair = cvt_e2m1x2(__fmul_rn(q, kBracketLo), __fmul_rn(q, kBracketHi));
+  const uint32_t lo = pair & 0x7u, hi = (pair >> 4) & 0x7u;
+  if (lo == hi) return lo;
+  return e2m1_code_exact(num, den);
+}
+
+// E4M3 code of RN(num / den), num >= 0, den > 0.
+__device__ __forceinline__ uint32_t e4m3_code_of_quotient(float num, float den) {
+  if (num == 0.0f) return 0u;
+  const float q = __fmul_rn(num, __frcp_rn(den));
+  const uint32_t pair = cvt_e4m3x2(__fmul_rn(q, kBracketLo), __fmul_rn(q, kBracketHi));
+  const uint32_t lo = pair & 0xFFu, hi = pair >> 8;
+  if (lo == hi) return lo;
+  return e4m3_code_exact(num, den);
+}
+
+// One candidate of the 4-vs-6 search on magnitudes ax[16] (block maximum a
+// mapped to c).  Returns the squared error; mags receives the 3-bit
+// magnitude codes (element i in bits [4i, 4i+4)), sf the scale code.
+// Uses |x - dec(q)S| = ||x| - |dec(q)|S|, which holds bit for bit because
+// rounding is symmetric in sign.
+__device__ __forceinline__ float nvfp4_candidate(const float* ax, float a, float s_g, float c, uint64_t& mags,
                                                  uint32_t& sf) {
-  const float denom = __fmul_rn(c, s_g);
-  const float ratio = __fdiv_rn(a, denom);
-  sf = e4m3_encode(ratio);
+  sf = e4m3_code_of_quotient(a, __fmul_rn(c, s_g));
   const float S = __fmul_rn(e4m3_decode(sf), s_g);
   float d2[16];
-  codes = 0;
+  mags = 0;
   if (S == 0.0f) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) d2[i] = __fmul_rn(x[i], x[i]);
-  } else {
+    for (int i = 0; i < 16; ++i) d2[i] = __fmul_rn(ax[i], ax[i]);
+  } else if (S >= 0x1p-100f) {
+    const float rS = __frcp_rn(S);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const float q = __fdiv_rn(fabsf(x[i]), S);
-      const uint32_t m = e2m1_mag_code(q);
-      const float r = __fmul_rn(e2m1_mag_value(m), S);
-      const bool neg = x[i] < 0.0f;
-      const uint32_t code = m | ((neg && m != 0u) ? 8u : 0u);
-      codes |= static_cast<uint64_t>(code) << (4 * i);
-      const float d = __fsub_rn(x[i], neg ? -r : r);
+      const uint32_t m = e2m1_code_of_quotient(ax[i], S, rS);
+      mags |= static_cast<uint64_t>(m) << (4 * i);
+      const float d = __fsub_rn(ax[i], __fmul_rn(e2m1_mag_value(m), S));
+      d2[i] = __fmul_rn(d, d);
+    }
+  } else {  // tiny scales: exact division throughout
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t m = e2m1_code_exact(ax[i], S);
+      mags |= static_cast<uint64_t>(m) << (4 * i);
+      const float d = __fsub_rn(ax[i], __fmul_rn(e2m1_mag_value(m), S));
       d2[i] = __fmul_rn(d, d);
     }
   }
-  // fixed pairwise tree
 #pragma unroll
   for (int w = 8; w >= 1; w >>= 1) {
 #pragma unroll
@@ -94,16 +152,25 @@ __device__ __forceinline__ float nvfp4_candidate(const float* x, float a, float 
 
 // NVFP4 4-vs-6 quantization of 16 float32 values with tensor scale s_g > 0.
 __device__ __forceinline__ Nvfp4Block nvfp4_quantize16(const float* x, float s_g) {
+  float ax[16];
   float a = 0.0f;
+  uint64_t neg = 0;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
-  uint64_t c6, c4;
+  for (int i = 0; i < 16; ++i) {
+    ax[i] = fabsf(x[i]);
+    a = fmaxf(a, ax[i]);
+    neg |= static_cast<uint64_t>(x[i] < 0.0f) << (4 * i + 3);
+  }
+  uint64_t m6, m4;
   uint32_t e6, e4;
-  const float err6 = nvfp4_candidate(x, a, s_g, 6.0f, c6, e6);
-  const float err4 = nvfp4_candidate(x, a, s_g, 4.0f, c4, e4);
-  Nvfp4Block b;
+  const float err6 = nvfp4_candidate(ax, a, s_g, 6.0f, m6, e6);
+  const float err4 = nvfp4_candidate(ax, a, s_g, 4.0f, m4, e4);
   const bool four = err4 < err6;
-  b.codes = four ? c4 : c6;
+  const uint64_t mags = four ? m4 : m6;
+  // sign bit only where the magnitude code is non-zero (canonical +0)
+  const uint64_t nz = (mags | (mags >> 1) | (mags >> 2)) & 0x1111111111111111ull;
+  Nvfp4Block b;
+  b.codes = mags | (neg & (nz << 3));
   b.sf = four ? e4 : e6;
   return b;
 }

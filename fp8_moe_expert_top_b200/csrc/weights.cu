@@ -62,15 +62,6 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(int H, int I, const f
   const int g = static_cast<int>(gid % G);
   const float* src = (m == 0 ? w_gate : (m == 1 ? w_up : w_down)) + static_cast<int64_t>(e) * n_per_matrix +
                      src_row * K + 64 * g;
-  float f[64];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(src) + i);
-    f[4 * i] = v.x;
-    f[4 * i + 1] = v.y;
-    f[4 * i + 2] = v.z;
-    f[4 * i + 3] = v.w;
-  }
   // destination row: gate/up interleaved in groups of 32 rows inside w13
   int64_t dst_row;
   uint8_t *codes, *sfbuf;
@@ -86,37 +77,54 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(int H, int I, const f
     codes = w13_codes;
     sfbuf = w13_sf;
   }
+  const float4* src4 = reinterpret_cast<const float4*>(src);
   if (FMT == MOE_NVFP4) {
     const float a = amax[e * 3 + m];
     const float s_g = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);
-    uint64_t c[4];
     uint32_t sfw = 0;
-#pragma unroll
+    uint8_t* dst = codes + (static_cast<int64_t>(e) * rows_per_expert + dst_row) * (K / 2) + 32 * g;
+#pragma unroll 1
     for (int b = 0; b < 4; ++b) {
-      const Nvfp4Block q = nvfp4_quantize16(f + 16 * b, s_g);
-      c[b] = q.codes;
+      float f[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = __ldg(src4 + 4 * b + i);
+        f[4 * i] = v.x;
+        f[4 * i + 1] = v.y;
+        f[4 * i + 2] = v.z;
+        f[4 * i + 3] = v.w;
+      }
+      const Nvfp4Block q = nvfp4_quantize16(f, s_g);
       sfw |= q.sf << (8 * b);
+      *reinterpret_cast<uint2*>(dst + 8 * b) =
+          make_uint2(static_cast<uint32_t>(q.codes), static_cast<uint32_t>(q.codes >> 32));
     }
-    const int64_t row_bytes = K / 2;
-    uint8_t* dst = codes + (static_cast<int64_t>(e) * rows_per_expert + dst_row) * row_bytes + 32 * g;
-    reinterpret_cast<uint4*>(dst)[0] = make_uint4(static_cast<uint32_t>(c[0]), static_cast<uint32_t>(c[0] >> 32),
-                                                  static_cast<uint32_t>(c[1]), static_cast<uint32_t>(c[1] >> 32));
-    reinterpret_cast<uint4*>(dst)[1] = make_uint4(static_cast<uint32_t>(c[2]), static_cast<uint32_t>(c[2] >> 32),
-                                                  static_cast<uint32_t>(c[3]), static_cast<uint32_t>(c[3] >> 32));
     const int64_t nsf = K / 16;
     uint8_t* sfe = sfbuf + static_cast<int64_t>(e) * rows_per_expert * nsf;
     *reinterpret_cast<uint32_t*>(sfe + sf_offset(dst_row, 4 * g, nsf)) = sfw;
   } else {
-    uint32_t w[16];
-    const uint32_t e0 = mxfp8_quantize32(f, w);
-    const uint32_t e1 = mxfp8_quantize32(f + 32, w + 8);
+    uint32_t sfw = 0;
     uint8_t* dst = codes + (static_cast<int64_t>(e) * rows_per_expert + dst_row) * K + 64 * g;
+#pragma unroll 1
+    for (int b = 0; b < 2; ++b) {
+      float f[32];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+      for (int i = 0; i < 8; ++i) {
+        const float4 v = __ldg(src4 + 8 * b + i);
+        f[4 * i] = v.x;
+        f[4 * i + 1] = v.y;
+        f[4 * i + 2] = v.z;
+        f[4 * i + 3] = v.w;
+      }
+      uint32_t w[8];
+      sfw |= mxfp8_quantize32(f, w) << (8 * b);
+      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * b);
+      d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
     const int64_t nsf = K / 32;
     uint8_t* sfe = sfbuf + static_cast<int64_t>(e) * rows_per_expert * nsf;
-    *reinterpret_cast<uint16_t*>(sfe + sf_offset(dst_row, 2 * g, nsf)) = static_cast<uint16_t>(e0 | (e1 << 8));
+    *reinterpret_cast<uint16_t*>(sfe + sf_offset(dst_row, 2 * g, nsf)) = static_cast<uint16_t>(sfw);
   }
 }
 
