@@ -61,6 +61,7 @@ SIGNATURES = {
     "moe_forward_gateup": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_forward_down": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_unpermute_combine": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P]),
+    "moe_route_topk_noalloc": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -151,6 +152,15 @@ def moe_route_topk(cfg, T, logits, topk_ids, topk_w, expert_counts, expert_offse
         ctypes.byref(cfg), int(T), _p(logits), _p(topk_ids), _p(topk_w), _p(expert_counts), _p(expert_offsets),
         _p(sorted_slots), _p(slot_to_row), _p(workspace), int(workspace.numel() * workspace.element_size()),
         _stream(stream)))
+
+
+def moe_route_topk_noalloc(cfg, T, logits, topk_ids, topk_w, expert_counts, expert_offsets, sorted_slots,
+                           slot_to_row, stream=None):
+    """moe_route_topk without a workspace, for callers that cannot allocate
+    device memory (the library's fixed 4 MiB scratch array is used instead)."""
+    _check("moe_route_topk_noalloc", lib().moe_route_topk_noalloc(
+        ctypes.byref(cfg), int(T), _p(logits), _p(topk_ids), _p(topk_w), _p(expert_counts), _p(expert_offsets),
+        _p(sorted_slots), _p(slot_to_row), _stream(stream)))
 
 
 def moe_permute(cfg, T, x, act_scale, slot_to_row, a_codes, a_sf, stream=None):

@@ -224,6 +224,27 @@ MOE_API moe_status moe_forward_down(const moe_config* cfg, int64_t T, const void
 MOE_API moe_status moe_unpermute_combine(const moe_config* cfg, int64_t T, const void* down_out, const float* topk_w,
                                  const int32_t* slot_to_row, void* y_bf16, void* stream);
 
+/* Routing for callers that cannot allocate device memory (no counterpart on
+ * the source pages; an addition of this library).  Same arguments, results
+ * and guarantees as moe_route_topk, bit for bit, without the workspace: its
+ * scratch is a fixed 4 MiB array compiled into the library, which every GPU
+ * that loads the library keeps until the process exits.  Use it where the
+ * caller has only its input and output buffers, for example a plugin inside
+ * another runtime or a host that plans all device memory once.
+ *   - Limit: moe_route_workspace_bytes(cfg, T) must be <= 4 MiB (for E = 384
+ *     that is up to 69,888 tokens); larger sizes return MOE_ERR_WORKSPACE
+ *     and enqueue nothing.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) for that device; make that first call outside
+ *     any CUDA stream capture.
+ *   - All calls share the one array: calls whose work overlaps on the GPU
+ *     (different streams, or different host threads) race and may return
+ *     wrong results.  Calls on one stream are safe.
+ *   - Calls no allocating routine (no cudaMalloc / cudaFree). */
+MOE_API moe_status moe_route_topk_noalloc(const moe_config* cfg, int64_t T, const float* logits, int32_t* topk_ids,
+                                          float* topk_w, int32_t* expert_counts, int32_t* expert_offsets,
+                                          int32_t* sorted_slots, int32_t* slot_to_row, void* stream);
+
 /* Static description of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
 
