@@ -94,6 +94,24 @@ __device__ __forceinline__ int find_expert(const int32_t* offs, int E, int row) 
   return lo;
 }
 
+// Tile order: expert by expert; inside an expert, weight tile (nt) by weight
+// tile, and the expert's 128-row blocks (mt) fastest.  CTAs running at the same
+// time therefore share one weight tile (read from HBM once, then from L2), and
+// an expert's activation rows are re-read from L2 for each weight tile.
+struct TileCoord {
+  int e, mt, nt, m_blocks;
+};
+__device__ __forceinline__ TileCoord tile_coord(int tile, const int32_t* offs, int E, int n_tiles) {
+  TileCoord c;
+  c.e = find_expert(offs, E, (tile / n_tiles) * kBM);
+  const int mt0 = offs[c.e] / kBM;
+  c.m_blocks = offs[c.e + 1] / kBM - mt0;
+  const int local = tile - mt0 * n_tiles;
+  c.nt = local / c.m_blocks;
+  c.mt = mt0 + local % c.m_blocks;
+  return c;
+}
+
 template <int FMT, bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -143,13 +161,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
+      // weights read by a single row block are streamed once; otherwise they
+      // are reused by the expert's other row blocks and stay in L2
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_normal();
       const uint64_t pol_a = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-        const int mt = tile / n_tiles, nt = tile % n_tiles;
-        const int e = find_expert(s_offsets, E, mt * kBM);
+        const TileCoord tc = tile_coord(tile, s_offsets, E, n_tiles);
+        const int mt = tc.mt, nt = tc.nt, e = tc.e;
+        const uint64_t pol_w = tc.m_blocks > 1 ? pol_keep : pol_stream;
         const uint8_t* a_sf = args.a_sf + static_cast<int64_t>(mt) * args.sf_rb_stride;
         const uint8_t* b_sf = args.b_sf + static_cast<int64_t>(e) * args.b_sf_expert_stride +
                               static_cast<int64_t>(nt) * (kBN / 128) * args.sf_rb_stride;
@@ -251,8 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int I = args.n_rows_b / 2;  // gate/up: channels; unused for down
     const int H = args.n_rows_b;      // down: output channels
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-      const int mt = tile / n_tiles, nt = tile % n_tiles;
-      const int e = find_expert(s_offsets, E, mt * kBM);
+      const TileCoord tc = tile_coord(tile, s_offsets, E, n_tiles);
+      const int mt = tc.mt, nt = tc.nt, e = tc.e;
       const int valid_rows = s_offsets[e] + __ldg(args.counts + e) - mt * kBM;
       const bool valid = row_l < valid_rows;
       const int64_t row = static_cast<int64_t>(mt) * kBM + row_l;

@@ -32,66 +32,45 @@ __device__ __forceinline__ void load16_bf16(const __nv_bfloat16* p, float* f) {
   }
 }
 
-// One warp per token; lane g handles 64-element groups g, g+32, ...
+// One thread per (token, scale block): 16 elements for NVFP4, 32 for MXFP8.
+// The block is read once, quantized once, and its codes and scale are written
+// to each of the token's k rows.
 template <int FMT>
-__global__ void __launch_bounds__(128) permute_kernel(int T, int H, int k, const __nv_bfloat16* __restrict__ x,
+__global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const __nv_bfloat16* __restrict__ x,
                                                       const float* __restrict__ act_scale,
                                                       const int32_t* __restrict__ slot_to_row,
                                                       uint8_t* __restrict__ a_codes, uint8_t* __restrict__ a_sf) {
-  const int t = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
-  const int groups = H / 64;
-  const float s_x = (FMT == MOE_NVFP4) ? __ldg(act_scale) : 1.0f;
-  int32_t rows[8];
+  constexpr int kBlock = (FMT == MOE_NVFP4) ? 16 : 32;
+  const int nsf = H / kBlock;
+  const int64_t id = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (id >= static_cast<int64_t>(T) * nsf) return;
+  const int t = static_cast<int>(id / nsf);
+  const int b = static_cast<int>(id % nsf);
+  const __nv_bfloat16* src = x + static_cast<int64_t>(t) * H + kBlock * b;
+  float f[kBlock];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) rows[j] = (j < k) ? __ldg(slot_to_row + static_cast<int64_t>(t) * k + j) : 0;
-  for (int g = lane; g < groups; g += 32) {
-    const __nv_bfloat16* src = x + static_cast<int64_t>(t) * H + 64 * g;
-    if (FMT == MOE_NVFP4) {
-      const int64_t nsf = H / 16;
-      uint32_t sfw = 0;
-#pragma unroll 1
-      for (int b = 0; b < 4; ++b) {
-        float f[16];
-        load16_bf16(src + 16 * b, f);
-        const Nvfp4Block q = nvfp4_quantize16(f, s_x);
-        sfw |= q.sf << (8 * b);
-        const uint2 c = make_uint2(static_cast<uint32_t>(q.codes), static_cast<uint32_t>(q.codes >> 32));
+  for (int i = 0; i < kBlock / 16; ++i) load16_bf16(src + 16 * i, f + 16 * i);
+  if (FMT == MOE_NVFP4) {
+    const Nvfp4Block q = nvfp4_quantize16(f, __ldg(act_scale));
+    const uint2 c = make_uint2(static_cast<uint32_t>(q.codes), static_cast<uint32_t>(q.codes >> 32));
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j >= k) break;
-          *reinterpret_cast<uint2*>(a_codes + static_cast<int64_t>(rows[j]) * (H / 2) + 32 * g + 8 * b) = c;
-        }
-      }
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) break;
+      const int64_t r = __ldg(slot_to_row + static_cast<int64_t>(t) * k + j);
+      *reinterpret_cast<uint2*>(a_codes + r * (H / 2) + 8 * b) = c;
+      a_sf[sf_offset(r, b, nsf)] = static_cast<uint8_t>(q.sf);
+    }
+  } else {
+    uint32_t w[8];
+    const uint32_t e = mxfp8_quantize32(f, w);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j >= k) break;
-        *reinterpret_cast<uint32_t*>(a_sf + sf_offset(rows[j], 4 * g, nsf)) = sfw;
-      }
-    } else {
-      const int64_t nsf = H / 32;
-      uint32_t sfw = 0;
-#pragma unroll 1
-      for (int b = 0; b < 2; ++b) {
-        float f[32];
-        load16_bf16(src + 32 * b, f);
-        load16_bf16(src + 32 * b + 16, f + 16);
-        uint32_t w[8];
-        sfw |= mxfp8_quantize32(f, w) << (8 * b);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j >= k) break;
-          uint4* dst = reinterpret_cast<uint4*>(a_codes + static_cast<int64_t>(rows[j]) * H + 64 * g + 32 * b);
-          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j >= k) break;
-        *reinterpret_cast<uint16_t*>(a_sf + sf_offset(rows[j], 2 * g, nsf)) = static_cast<uint16_t>(sfw);
-      }
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) break;
+      const int64_t r = __ldg(slot_to_row + static_cast<int64_t>(t) * k + j);
+      uint4* dst = reinterpret_cast<uint4*>(a_codes + r * H + 32 * b);
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      a_sf[sf_offset(r, b, nsf)] = static_cast<uint8_t>(e);
     }
   }
 }
@@ -99,7 +78,8 @@ __global__ void __launch_bounds__(128) permute_kernel(int T, int H, int k, const
 cudaError_t launch_permute(int fmt, int T, int H, int k, const void* x, const float* act_scale,
                            const int32_t* slot_to_row, uint8_t* a_codes, uint8_t* a_sf, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  const dim3 grid((T + 3) / 4), block(128);
+  const int64_t n = static_cast<int64_t>(T) * (H / (fmt == MOE_NVFP4 ? 16 : 32));
+  const dim3 grid(static_cast<unsigned>((n + 255) / 256)), block(256);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (fmt == MOE_NVFP4)
     permute_kernel<MOE_NVFP4><<<grid, block, 0, stream>>>(T, H, k, xb, act_scale, slot_to_row, a_codes, a_sf);

@@ -49,7 +49,159 @@ __device__ __forceinline__ float exp_own(float x) {
 }
 
 constexpr int kChunk = 128;       // tokens per CTA in the top-k kernel
-constexpr int kTopkWarps = 8;
+constexpr int kTopkWarps = 32;
+constexpr int kSmallT = 1024;     // batches up to this size take the one-CTA path
+
+// Top-k of one token's logits by k warp-wide arg-max rounds, then the softmax.
+// Every lane ends with the same sel_i / w for j < k.
+template <int NPL>
+__device__ __forceinline__ void topk_token(const float* __restrict__ row, int E, int k, int lane, int* sel_i,
+                                           float* w) {
+  float v[NPL];
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = (e < E) ? __ldg(row + e) : -INFINITY;
+  }
+  uint32_t taken = 0u;
+  float sel_v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j >= k) break;
+    float bv = -INFINITY;
+    int bi = 0x7FFFFFFF;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      // strict '>' keeps the lower index among equal values of this lane
+      if (e < E && !((taken >> i) & 1u) && (v[i] > bv || bi == 0x7FFFFFFF)) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+      const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
+      if (oi != 0x7FFFFFFF && (bi == 0x7FFFFFFF || ov > bv || (ov == bv && oi < bi))) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    sel_v[j] = bv;
+    sel_i[j] = bi;
+  }
+  // softmax over the selected logits, in rank order
+  float ex[8];
+  float s = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j >= k) break;
+    ex[j] = exp_own(__fsub_rn(sel_v[j], sel_v[0]));
+    s = (j == 0) ? ex[0] : __fadd_rn(s, ex[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j >= k) break;
+    w[j] = __fdiv_rn(ex[j], s);
+  }
+}
+
+// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024).
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_sums, int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t ws = (lane < static_cast<int>(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xFFFFFFFFu, ws, off);
+      if (lane >= off) ws += o;
+    }
+    warp_sums[lane] = ws;
+  }
+  __syncthreads();
+  *total = warp_sums[(blockDim.x >> 5) - 1];
+  return incl - v + (warp > 0 ? warp_sums[warp - 1] : 0);
+}
+
+// The whole routing step for T <= kSmallT in one CTA of 1024 threads: no
+// workspace, no memset.  Token bitmaps per expert live in shared memory
+// ([E][W] words, W = ceil(T / 32)), so slot ranks are popc counts and do not
+// depend on thread timing.
+template <int NPL>
+__global__ void __launch_bounds__(1024) route_small_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                           int R_max, int32_t* __restrict__ topk_ids,
+                                                           float* __restrict__ topk_w,
+                                                           int32_t* __restrict__ expert_counts,
+                                                           int32_t* __restrict__ expert_offsets,
+                                                           int32_t* __restrict__ sorted_slots,
+                                                           int32_t* __restrict__ slot_to_row) {
+  extern __shared__ uint32_t sm[];
+  const int W = (T + 31) / 32;
+  uint32_t* bitmap = sm;                                   // [E][W]
+  int32_t* s_off = reinterpret_cast<int32_t*>(sm + E * W);  // [E + 1]
+  int32_t* s_cnt = s_off + E + 1;                          // [E]
+  __shared__ int32_t warp_sums[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < E * W; i += blockDim.x) bitmap[i] = 0u;
+  __syncthreads();
+  for (int t = warp; t < T; t += 32) {
+    int sel_i[8];
+    float w[8];
+    topk_token<NPL>(logits + static_cast<int64_t>(t) * E, E, k, lane, sel_i, w);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) break;
+      if (lane == j) {
+        topk_ids[static_cast<int64_t>(t) * k + j] = sel_i[j];
+        topk_w[static_cast<int64_t>(t) * k + j] = w[j];
+        atomicOr(&bitmap[sel_i[j] * W + (t >> 5)], 1u << (t & 31));
+      }
+    }
+  }
+  __syncthreads();
+  int32_t cnt = 0;
+  const int e = threadIdx.x;
+  if (e < E)
+    for (int i = 0; i < W; ++i) cnt += __popc(bitmap[e * W + i]);
+  const int32_t padded = ((cnt + 127) / 128) * 128;
+  int32_t total = 0;
+  const int32_t off = block_exclusive_scan(e < E ? padded : 0, warp_sums, &total);
+  if (e < E) {
+    s_off[e] = off;
+    s_cnt[e] = cnt;
+    expert_counts[e] = cnt;
+    expert_offsets[e] = off;
+  }
+  if (threadIdx.x == 0) {
+    s_off[E] = total;
+    expert_offsets[E] = total;
+  }
+  __syncthreads();
+  for (int s = threadIdx.x; s < T * k; s += blockDim.x) {
+    const int t = s / k;
+    const int ex = topk_ids[s];
+    const uint32_t* bm = bitmap + ex * W;
+    int rank = __popc(bm[t >> 5] & ((1u << (t & 31)) - 1u));
+    for (int i = 0; i < (t >> 5); ++i) rank += __popc(bm[i]);
+    const int32_t row = s_off[ex] + rank;
+    sorted_slots[row] = s;
+    slot_to_row[s] = row;
+  }
+  // padding rows of every expert, and every row past the last expert
+  if (e < E)
+    for (int r = s_off[e] + s_cnt[e]; r < s_off[e + 1]; ++r) sorted_slots[r] = -1;
+  for (int r = total + threadIdx.x; r < R_max; r += blockDim.x) sorted_slots[r] = -1;
+}
 
 // NPL = logits per lane (ceil(E / 32)).
 template <int NPL>
@@ -67,56 +219,15 @@ __global__ void __launch_bounds__(kTopkWarps * 32) route_topk_kernel(const float
   for (int tl = warp; tl < kChunk; tl += kTopkWarps) {
     const int t = chunk * kChunk + tl;
     if (t >= T) break;
-    const float* row = logits + static_cast<int64_t>(t) * E;
-    float v[NPL];
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
-      v[i] = (e < E) ? __ldg(row + e) : -INFINITY;
-    }
-    uint32_t taken = 0u;
-    float sel_v[8];
     int sel_i[8];
-#pragma unroll 1
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7FFFFFFF;
+    float w[8];
+    topk_token<NPL>(logits + static_cast<int64_t>(t) * E, E, k, lane, sel_i, w);
 #pragma unroll
-      for (int i = 0; i < NPL; ++i) {
-        const int e = lane + 32 * i;
-        // strict '>' keeps the lower index among equal values of this lane
-        if (e < E && !((taken >> i) & 1u) && (v[i] > bv || bi == 0x7FFFFFFF)) {
-          bv = v[i];
-          bi = e;
-        }
-      }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
-        if (oi != 0x7FFFFFFF && (bi == 0x7FFFFFFF || ov > bv || (ov == bv && oi < bi))) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      sel_v[j] = bv;
-      sel_i[j] = bi;
-    }
-    // softmax over the selected logits, in rank order (every lane computes it)
-    float ex[8];
-    float s = 0.0f;
-    const float m = sel_v[0];
-#pragma unroll 1
-    for (int j = 0; j < k; ++j) {
-      ex[j] = exp_own(__fsub_rn(sel_v[j], m));
-      s = (j == 0) ? ex[0] : __fadd_rn(s, ex[j]);
-    }
-#pragma unroll 1
-    for (int j = 0; j < k; ++j) {
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) break;
       if (lane == j) {
         topk_ids[static_cast<int64_t>(t) * k + j] = sel_i[j];
-        topk_w[static_cast<int64_t>(t) * k + j] = __fdiv_rn(ex[j], s);
+        topk_w[static_cast<int64_t>(t) * k + j] = w[j];
         atomicOr(&bitmap[sel_i[j] * 4 + (tl >> 5)], 1u << (tl & 31));
       }
     }
@@ -206,6 +317,36 @@ int64_t route_workspace_bytes(int E, int64_t T) {
 cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w,
                          int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
                          int32_t* slot_to_row, int64_t R_max, void* workspace, cudaStream_t stream) {
+  const int npl_small = (E + 31) / 32;
+  if (T > 0 && T <= kSmallT) {
+    const int W = (T + 31) / 32;
+    const size_t smem = static_cast<size_t>(E) * W * 4 + (2 * static_cast<size_t>(E) + 1) * 4;
+    static bool configured[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !configured[dev]) {
+      const int max_smem = 1024 * 32 * 4 + (2 * 1024 + 1) * 4;
+      cudaFuncSetAttribute(route_small_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+      cudaFuncSetAttribute(route_small_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+      cudaFuncSetAttribute(route_small_kernel<12>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+      cudaFuncSetAttribute(route_small_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+      if (dev < 64) configured[dev] = true;
+    }
+    const int R = static_cast<int>(R_max);
+    if (npl_small <= 1)
+      route_small_kernel<1><<<1, 1024, smem, stream>>>(logits, T, E, k, R, topk_ids, topk_w, expert_counts,
+                                                        expert_offsets, sorted_slots, slot_to_row);
+    else if (npl_small <= 4)
+      route_small_kernel<4><<<1, 1024, smem, stream>>>(logits, T, E, k, R, topk_ids, topk_w, expert_counts,
+                                                        expert_offsets, sorted_slots, slot_to_row);
+    else if (npl_small <= 12)
+      route_small_kernel<12><<<1, 1024, smem, stream>>>(logits, T, E, k, R, topk_ids, topk_w, expert_counts,
+                                                         expert_offsets, sorted_slots, slot_to_row);
+    else
+      route_small_kernel<32><<<1, 1024, smem, stream>>>(logits, T, E, k, R, topk_ids, topk_w, expert_counts,
+                                                         expert_offsets, sorted_slots, slot_to_row);
+    return cudaGetLastError();
+  }
   const int nchunks = (T + kChunk - 1) / kChunk;
   uint32_t* ws_bitmap = static_cast<uint32_t*>(workspace);
   int32_t* ws_counts = reinterpret_cast<int32_t*>(ws_bitmap + static_cast<int64_t>(nchunks) * E * 4);
