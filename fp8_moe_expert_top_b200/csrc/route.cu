@@ -149,7 +149,6 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restri
   const int W = (T + 31) / 32;
   uint32_t* bitmap = sm;                                   // [E][W]
   int32_t* s_off = reinterpret_cast<int32_t*>(sm + E * W);  // [E + 1]
-  int32_t* s_cnt = s_off + E + 1;                          // [E]
   __shared__ int32_t warp_sums[32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < E * W; i += blockDim.x) bitmap[i] = 0u;
@@ -178,7 +177,6 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restri
   const int32_t off = block_exclusive_scan(e < E ? padded : 0, warp_sums, &total);
   if (e < E) {
     s_off[e] = off;
-    s_cnt[e] = cnt;
     expert_counts[e] = cnt;
     expert_offsets[e] = off;
   }
@@ -186,6 +184,8 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restri
     s_off[E] = total;
     expert_offsets[E] = total;
   }
+  // every row starts as padding (coalesced), then the slots overwrite theirs
+  for (int r = threadIdx.x; r < R_max; r += blockDim.x) sorted_slots[r] = -1;
   __syncthreads();
   for (int s = threadIdx.x; s < T * k; s += blockDim.x) {
     const int t = s / k;
@@ -197,10 +197,6 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restri
     sorted_slots[row] = s;
     slot_to_row[s] = row;
   }
-  // padding rows of every expert, and every row past the last expert
-  if (e < E)
-    for (int r = s_off[e] + s_cnt[e]; r < s_off[e + 1]; ++r) sorted_slots[r] = -1;
-  for (int r = total + threadIdx.x; r < R_max; r += blockDim.x) sorted_slots[r] = -1;
 }
 
 // NPL = logits per lane (ceil(E / 32)).
@@ -320,7 +316,7 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
   const int npl_small = (E + 31) / 32;
   if (T > 0 && T <= kSmallT) {
     const int W = (T + 31) / 32;
-    const size_t smem = static_cast<size_t>(E) * W * 4 + (2 * static_cast<size_t>(E) + 1) * 4;
+    const size_t smem = static_cast<size_t>(E) * W * 4 + (static_cast<size_t>(E) + 1) * 4;
     static bool configured[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);

@@ -89,6 +89,44 @@ class ExpertLayer:
     def combine(self, T):
         B.moe_unpermute_combine(self.cfg, T, self.down_out, self.topk_w, self.slot_to_row, self.y)
 
+    # ------------------------------------------------------------- graphs
+    def capture(self, T, events=None):
+        """Capture the whole layer for T tokens as a CUDA graph.
+
+        The graph reads its inputs from self.x_in [T_max, H] (bf16) and
+        self.logits_in [T_max, E] (float32) and writes self.y.  `events`, if
+        given, is a list of six timing events created with external=True; they
+        are recorded before the layer and after each of its five steps.  Run
+        one eager forward first so that every kernel is set up.
+        """
+        if getattr(self, "x_in", None) is None:
+            self.x_in = torch.zeros(self.T_max, self.H, dtype=torch.bfloat16, device=self.device)
+            self.logits_in = torch.zeros(self.T_max, self.E, dtype=torch.float32, device=self.device)
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        steps = (lambda: self.route(self.logits_in, T), lambda: self.permute(self.x_in, T),
+                 lambda: self.gateup(T), lambda: self.down(T), lambda: self.combine(T))
+        with torch.cuda.graph(g, stream=side):
+            if events is not None:
+                events[0].record()
+            for i, fn in enumerate(steps):
+                fn()
+                if events is not None:
+                    events[i + 1].record()
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        self._graph_T = T
+        return g
+
+    def forward_graph(self, graph, x, logits):
+        """Copy x / logits into the graph's input buffers and replay it."""
+        T = self._graph_T
+        assert x.shape[0] == T and logits.shape[0] == T
+        self.x_in[:T].copy_(x, non_blocking=True)
+        self.logits_in[:T].copy_(logits, non_blocking=True)
+        graph.replay()
+        return self.y[:T]
+
     def forward(self, x, logits):
         """y[:T] for bf16 x [T, H] and float32 logits [T, E] already on the device."""
         T = x.shape[0]

@@ -137,3 +137,21 @@ def test_empty_batch(cuda_device):
     torch.cuda.synchronize()
     assert y.shape == (0, TINY.d_model)
     assert int(layer.expert_offsets[-1].item()) == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl", [TINY, TINY_MX], ids=lambda w: w.name)
+def test_cuda_graph_replay_matches_eager(cuda_device, wl):
+    """The layer captured as one CUDA graph gives the eager results bit for bit."""
+    layer = get_layer(wl, cuda_device)
+    x, lg = inputs.make_x(wl, seed=31).to(cuda_device), inputs.make_logits(wl, seed=32).to(cuda_device)
+    y_eager = layer.forward(x, lg).clone()
+    h_eager = layer.h_codes.clone()
+    torch.cuda.synchronize()
+    g = layer.capture(wl.T)
+    for _ in range(2):
+        layer.y.zero_()
+        y_graph = layer.forward_graph(g, x, lg)
+        torch.cuda.synchronize()
+        assert torch.equal(y_graph.view(torch.int16), y_eager.view(torch.int16))
+    assert torch.equal(layer.h_codes, h_eager)
