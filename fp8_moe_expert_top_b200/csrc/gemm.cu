@@ -114,8 +114,8 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const int32_t* offs, i
 
 template <int FMT, bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
-    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                    const GemmArgs args) {
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_a16,
+                    const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
   using Tr = GemmTraits<FMT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmap_a);
+    prefetch_tensormap(&tmap_a16);
     prefetch_tensormap(&tmap_b);
   }
   if (warp == 1) {
@@ -176,6 +177,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint8_t* b_sf = args.b_sf + static_cast<int64_t>(e) * args.b_sf_expert_stride +
                               static_cast<int64_t>(nt) * (kBN / 128) * args.sf_rb_stride;
         const int b_row = e * args.n_rows_b + nt * kBN;
+        // Only the row block's valid rows are loaded, in 16-row boxes; the
+        // rest of the A tile keeps stale data, whose output rows are never
+        // stored (each output row depends only on its own A row).
+        const int valid_rows = min(kBM, s_offsets[e] + __ldg(args.counts + e) - mt * kBM);
+        const int a_boxes = (valid_rows + 15) / 16;
+        const uint32_t a_bytes = (a_boxes == kBM / 16) ? Tr::kABytes : a_boxes * 16 * kRowBytesPerStage;
         for (int kt = 0; kt < k_tiles; ++kt) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
             fail_bits |= MOE_DEVICE_TIMEOUT_PRODUCER;
@@ -184,8 +191,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
           const uint32_t sf_bytes = (FMT == MOE_NVFP4) ? 512u * kb_here : 512u;
           uint8_t* st = smem + stage * Tr::kStageBytes;
-          mbar_arrive_expect_tx(&full_bar[stage], Tr::kABytes + Tr::kBBytes + sf_bytes * (1 + kBN / 128));
-          tma_load_2d(st, &tmap_a, kt * kRowBytesPerStage, mt * kBM, &full_bar[stage], pol_a);
+          mbar_arrive_expect_tx(&full_bar[stage], a_bytes + Tr::kBBytes + sf_bytes * (1 + kBN / 128));
+          if (a_boxes == kBM / 16) {
+            tma_load_2d(st, &tmap_a, kt * kRowBytesPerStage, mt * kBM, &full_bar[stage], pol_a);
+          } else {
+            for (int i = 0; i < a_boxes; ++i)
+              tma_load_2d(st + i * 16 * kRowBytesPerStage, &tmap_a16, kt * kRowBytesPerStage, mt * kBM + 16 * i,
+                          &full_bar[stage], pol_a);
+          }
           tma_load_2d(st + Tr::kABytes, &tmap_b, kt * kRowBytesPerStage, b_row, &full_bar[stage], pol_w);
           bulk_load(st + Tr::kSfaOff, a_sf + kt * Tr::kSfBytes128, sf_bytes, &full_bar[stage], pol_a);
 #pragma unroll
@@ -411,7 +424,8 @@ static bool make_map(CUtensorMap* map, const void* base, int64_t row_bytes, int6
 }
 
 template <int FMT, bool GATEUP>
-static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& a, cudaStream_t stream) {
+static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& ma16, const CUtensorMap& mb, const GemmArgs& a,
+                              cudaStream_t stream) {
   using Tr = GemmTraits<FMT>;
   const size_t smem = 1024 + kStages * Tr::kStageBytes + (2 * kStages + 2) * 8 + 16 + (a.E + 1) * 4;
   int dev = 0;
@@ -429,7 +443,7 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, cons
   int sms = 0;
   err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (err != cudaSuccess) return err;
-  moe_gemm_kernel<FMT, GATEUP><<<sms, kThreads, smem, stream>>>(ma, mb, a);
+  moe_gemm_kernel<FMT, GATEUP><<<sms, kThreads, smem, stream>>>(ma, ma16, mb, a);
   return cudaGetLastError();
 }
 
@@ -442,8 +456,9 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
   const int bits = (g.fmt == MOE_NVFP4) ? 4 : 8;
   const int sfvec = (g.fmt == MOE_NVFP4) ? 16 : 32;
   const int64_t row_bytes = static_cast<int64_t>(g.K) * bits / 8;
-  CUtensorMap ma, mb;
+  CUtensorMap ma, ma16, mb;
   if (!make_map(&ma, g.a_codes, row_bytes, g.R_max, kBM)) return cudaErrorInvalidValue;
+  if (!make_map(&ma16, g.a_codes, row_bytes, g.R_max, 16)) return cudaErrorInvalidValue;
   if (!make_map(&mb, g.b_codes, row_bytes, static_cast<int64_t>(g.E) * g.n_rows_b, kBN)) return cudaErrorInvalidValue;
   GemmArgs a;
   a.a_sf = g.a_sf;
@@ -464,8 +479,10 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
   a.sf_rb_stride = static_cast<int64_t>(g.K / sfvec) * 128;
   a.b_sf_expert_stride = static_cast<int64_t>(g.n_rows_b) * (g.K / sfvec);
   if (g.fmt == MOE_NVFP4)
-    return g.gateup ? launch_one<MOE_NVFP4, true>(ma, mb, a, stream) : launch_one<MOE_NVFP4, false>(ma, mb, a, stream);
-  return g.gateup ? launch_one<MOE_MXFP8, true>(ma, mb, a, stream) : launch_one<MOE_MXFP8, false>(ma, mb, a, stream);
+    return g.gateup ? launch_one<MOE_NVFP4, true>(ma, ma16, mb, a, stream)
+                    : launch_one<MOE_NVFP4, false>(ma, ma16, mb, a, stream);
+  return g.gateup ? launch_one<MOE_MXFP8, true>(ma, ma16, mb, a, stream)
+                  : launch_one<MOE_MXFP8, false>(ma, ma16, mb, a, stream);
 }
 
 }  // namespace moe

@@ -1,7 +1,7 @@
 // Routing without a caller-provided workspace.
 //
-// moe_route_topk needs scratch device memory (per-chunk token bitmaps and
-// counts).  Some callers cannot hand it any: a plugin inside another runtime
+// moe_route_topk needs scratch device memory (per-expert token bitmaps and
+// their prefix counts).  Some callers cannot hand it any: a plugin inside another runtime
 // that only receives its input and output tensors, a real-time or embedded
 // host whose device memory is planned once up front, or a caller that may not
 // touch the allocator at that point.  moe_route_topk_noalloc serves them by

@@ -232,7 +232,7 @@ MOE_API moe_status moe_unpermute_combine(const moe_config* cfg, int64_t T, const
  * caller has only its input and output buffers, for example a plugin inside
  * another runtime or a host that plans all device memory once.
  *   - Limit: moe_route_workspace_bytes(cfg, T) must be <= 4 MiB (for E = 384
- *     that is up to 69,888 tokens); larger sizes return MOE_ERR_WORKSPACE
+ *     that is up to 43,680 tokens); larger sizes return MOE_ERR_WORKSPACE
  *     and enqueue nothing.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) for that device; make that first call outside
