@@ -22,6 +22,7 @@ FORMATS = {"nvfp4": MOE_NVFP4, "mxfp8": MOE_MXFP8}
 MOE_DEVICE_TIMEOUT_PRODUCER = 0x1
 MOE_DEVICE_TIMEOUT_MMA = 0x2
 MOE_DEVICE_TIMEOUT_EPILOGUE = 0x4
+MOE_DEVICE_TIMEOUT_SELFTEST = 0x8
 
 
 class MoeError(RuntimeError):
@@ -62,6 +63,7 @@ SIGNATURES = {
     "moe_forward_down": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_unpermute_combine": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P]),
     "moe_route_topk_noalloc": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_selftest_bounded_wait": (ctypes.c_int, [_P, _I64, _P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -194,3 +196,8 @@ def moe_forward_down(cfg, T, packed, h_codes, h_sf, inter_scale, expert_offsets,
 def moe_unpermute_combine(cfg, T, down_out, topk_w, slot_to_row, y, stream=None):
     _check("moe_unpermute_combine", lib().moe_unpermute_combine(
         ctypes.byref(cfg), int(T), _p(down_out), _p(topk_w), _p(slot_to_row), _p(y), _stream(stream)))
+
+
+def moe_selftest_bounded_wait(status_word, limit_ns, stream=None):
+    _check("moe_selftest_bounded_wait", lib().moe_selftest_bounded_wait(_p(status_word), int(limit_ns),
+                                                                        _stream(stream)))

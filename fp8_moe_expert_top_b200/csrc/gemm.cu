@@ -147,6 +147,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  // everything above overlaps the previous kernel; from here on its outputs are read
+  pdl_wait();
+  pdl_trigger();
   for (int i = threadIdx.x; i <= E; i += kThreads) s_offsets[i] = args.offsets[i];
   tc_fence_before();
   __syncthreads();
@@ -443,8 +446,7 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& ma16, co
   int sms = 0;
   err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (err != cudaSuccess) return err;
-  moe_gemm_kernel<FMT, GATEUP><<<sms, kThreads, smem, stream>>>(ma, ma16, mb, a);
-  return cudaGetLastError();
+  return launch_pdl(moe_gemm_kernel<FMT, GATEUP>, dim3(sms), dim3(kThreads), smem, stream, ma, ma16, mb, a);
 }
 
 size_t gemm_smem_bytes(int fmt, int E) {

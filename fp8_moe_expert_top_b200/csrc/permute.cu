@@ -43,6 +43,8 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
   constexpr int kBlock = (FMT == MOE_NVFP4) ? 16 : 32;
   const int nsf = H / kBlock;
   const int64_t id = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (id >= static_cast<int64_t>(T) * nsf) return;
   const int t = static_cast<int>(id / nsf);
   const int b = static_cast<int>(id % nsf);
@@ -82,10 +84,10 @@ cudaError_t launch_permute(int fmt, int T, int H, int k, const void* x, const fl
   const dim3 grid(static_cast<unsigned>((n + 255) / 256)), block(256);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (fmt == MOE_NVFP4)
-    permute_kernel<MOE_NVFP4><<<grid, block, 0, stream>>>(T, H, k, xb, act_scale, slot_to_row, a_codes, a_sf);
-  else
-    permute_kernel<MOE_MXFP8><<<grid, block, 0, stream>>>(T, H, k, xb, act_scale, slot_to_row, a_codes, a_sf);
-  return cudaGetLastError();
+    return launch_pdl(permute_kernel<MOE_NVFP4>, grid, block, 0, stream, T, H, k, xb, act_scale, slot_to_row, a_codes,
+                      a_sf);
+  return launch_pdl(permute_kernel<MOE_MXFP8>, grid, block, 0, stream, T, H, k, xb, act_scale, slot_to_row, a_codes,
+                    a_sf);
 }
 
 // y[t] = sum_j w[t][j] * out[row(t, j)], float32 in rank order, then bf16.
@@ -95,6 +97,8 @@ __global__ void __launch_bounds__(256) combine_kernel(int H, int k, const __nv_b
                                                       const int32_t* __restrict__ slot_to_row,
                                                       __nv_bfloat16* __restrict__ y) {
   const int t = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   float w[8];
   int64_t rows[8];
 #pragma unroll
@@ -130,9 +134,8 @@ __global__ void __launch_bounds__(256) combine_kernel(int H, int k, const __nv_b
 cudaError_t launch_combine(int T, int H, int k, const void* down_out, const float* topk_w,
                            const int32_t* slot_to_row, void* y, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  combine_kernel<<<T, 256, 0, stream>>>(H, k, static_cast<const __nv_bfloat16*>(down_out), topk_w, slot_to_row,
-                                        static_cast<__nv_bfloat16*>(y));
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(T), dim3(256), 0, stream, H, k,
+                    static_cast<const __nv_bfloat16*>(down_out), topk_w, slot_to_row, static_cast<__nv_bfloat16*>(y));
 }
 
 }  // namespace moe

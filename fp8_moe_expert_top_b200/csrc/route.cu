@@ -113,6 +113,8 @@ __global__ void __launch_bounds__(kTopkWarps * 32) route_topk_kernel(const float
                                                                      uint32_t* __restrict__ bitmap) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTopkWarps + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_trigger();
   if (t >= T) return;
   int sel_i[8];
   float w;
@@ -163,6 +165,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int E, int W, const ui
   __shared__ int32_t s_count[1024];
   __shared__ int32_t warp_sums[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
   for (int e = warp; e < E; e += 32) {
     const uint32_t* bm = bitmap + static_cast<int64_t>(e) * W;
     int32_t* pf = prefix + static_cast<int64_t>(e) * W;
@@ -198,6 +202,8 @@ __global__ void route_scatter_kernel(int T, int E, int k, int W, const int32_t* 
                                      const int32_t* __restrict__ expert_offsets, int32_t* __restrict__ sorted_slots,
                                      int32_t* __restrict__ slot_to_row) {
   const int64_t s = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (s >= static_cast<int64_t>(T) * k) return;
   const int t = static_cast<int>(s / k);
   const int e = topk_ids[s];
@@ -230,23 +236,24 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
   if (err != cudaSuccess) return err;
   const int npl = (E + 31) / 32;
   const dim3 grid((T + kTopkWarps - 1) / kTopkWarps), block(kTopkWarps * 32);
+  const float* lg = logits;
   if (npl <= 1)
-    route_topk_kernel<1><<<grid, block, 0, stream>>>(logits, T, E, k, W, topk_ids, topk_w, bitmap);
+    err = launch_pdl(route_topk_kernel<1>, grid, block, 0, stream, lg, T, E, k, W, topk_ids, topk_w, bitmap);
   else if (npl <= 4)
-    route_topk_kernel<4><<<grid, block, 0, stream>>>(logits, T, E, k, W, topk_ids, topk_w, bitmap);
+    err = launch_pdl(route_topk_kernel<4>, grid, block, 0, stream, lg, T, E, k, W, topk_ids, topk_w, bitmap);
   else if (npl <= 12)
-    route_topk_kernel<12><<<grid, block, 0, stream>>>(logits, T, E, k, W, topk_ids, topk_w, bitmap);
+    err = launch_pdl(route_topk_kernel<12>, grid, block, 0, stream, lg, T, E, k, W, topk_ids, topk_w, bitmap);
   else
-    route_topk_kernel<32><<<grid, block, 0, stream>>>(logits, T, E, k, W, topk_ids, topk_w, bitmap);
-  err = cudaGetLastError();
+    err = launch_pdl(route_topk_kernel<32>, grid, block, 0, stream, lg, T, E, k, W, topk_ids, topk_w, bitmap);
   if (err != cudaSuccess) return err;
-  route_scan_kernel<<<1, 1024, 0, stream>>>(E, W, bitmap, prefix, expert_counts, expert_offsets);
-  err = cudaGetLastError();
+  err = launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, stream, E, W, static_cast<const uint32_t*>(bitmap),
+                   prefix, expert_counts, expert_offsets);
   if (err != cudaSuccess) return err;
   const int64_t slots = static_cast<int64_t>(T) * k;
-  route_scatter_kernel<<<static_cast<unsigned>((slots + 255) / 256), 256, 0, stream>>>(
-      T, E, k, W, topk_ids, bitmap, prefix, expert_offsets, sorted_slots, slot_to_row);
-  return cudaGetLastError();
+  return launch_pdl(route_scatter_kernel, dim3(static_cast<unsigned>((slots + 255) / 256)), dim3(256), 0, stream, T,
+                    E, k, W, static_cast<const int32_t*>(topk_ids), static_cast<const uint32_t*>(bitmap),
+                    static_cast<const int32_t*>(prefix), static_cast<const int32_t*>(expert_offsets), sorted_slots,
+                    slot_to_row);
 }
 
 }  // namespace moe

@@ -86,6 +86,7 @@ typedef struct {
 #define MOE_DEVICE_TIMEOUT_PRODUCER 0x1u
 #define MOE_DEVICE_TIMEOUT_MMA 0x2u
 #define MOE_DEVICE_TIMEOUT_EPILOGUE 0x4u
+#define MOE_DEVICE_TIMEOUT_SELFTEST 0x8u
 
 /* Layout of the packed expert weights (byte offsets from the buffer start).
  * For NVFP4 (bits = 4, sfvec = 16) and MXFP8 (bits = 8, sfvec = 32):
@@ -244,6 +245,14 @@ MOE_API moe_status moe_unpermute_combine(const moe_config* cfg, int64_t T, const
 MOE_API moe_status moe_route_topk_noalloc(const moe_config* cfg, int64_t T, const float* logits, int32_t* topk_ids,
                                           float* topk_w, int32_t* expert_counts, int32_t* expert_offsets,
                                           int32_t* sorted_slots, int32_t* slot_to_row, void* stream);
+
+/* Failure-detection self-test (diagnostic; no counterpart on the pages):
+ * enqueues one CTA that waits, with the same bounded mbarrier wait the GEMM
+ * roles use, on a barrier that nothing ever arrives at.  The wait gives up
+ * after limit_ns nanoseconds (1 us .. 5 s) and sets
+ * MOE_DEVICE_TIMEOUT_SELFTEST in *status_word (device uint32).  The kernel
+ * then returns normally: no trap, no fault, the context stays usable. */
+MOE_API moe_status moe_selftest_bounded_wait(uint32_t* status_word, int64_t limit_ns, void* stream);
 
 /* Static description of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
