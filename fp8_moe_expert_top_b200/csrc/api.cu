@@ -24,7 +24,7 @@ moe_status check(const moe_config* c) {
   if (c->top_k < 1 || c->top_k > 8 || c->top_k > c->num_experts) return MOE_ERR_UNSUPPORTED;
   if (c->d_model < 256 || c->d_model % 256 != 0) return MOE_ERR_UNSUPPORTED;
   if (c->d_ffn < 128 || c->d_ffn % 128 != 0) return MOE_ERR_UNSUPPORTED;
-  // weight rows of all experts must be addressable by a 32-bit TMA coordinate
+  // row indices of all experts' weights stay within int32
   if (static_cast<int64_t>(c->num_experts) * 2 * c->d_ffn >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(c->num_experts) * c->d_model >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
@@ -47,11 +47,11 @@ void layout(const moe_config* c, moe_weights_layout* L) {
   auto up256 = [](int64_t x) { return (x + 255) / 256 * 256; };
   int64_t off = 0;
   L->w13_codes = off;
-  off = up256(off + E * 2 * I * H * b / 8);
+  off = up256(off + E * 2 * I * moe::kb_padded(H, b));
   L->w13_sf = off;
   off = up256(off + E * 2 * I * H / v);
   L->w2_codes = off;
-  off = up256(off + E * H * I * b / 8);
+  off = up256(off + E * H * moe::kb_padded(I, b));
   L->w2_sf = off;
   off = up256(off + E * H * I / v);
   L->scales = off;
@@ -79,8 +79,8 @@ int64_t moe_max_rows(const moe_config* cfg, int64_t T) {
 }
 
 int64_t moe_codes_bytes(const moe_config* cfg, int64_t rows, int64_t K) {
-  if (check(cfg) != MOE_OK || rows < 0 || K <= 0) return -1;
-  return rows * K * bits_of(cfg) / 8;
+  if (check(cfg) != MOE_OK || rows < 0 || K <= 0 || rows % 128 != 0) return -1;
+  return rows * moe::kb_padded(K, bits_of(cfg));
 }
 
 int64_t moe_sf_bytes(const moe_config* cfg, int64_t rows, int64_t K) {

@@ -31,6 +31,30 @@ __host__ __device__ inline int64_t sf_offset(int64_t row, int64_t col, int64_t n
 }
 
 // ---------------------------------------------------------------------------
+// Tiled operand layout.  Every GEMM operand (weight codes, permuted activation
+// codes, intermediate codes) is a [rows, kb] byte matrix (kb = K * bits / 8
+// rounded up to a multiple of 128) stored as tiles of TR rows x 128 bytes,
+// K tile fastest: tile (g, kt) of row group g = row / TR and K tile
+// kt = byte / 128 sits at (g * (kb / 128) + kt) * TR *
+// 128.  Inside a tile, bytes are already in the 128-byte-swizzle order of the
+// tensor core's shared-memory operand layout: row r at r * 128, and its 16-byte
+// chunk c at chunk position c ^ (r % 8).  One contiguous bulk copy therefore
+// lands a ready-to-use operand tile in shared memory.
+// TR is 256 for weights (one GEMM N tile) and 128 for activations (one M tile).
+// ---------------------------------------------------------------------------
+constexpr int kWeightTileRows = 256;
+constexpr int kActTileRows = 128;
+
+__host__ __device__ inline int64_t kb_padded(int64_t K, int bits) { return ((K * bits / 8) + 127) / 128 * 128; }
+
+__host__ __device__ inline int64_t tile_offset(int64_t row, int64_t byte, int64_t kb, int64_t TR) {
+  const int64_t tile = (row / TR) * (kb >> 7) + (byte >> 7);
+  const int64_t r = row % TR;
+  const int64_t b = byte & 127;
+  return tile * TR * 128 + r * 128 + ((((b >> 4) ^ (r & 7)) << 4) | (b & 15));
+}
+
+// ---------------------------------------------------------------------------
 // small helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -120,17 +144,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
-// TMA (tiled tensor copies, no multicast) and untiled bulk copies
+// Bulk copies global -> shared (the TMA engine's 1-D mode, no multicast)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y,
-                                            uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar,
                                           uint64_t policy) {
   asm volatile(
@@ -154,10 +169,6 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
-}
-
-__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 // ---------------------------------------------------------------------------

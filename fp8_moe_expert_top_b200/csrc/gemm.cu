@@ -65,6 +65,8 @@ struct GemmTraits {
 };
 
 struct GemmArgs {
+  const uint8_t* a_codes;     // tiled activation codes (128-row tiles)
+  const uint8_t* b_codes;     // tiled weight codes (256-row tiles), expert 0
   const uint8_t* a_sf;
   const uint8_t* b_sf;
   const int32_t* offsets;
@@ -80,6 +82,9 @@ struct GemmArgs {
   int E;
   int K;            // reduction length in elements
   int n_rows_b;     // weight rows per expert (2I for gate/up, H for down)
+  int64_t kb;                 // bytes of one code row, padded to a multiple of 128
+  int64_t b_expert_stride;    // code bytes of one expert's weight matrix
+  int64_t h_kb;               // gate/up: padded code-row bytes of h
   int64_t sf_rb_stride;       // scale bytes of one 128-row block (= K / sfvec * 128)
   int64_t b_sf_expert_stride; // scale bytes of one expert's weight matrix
 };
@@ -114,8 +119,7 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const int32_t* offs, i
 
 template <int FMT, bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
-    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_a16,
-                    const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+    moe_gemm_kernel(const GemmArgs args) {
   using Tr = GemmTraits<FMT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -139,9 +143,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(tempty_bar, 32 * kEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
-    prefetch_tensormap(&tmap_a);
-    prefetch_tensormap(&tmap_a16);
-    prefetch_tensormap(&tmap_b);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -179,13 +180,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint8_t* a_sf = args.a_sf + static_cast<int64_t>(mt) * args.sf_rb_stride;
         const uint8_t* b_sf = args.b_sf + static_cast<int64_t>(e) * args.b_sf_expert_stride +
                               static_cast<int64_t>(nt) * (kBN / 128) * args.sf_rb_stride;
-        const int b_row = e * args.n_rows_b + nt * kBN;
-        // Only the row block's valid rows are loaded, in 16-row boxes; the
+        const int64_t ktiles_row = args.kb >> 7;  // K tiles per code row
+        const uint8_t* a_tiles = args.a_codes + static_cast<int64_t>(mt) * ktiles_row * Tr::kABytes;
+        const uint8_t* b_tiles = args.b_codes + static_cast<int64_t>(e) * args.b_expert_stride +
+                                 static_cast<int64_t>(nt) * ktiles_row * Tr::kBBytes;
+        // Only the row block's valid rows are loaded (rounded up to 16); the
         // rest of the A tile keeps stale data, whose output rows are never
         // stored (each output row depends only on its own A row).
         const int valid_rows = min(kBM, s_offsets[e] + __ldg(args.counts + e) - mt * kBM);
-        const int a_boxes = (valid_rows + 15) / 16;
-        const uint32_t a_bytes = (a_boxes == kBM / 16) ? Tr::kABytes : a_boxes * 16 * kRowBytesPerStage;
+        const uint32_t a_bytes = static_cast<uint32_t>((valid_rows + 15) / 16) * 16 * kRowBytesPerStage;
         for (int kt = 0; kt < k_tiles; ++kt) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
             fail_bits |= MOE_DEVICE_TIMEOUT_PRODUCER;
@@ -195,14 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sf_bytes = (FMT == MOE_NVFP4) ? 512u * kb_here : 512u;
           uint8_t* st = smem + stage * Tr::kStageBytes;
           mbar_arrive_expect_tx(&full_bar[stage], a_bytes + Tr::kBBytes + sf_bytes * (1 + kBN / 128));
-          if (a_boxes == kBM / 16) {
-            tma_load_2d(st, &tmap_a, kt * kRowBytesPerStage, mt * kBM, &full_bar[stage], pol_a);
-          } else {
-            for (int i = 0; i < a_boxes; ++i)
-              tma_load_2d(st + i * 16 * kRowBytesPerStage, &tmap_a16, kt * kRowBytesPerStage, mt * kBM + 16 * i,
-                          &full_bar[stage], pol_a);
-          }
-          tma_load_2d(st + Tr::kABytes, &tmap_b, kt * kRowBytesPerStage, b_row, &full_bar[stage], pol_w);
+          bulk_load(st, a_tiles + static_cast<int64_t>(kt) * Tr::kABytes, a_bytes, &full_bar[stage], pol_a);
+          bulk_load(st + Tr::kABytes, b_tiles + static_cast<int64_t>(kt) * Tr::kBBytes, Tr::kBBytes, &full_bar[stage],
+                    pol_w);
           bulk_load(st + Tr::kSfaOff, a_sf + kt * Tr::kSfBytes128, sf_bytes, &full_bar[stage], pol_a);
 #pragma unroll
           for (int h = 0; h < kBN / 128; ++h)
@@ -347,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               blk[i] = (b == 0) ? acc[i] : (b == 1) ? acc[16 + i] : (b == 2) ? acc[64 + i] : acc[80 + i];
             const Nvfp4Block qb = nvfp4_quantize16(blk, sh);
             const int ch = ch0 + 16 * b;
-            *reinterpret_cast<uint2*>(args.h_codes + row * (I / 2) + ch / 2) =
+            *reinterpret_cast<uint2*>(args.h_codes + tile_offset(row, ch / 2, args.h_kb, kActTileRows)) =
                 make_uint2(static_cast<uint32_t>(qb.codes), static_cast<uint32_t>(qb.codes >> 32));
             args.h_sf[sf_offset(row, ch / 16, I / 16)] = static_cast<uint8_t>(qb.sf);
           }
@@ -360,9 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t w[8];
             const uint32_t ex = mxfp8_quantize32(blk, w);
             const int ch = ch0 + 32 * b;
-            uint4* dst = reinterpret_cast<uint4*>(args.h_codes + row * I + ch);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            *reinterpret_cast<uint4*>(args.h_codes + tile_offset(row, ch, args.h_kb, kActTileRows)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(args.h_codes + tile_offset(row, ch + 16, args.h_kb, kActTileRows)) =
+                make_uint4(w[4], w[5], w[6], w[7]);
             args.h_sf[sf_offset(row, ch / 32, I / 32)] = static_cast<uint8_t>(ex);
           }
         }
@@ -395,40 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 2-D map over a [rows][row_bytes] byte matrix, box 128 bytes x box_rows,
-// 128-byte swizzle; columns past row_bytes read as zero.
-static bool make_map(CUtensorMap* map, const void* base, int64_t row_bytes, int64_t rows, int box_rows) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (enc == nullptr) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
-  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
-  const cuuint32_t estr[2] = {1u, 1u};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int FMT, bool GATEUP>
-static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& ma16, const CUtensorMap& mb, const GemmArgs& a,
-                              cudaStream_t stream) {
+static cudaError_t launch_one(const GemmArgs& a, cudaStream_t stream) {
   using Tr = GemmTraits<FMT>;
   const size_t smem = 1024 + kStages * Tr::kStageBytes + (2 * kStages + 2) * 8 + 16 + (a.E + 1) * 4;
   int dev = 0;
@@ -446,7 +413,7 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& ma16, co
   int sms = 0;
   err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (err != cudaSuccess) return err;
-  return launch_pdl(moe_gemm_kernel<FMT, GATEUP>, dim3(sms), dim3(kThreads), smem, stream, ma, ma16, mb, a);
+  return launch_pdl(moe_gemm_kernel<FMT, GATEUP>, dim3(sms), dim3(kThreads), smem, stream, a);
 }
 
 size_t gemm_smem_bytes(int fmt, int E) {
@@ -457,12 +424,12 @@ size_t gemm_smem_bytes(int fmt, int E) {
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
   const int bits = (g.fmt == MOE_NVFP4) ? 4 : 8;
   const int sfvec = (g.fmt == MOE_NVFP4) ? 16 : 32;
-  const int64_t row_bytes = static_cast<int64_t>(g.K) * bits / 8;
-  CUtensorMap ma, ma16, mb;
-  if (!make_map(&ma, g.a_codes, row_bytes, g.R_max, kBM)) return cudaErrorInvalidValue;
-  if (!make_map(&ma16, g.a_codes, row_bytes, g.R_max, 16)) return cudaErrorInvalidValue;
-  if (!make_map(&mb, g.b_codes, row_bytes, static_cast<int64_t>(g.E) * g.n_rows_b, kBN)) return cudaErrorInvalidValue;
   GemmArgs a;
+  a.a_codes = g.a_codes;
+  a.b_codes = g.b_codes;
+  a.kb = kb_padded(g.K, bits);
+  a.b_expert_stride = static_cast<int64_t>(g.n_rows_b) * a.kb;
+  a.h_kb = g.gateup ? kb_padded(g.n_rows_b / 2, bits) : 0;
   a.a_sf = g.a_sf;
   a.b_sf = g.b_sf;
   a.offsets = g.offsets;
@@ -481,10 +448,8 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
   a.sf_rb_stride = static_cast<int64_t>(g.K / sfvec) * 128;
   a.b_sf_expert_stride = static_cast<int64_t>(g.n_rows_b) * (g.K / sfvec);
   if (g.fmt == MOE_NVFP4)
-    return g.gateup ? launch_one<MOE_NVFP4, true>(ma, ma16, mb, a, stream)
-                    : launch_one<MOE_NVFP4, false>(ma, ma16, mb, a, stream);
-  return g.gateup ? launch_one<MOE_MXFP8, true>(ma, ma16, mb, a, stream)
-                  : launch_one<MOE_MXFP8, false>(ma, ma16, mb, a, stream);
+    return g.gateup ? launch_one<MOE_NVFP4, true>(a, stream) : launch_one<MOE_NVFP4, false>(a, stream);
+  return g.gateup ? launch_one<MOE_MXFP8, true>(a, stream) : launch_one<MOE_MXFP8, false>(a, stream);
 }
 
 }  // namespace moe

@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
   float f[kBlock];
 #pragma unroll
   for (int i = 0; i < kBlock / 16; ++i) load16_bf16(src + 16 * i, f + 16 * i);
+  const int64_t kb = kb_padded(H, FMT == MOE_NVFP4 ? 4 : 8);
   if (FMT == MOE_NVFP4) {
     const Nvfp4Block q = nvfp4_quantize16(f, __ldg(act_scale));
     const uint2 c = make_uint2(static_cast<uint32_t>(q.codes), static_cast<uint32_t>(q.codes >> 32));
@@ -59,7 +60,7 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
     for (int j = 0; j < 8; ++j) {
       if (j >= k) break;
       const int64_t r = __ldg(slot_to_row + static_cast<int64_t>(t) * k + j);
-      *reinterpret_cast<uint2*>(a_codes + r * (H / 2) + 8 * b) = c;
+      *reinterpret_cast<uint2*>(a_codes + tile_offset(r, 8 * b, kb, kActTileRows)) = c;
       a_sf[sf_offset(r, b, nsf)] = static_cast<uint8_t>(q.sf);
     }
   } else {
@@ -69,9 +70,9 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
     for (int j = 0; j < 8; ++j) {
       if (j >= k) break;
       const int64_t r = __ldg(slot_to_row + static_cast<int64_t>(t) * k + j);
-      uint4* dst = reinterpret_cast<uint4*>(a_codes + r * H + 32 * b);
-      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 32 * b, kb, kActTileRows)) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 32 * b + 16, kb, kActTileRows)) =
+          make_uint4(w[4], w[5], w[6], w[7]);
       a_sf[sf_offset(r, b, nsf)] = static_cast<uint8_t>(e);
     }
   }

@@ -78,11 +78,12 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(int H, int I, const f
     sfbuf = w13_sf;
   }
   const float4* src4 = reinterpret_cast<const float4*>(src);
+  const int64_t kb = kb_padded(K, FMT == MOE_NVFP4 ? 4 : 8);
+  uint8_t* ecodes = codes + static_cast<int64_t>(e) * rows_per_expert * kb;  // this expert's tiles
   if (FMT == MOE_NVFP4) {
     const float a = amax[e * 3 + m];
     const float s_g = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);
     uint32_t sfw = 0;
-    uint8_t* dst = codes + (static_cast<int64_t>(e) * rows_per_expert + dst_row) * (K / 2) + 32 * g;
 #pragma unroll 1
     for (int b = 0; b < 4; ++b) {
       float f[16];
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(int H, int I, const f
       }
       const Nvfp4Block q = nvfp4_quantize16(f, s_g);
       sfw |= q.sf << (8 * b);
-      *reinterpret_cast<uint2*>(dst + 8 * b) =
+      *reinterpret_cast<uint2*>(ecodes + tile_offset(dst_row, 32 * g + 8 * b, kb, kWeightTileRows)) =
           make_uint2(static_cast<uint32_t>(q.codes), static_cast<uint32_t>(q.codes >> 32));
     }
     const int64_t nsf = K / 16;
@@ -104,7 +105,6 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(int H, int I, const f
     *reinterpret_cast<uint32_t*>(sfe + sf_offset(dst_row, 4 * g, nsf)) = sfw;
   } else {
     uint32_t sfw = 0;
-    uint8_t* dst = codes + (static_cast<int64_t>(e) * rows_per_expert + dst_row) * K + 64 * g;
 #pragma unroll 1
     for (int b = 0; b < 2; ++b) {
       float f[32];
@@ -118,9 +118,11 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(int H, int I, const f
       }
       uint32_t w[8];
       sfw |= mxfp8_quantize32(f, w) << (8 * b);
-      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * b);
-      d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      const int byte0 = 64 * g + 32 * b;
+      *reinterpret_cast<uint4*>(ecodes + tile_offset(dst_row, byte0, kb, kWeightTileRows)) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(ecodes + tile_offset(dst_row, byte0 + 16, kb, kWeightTileRows)) =
+          make_uint4(w[4], w[5], w[6], w[7]);
     }
     const int64_t nsf = K / 32;
     uint8_t* sfe = sfbuf + static_cast<int64_t>(e) * rows_per_expert * nsf;
@@ -149,9 +151,9 @@ cudaError_t launch_quantize_weights(int fmt, int E, int H, int I, int expert_beg
   const int sfvec = (fmt == MOE_NVFP4) ? 16 : 32;
   const int64_t rows13 = 2 * static_cast<int64_t>(I);
   // offset every output by the slice start so the kernels index experts 0..count-1
-  uint8_t* c13 = w13_codes + static_cast<int64_t>(expert_begin) * rows13 * H * bits / 8;
+  uint8_t* c13 = w13_codes + static_cast<int64_t>(expert_begin) * rows13 * kb_padded(H, bits);
   uint8_t* s13 = w13_sf + static_cast<int64_t>(expert_begin) * rows13 * H / sfvec;
-  uint8_t* c2 = w2_codes + static_cast<int64_t>(expert_begin) * H * static_cast<int64_t>(I) * bits / 8;
+  uint8_t* c2 = w2_codes + static_cast<int64_t>(expert_begin) * H * kb_padded(I, bits);
   uint8_t* s2 = w2_sf + static_cast<int64_t>(expert_begin) * H * static_cast<int64_t>(I) / sfvec;
   float* sc = scales + static_cast<int64_t>(expert_begin) * 3;
   cudaError_t err = cudaMemsetAsync(sc, 0, sizeof(float) * 3 * expert_count, stream);

@@ -37,11 +37,19 @@
  *     MOE_DEVICE_*), which the caller reads after synchronizing.
  *   - Supported shapes: d_model % 256 == 0, d_ffn % 128 == 0, 1 <= top_k <=
  *     min(8, num_experts), 1 <= num_experts <= 1024, 0 <= T <= 2^20.
- *   - Layout of quantized row-major operands: codes are stored row-major with
- *     K contiguous.  NVFP4 packs two E2M1 codes per byte, element 2i in the
- *     low nibble of byte i; MXFP8 stores one E4M3 code per byte.  Zero codes
- *     are always the +0 code.  Block scales are stored in 512-byte atoms of
- *     128 rows x 4 scale columns (see moe_sf_offset()).
+ *   - Layout of quantized operands.  A code row holds K codes: NVFP4 packs
+ *     two E2M1 codes per byte, element 2i in the low nibble of byte i; MXFP8
+ *     stores one E4M3 code per byte.  Zero codes are always the +0 code.  Each
+ *     row is padded to kb = roundup(K * bits / 8, 128) bytes.  A [rows, kb]
+ *     code matrix is stored tiled, ready to copy into the tensor core's
+ *     shared-memory operand layout: tiles of TR rows x 128 bytes, K tile
+ *     fastest (tile (row / TR, byte / 128) at ((row / TR) * (kb / 128) +
+ *     byte / 128) * TR * 128), and inside a tile row r = row % TR at r * 128
+ *     with its 16-byte chunk c = (byte % 128) / 16 at chunk position
+ *     c ^ (r % 8) (the 128-byte swizzle).  TR = 256 for weights and 128 for
+ *     activations (permuted x and the intermediate h).  Block scales are
+ *     stored in 512-byte atoms of 128 rows x 4 scale columns (see
+ *     moe_sf_offset()).
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -89,12 +97,13 @@ typedef struct {
 #define MOE_DEVICE_TIMEOUT_SELFTEST 0x8u
 
 /* Layout of the packed expert weights (byte offsets from the buffer start).
- * For NVFP4 (bits = 4, sfvec = 16) and MXFP8 (bits = 8, sfvec = 32):
- *   w13_codes  [E][2I][H*bits/8]  gate and up rows interleaved in groups of
+ * For NVFP4 (bits = 4, sfvec = 16) and MXFP8 (bits = 8, sfvec = 32), with
+ * kb(K) = roundup(K * bits / 8, 128) and code matrices tiled with TR = 256:
+ *   w13_codes  [E][2I x kb(H)]    gate and up rows interleaved in groups of
  *                                 32: row 64g + i is gate channel 32g + i and
  *                                 row 64g + 32 + i is up channel 32g + i
  *   w13_sf     [E][2I*H/sfvec]    block scales of w13, atom layout per expert
- *   w2_codes   [E][H][I*bits/8]   down projection, one row per output channel
+ *   w2_codes   [E][H x kb(I)]     down projection, one row per output channel
  *   w2_sf      [E][H*I/sfvec]     block scales of w2, atom layout per expert
  *   scales     [E][3] float32     tensor scales of (gate, up, down); 1.0 for
  *                                 MXFP8
@@ -121,9 +130,10 @@ MOE_API moe_status moe_get_weights_layout(const moe_config* cfg, moe_weights_lay
  * R_max = roundup128(T*k + 127*min(E, T*k)).  Returns -1 on a bad config. */
 MOE_API int64_t moe_max_rows(const moe_config* cfg, int64_t T);
 
-/* Bytes of the quantized codes / block scales of `rows` rows of length K in
- * the configured format (K = d_model for the permuted activations A, K =
- * d_ffn for the intermediate h).  Returns -1 on a bad argument. */
+/* Bytes of the (tiled) quantized codes / block scales of `rows` rows of
+ * length K in the configured format (K = d_model for the permuted activations
+ * A, K = d_ffn for the intermediate h; rows a multiple of 128).  Returns -1
+ * on a bad argument. */
 MOE_API int64_t moe_codes_bytes(const moe_config* cfg, int64_t rows, int64_t K);
 MOE_API int64_t moe_sf_bytes(const moe_config* cfg, int64_t rows, int64_t K);
 
@@ -181,7 +191,7 @@ MOE_API moe_status moe_route_topk(const moe_config* cfg, int64_t T, const float*
  * experts": activations quantized to the weight format inside the producing
  * kernel; P2 TL;DR: the 4-vs-6 pick].  Token t's row x[t] (bf16 [T][H]) is
  * quantized once and written to each of its k rows slot_to_row[t*k+j] of
- *   a_codes  [R_max][H*bits/8]  (moe_codes_bytes(cfg, R_max, H))
+ *   a_codes  tiled codes, TR = 128 (moe_codes_bytes(cfg, R_max, H))
  *   a_sf     block scales       (moe_sf_bytes(cfg, R_max, H))
  * act_scale: device float32 scalar, the static NVFP4 tensor scale of x
  * (ignored, may be NULL, for MXFP8).  Padding rows are not written. */

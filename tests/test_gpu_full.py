@@ -27,7 +27,7 @@ from oracle import moe as omoe
 from oracle import route as ort
 
 from gpu_common import assert_expert_equal, build_layer, gpu_expert
-from helpers import rel_fro, sfvec, unpack_codes, unswizzle_sf
+from helpers import ACT_TR, kb_padded, rel_fro, sfvec, sf_index, tile_offsets, unpack_codes
 
 FULL = ["decode_nvfp4", "decode_mxfp8", "prefill_nvfp4", "prefill_nvfp4_skewed"]
 
@@ -50,6 +50,14 @@ def oracle_experts(wl, experts, device):
 def rows_np(t, rows):
     idx = torch.as_tensor(np.asarray(rows, dtype=np.int64), device=t.device)
     return t.index_select(0, idx).cpu().numpy()
+
+
+def tiled_rows(t, rows, K, fmt):
+    """Codes [len(rows), K] of the given rows of a tiled device code buffer."""
+    kb = kb_padded(K, fmt)
+    off = torch.as_tensor(tile_offsets(rows, kb, ACT_TR).reshape(-1), device=t.device)
+    raw = t.reshape(-1).index_select(0, off).cpu().numpy().reshape(len(rows), kb)
+    return unpack_codes(fmt, raw, len(rows), K)
 
 
 @pytest.mark.gpu
@@ -89,11 +97,8 @@ def test_full_size_layer(cuda_device, name):
     ref = omoe.forward_tokens(xs, lg[sample].numpy(), oq, k, wl.fmt, inputs.S_X, inputs.S_H)
     rows = [int(r["slot_to_row"][t * k + j]) for t in sample for j in range(k)]
     # activation codes of the sampled rows
-    bpe = 4 if wl.fmt == inputs.NVFP4 else 8
-    ac = layer.a_codes.view(layer.R_max, H * bpe // 8)
-    a_codes = unpack_codes(wl.fmt, rows_np(ac, rows), len(rows), H)
+    a_codes = tiled_rows(layer.a_codes, rows, H, wl.fmt)
     a_sf_all = layer.a_sf.cpu().numpy()
-    from helpers import sf_index
     sfi = sf_index(layer.R_max, H // v)
     a_sf = a_sf_all[sfi[rows]]
     for i, t in enumerate(sample):
@@ -102,8 +107,7 @@ def test_full_size_layer(cuda_device, name):
             np.testing.assert_array_equal(a_sf[i * k + j], ref["a_sf"][i])
     # gate/up and the intermediate on the sampled rows
     dbg = rows_np(layer.gateup_debug, rows)
-    hcv = layer.h_codes.view(layer.R_max, I * bpe // 8)
-    h_codes = unpack_codes(wl.fmt, rows_np(hcv, rows), len(rows), I)
+    h_codes = tiled_rows(layer.h_codes, rows, I, wl.fmt)
     h_sf = layer.h_sf.cpu().numpy()[sf_index(layer.R_max, I // v)[rows]]
     a_deq = omoe.dequantize_rows(ref["a_codes"], ref["a_sf"], wl.fmt, inputs.S_X)
     g_ref, u_ref, hc_ref, hs_ref = [], [], [], []

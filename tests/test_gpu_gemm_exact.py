@@ -18,7 +18,7 @@ import torch
 from fp8_moe_expert_top_b200 import binding as B
 from oracle import formats as fm
 
-from helpers import encode_expert_into, pack_nvfp4, swizzle_sf, sfvec, w13_row
+from helpers import ACT_TR, encode_expert_into, kb_padded, pack_nvfp4, pad_row_bytes, swizzle_sf, sfvec, tile_matrix
 
 GRID_E2M1 = np.array([0, 1, 2, 3, 4, 5, 6, 7, 9, 10, 11, 12, 13, 14, 15], dtype=np.uint8)   # no -0
 GRID_E4M3 = np.array([0x00, 0x30, 0x38, 0x3C, 0x40, 0x44, 0x48, 0x4C,
@@ -78,7 +78,7 @@ def test_gemm_integer_exact(cuda_device, fmt, H, I):
 
     # activations: valid rows from the grid, padding rows random bytes
     bpe = 4 if fmt == "nvfp4" else 8
-    a_codes = rng.integers(0, 256, (R, H * bpe // 8), dtype=np.uint8)
+    a_codes = rng.integers(0, 256, (R, kb_padded(H, fmt)), dtype=np.uint8)
     a_sf = rng.integers(0, 256, (R, H // v), dtype=np.uint8)
     A = np.zeros((R, H))
     for e in range(E):
@@ -87,13 +87,13 @@ def test_gemm_integer_exact(cuda_device, fmt, H, I):
             continue
         codes = rand_codes(rng, fmt, (c, H))
         sf = rand_sf(rng, fmt, (c, H // v))
-        a_codes[lo:lo + c] = to_rows_bytes(fmt, codes)
+        a_codes[lo:lo + c, :H * bpe // 8] = to_rows_bytes(fmt, codes)
         a_sf[lo:lo + c] = sf
         A[lo:lo + c] = decode(fmt, codes, sf)
 
     t = lambda a, dt=torch.uint8: torch.from_numpy(np.ascontiguousarray(a)).to(dt).to(dev)
     d_packed = t(packed)
-    d_a = t(a_codes)
+    d_a = t(tile_matrix(a_codes, ACT_TR))
     d_asf = t(swizzle_sf(a_sf))
     d_off = t(offsets, torch.int32)
     d_cnt = t(counts, torch.int32)
@@ -123,7 +123,7 @@ def test_gemm_integer_exact(cuda_device, fmt, H, I):
     assert np.all(np.isnan(got[~valid]))
 
     # down GEMM on intermediate codes chosen the same way
-    hc = rng.integers(0, 256, (R, I * bpe // 8), dtype=np.uint8)
+    hc = rng.integers(0, 256, (R, kb_padded(I, fmt)), dtype=np.uint8)
     hs = rng.integers(0, 256, (R, I // v), dtype=np.uint8)
     Hm = np.zeros((R, I))
     for e in range(E):
@@ -132,11 +132,12 @@ def test_gemm_integer_exact(cuda_device, fmt, H, I):
             continue
         codes = rand_codes(rng, fmt, (c, I))
         sf = rand_sf(rng, fmt, (c, I // v))
-        hc[lo:lo + c] = to_rows_bytes(fmt, codes)
+        hc[lo:lo + c, :I * bpe // 8] = to_rows_bytes(fmt, codes)
         hs[lo:lo + c] = sf
         Hm[lo:lo + c] = decode(fmt, codes, sf)
     out = torch.full((R, H), float("nan"), dtype=torch.bfloat16, device=dev)
-    B.moe_forward_down(cfg, T, d_packed, t(hc), t(swizzle_sf(hs)), scale, d_off, d_cnt, out, status)
+    B.moe_forward_down(cfg, T, d_packed, t(tile_matrix(hc, ACT_TR)), t(swizzle_sf(hs)), scale, d_off, d_cnt, out,
+                       status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     o = out.float().cpu().numpy().astype(np.float64)

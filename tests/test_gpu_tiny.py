@@ -21,7 +21,7 @@ from fp8_moe_expert_top_b200 import inputs
 from oracle import moe as omoe
 
 from gpu_common import assert_expert_equal, build_layer, gpu_expert, oracle_expert
-from helpers import rel_fro, sfvec, unpack_codes, unswizzle_sf
+from helpers import ACT_TR, rel_fro, sfvec, tiled_codes, unswizzle_sf
 
 TINY = inputs.WORKLOADS["tiny_nvfp4"]
 TINY_MX = dataclasses.replace(TINY, name="tiny_mxfp8", fmt=inputs.MXFP8)
@@ -65,7 +65,7 @@ def run_and_compare(layer, wl, x, logits, experts_q):
     H, I, v = wl.d_model, wl.d_ffn, sfvec(wl.fmt)
     Rb = layer.R_max
     # activation codes: bit-exact on valid rows
-    a_codes = unpack_codes(wl.fmt, layer.a_codes.cpu().numpy(), Rb, H)[:R]
+    a_codes = tiled_codes(wl.fmt, layer.a_codes.cpu().numpy(), np.arange(R), H, ACT_TR)
     a_sf = unswizzle_sf(layer.a_sf.cpu().numpy(), Rb, H // v)[:R]
     np.testing.assert_array_equal(a_codes[valid], ref["a_codes"][valid])
     np.testing.assert_array_equal(a_sf[valid], ref["a_sf"][valid])
@@ -76,7 +76,7 @@ def run_and_compare(layer, wl, x, logits, experts_q):
     assert err_g <= 1e-4 and err_u <= 1e-4, (err_g, err_u)
     assert np.all(np.isnan(dbg[~valid]))
     # requantized intermediate
-    hc = unpack_codes(wl.fmt, layer.h_codes.cpu().numpy(), Rb, I)[:R]
+    hc = tiled_codes(wl.fmt, layer.h_codes.cpu().numpy(), np.arange(R), I, ACT_TR)
     hs = unswizzle_sf(layer.h_sf.cpu().numpy(), Rb, I // v)[:R]
     rc, rs = ref["h_codes"], ref["h_sf"]
     differ = (hc != rc) | (np.repeat(hs, v, axis=1) != np.repeat(rs, v, axis=1))
