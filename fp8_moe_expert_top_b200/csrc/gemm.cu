@@ -16,13 +16,23 @@
 // over N tiles, so the tiles sharing an activation block run together and
 // the weight tiles of one expert are reused from L2 across its row blocks).
 //
-// Warp roles (192 threads):
-//   warp 0      TMA producer: codes via 2-D tensor maps (128-byte swizzle),
-//               block scales via 1-D bulk copies, into a 4-stage ring
-//   warp 1      MMA issuer: TMEM allocation, scale atoms SMEM->TMEM with
-//               tcgen05.cp, tcgen05.mma block-scaled M=128 N=256, commits
-//   warps 2-5   epilogue: tcgen05.ld of the 128x256 fp32 accumulator, tensor
-//               scales, SwiGLU + requantization (gate/up) or bf16 store (down)
+// Operands are stored pre-tiled and pre-swizzled (tiles of rows x 128 bytes,
+// K tile fastest, the 128-byte swizzle applied in memory), so every stage is
+// one contiguous 1-D bulk copy per operand.
+//
+// Warp roles (352 threads):
+//   warp 0      producer: bulk copies of A, B and their scale atoms into a
+//               4-stage ring
+//   warp 1      MMA issuer: TMEM allocation, tcgen05.mma block-scaled
+//               M=128 N=256, commits
+//   warps 2-9   epilogue: tcgen05.ld of the 128x256 fp32 accumulator (two
+//               warps per TMEM lane quarter, 128 columns each), tensor scales,
+//               SwiGLU + requantization (gate/up) or bf16 store (down)
+//   warp 10     scale copier: moves a stage's scale atoms SMEM -> TMEM with
+//               tcgen05.cp into that stage's own TMEM columns.  Copies take
+//               as long as the MMAs in the tensor pipe; issued from their own
+//               thread they run ahead of and overlap the MMA stream instead
+//               of sitting in front of every stage's MMAs.
 // Every mbarrier wait is bounded; a wait that runs out raises a CTA-wide
 // abort flag, every role stops issuing, TMEM is freed and a status bit is
 // set.
@@ -31,74 +41,19 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "gemm_common.cuh"
 #include "kernels.cuh"
 #include "quant.cuh"
 
 namespace moe {
 
-constexpr int kBM = 128;
-constexpr int kBN = 256;
 constexpr int kStages = 4;
-constexpr int kRowBytesPerStage = 128;  // K bytes of one row per stage
-constexpr int kEpiWarps = 8;             // two warps per TMEM lane quarter
-constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr uint32_t kTmemCols = 512;
-
+constexpr int kThreadsOne = kThreads + 32;  // + the scale-copier warp
+// TMEM columns of one stage's scales: NVFP4 4 (A) + 8 (B) per 64-element k
+// block x 4 k blocks; MXFP8 4 + 8 (one 32-bit column holds 4 k blocks)
 template <int FMT>
-struct GemmTraits {
-  static constexpr int kElemsPerStage = (FMT == MOE_NVFP4) ? 256 : 128;
-  static constexpr int kMmaK = (FMT == MOE_NVFP4) ? 64 : 32;
-  static constexpr int kSfVec = (FMT == MOE_NVFP4) ? 16 : 32;
-  // scale bytes of 128 rows for one stage: NVFP4 16 scales/row = 4 atoms,
-  // MXFP8 4 scales/row = 1 atom
-  static constexpr int kSfBytes128 = 128 * (kElemsPerStage / kSfVec);
-  static constexpr int kABytes = kBM * kRowBytesPerStage;
-  static constexpr int kBBytes = kBN * kRowBytesPerStage;
-  static constexpr int kSfaOff = kABytes + kBBytes;
-  static constexpr int kSfbOff = kSfaOff + kSfBytes128;
-  static constexpr int kStageRaw = kSfbOff + (kBN / 128) * kSfBytes128;
-  static constexpr int kStageBytes = (kStageRaw + 1023) / 1024 * 1024;
-  // TMEM columns: accumulator [0, kBN), scales of A, then scales of B
-  static constexpr int kTmemSfa = kBN;
-  static constexpr int kSfaCols = (FMT == MOE_NVFP4) ? 16 : 4;
-  static constexpr int kTmemSfb = kTmemSfa + kSfaCols;
-};
-
-struct GemmArgs {
-  const uint8_t* a_codes;     // tiled activation codes (128-row tiles)
-  const uint8_t* b_codes;     // tiled weight codes (256-row tiles), expert 0
-  const uint8_t* a_sf;
-  const uint8_t* b_sf;
-  const int32_t* offsets;
-  const int32_t* counts;
-  const float* a_scale;
-  const float* w_scales;
-  const float* h_scale;
-  uint8_t* h_codes;
-  uint8_t* h_sf;
-  float* dbg;
-  __nv_bfloat16* out;
-  uint32_t* status;
-  int E;
-  int K;            // reduction length in elements
-  int n_rows_b;     // weight rows per expert (2I for gate/up, H for down)
-  int64_t kb;                 // bytes of one code row, padded to a multiple of 128
-  int64_t b_expert_stride;    // code bytes of one expert's weight matrix
-  int64_t h_kb;               // gate/up: padded code-row bytes of h
-  int64_t sf_rb_stride;       // scale bytes of one 128-row block (= K / sfvec * 128)
-  int64_t b_sf_expert_stride; // scale bytes of one expert's weight matrix
-};
-
-__device__ __forceinline__ int find_expert(const int32_t* offs, int E, int row) {
-  int lo = 0, hi = E;  // offs[lo] <= row < offs[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (offs[mid] <= row) lo = mid;
-    else hi = mid;
-  }
-  return lo;
-}
-
+constexpr uint32_t kSfColsPerStage = (FMT == MOE_NVFP4) ? 48u : 12u;
+static_assert(kBN + kStages * 48 <= kTmemCols, "scale buffers do not fit in TMEM");
 // Tile order: expert by expert; inside an expert, weight tile (nt) by weight
 // tile, and the expert's 128-row blocks (mt) fastest.  CTAs running at the same
 // time therefore share one weight tile (read from HBM once, then from L2), and
@@ -118,16 +73,17 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const int32_t* offs, i
 }
 
 template <int FMT, bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsOne, 1)
     moe_gemm_kernel(const GemmArgs args) {
-  using Tr = GemmTraits<FMT>;
+  using Tr = GemmTraits<FMT, kBN, kStages>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kStages * Tr::kStageBytes);
   uint64_t* empty_bar = full_bar + kStages;
   uint64_t* tfull_bar = empty_bar + kStages;
   uint64_t* tempty_bar = tfull_bar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 1);
+  uint64_t* sf_bar = tempty_bar + 1;  // a stage's scales are in TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_bar + kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_offsets = reinterpret_cast<int32_t*>(tmem_slot + 4);
 
@@ -138,6 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
+      mbar_init(&sf_bar[s], 1);
     }
     mbar_init(tfull_bar, 1);
     mbar_init(tempty_bar, 32 * kEpiWarps);
@@ -151,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // everything above overlaps the previous kernel; from here on its outputs are read
   pdl_wait();
   pdl_trigger();
-  for (int i = threadIdx.x; i <= E; i += kThreads) s_offsets[i] = args.offsets[i];
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) s_offsets[i] = args.offsets[i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -227,7 +184,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         bool ok = true;
         for (int kt = 0; kt < k_tiles; ++kt) {
-          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+          // the scale copier has seen the stage's operands land and its
+          // scale copies have completed (the operand wait then returns at once)
+          if (!mbar_wait(&sf_bar[stage], phase, abort_flag) || !mbar_wait(&full_bar[stage], phase, abort_flag)) {
             fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
             ok = false;
             break;
@@ -237,28 +196,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t st = smem_u32(smem + stage * Tr::kStageBytes);
           const uint64_t adesc = make_desc_sw128(st);
           const uint64_t bdesc = make_desc_sw128(st + Tr::kABytes);
+          const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kSfColsPerStage<FMT>;
+          const uint32_t sfb = sfa + Tr::kSfaCols;
           if (FMT == MOE_NVFP4) {
             for (int kb = 0; kb < kb_here; ++kb) {
-              tc_cp_sf_atom(tmem_base + Tr::kTmemSfa + 4 * kb, make_desc_sf(st + Tr::kSfaOff + 512 * kb));
-#pragma unroll
-              for (int h = 0; h < kBN / 128; ++h)
-                tc_cp_sf_atom(tmem_base + Tr::kTmemSfb + (kBN / 32) * kb + 4 * h,
-                              make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
-            }
-            for (int kb = 0; kb < kb_here; ++kb) {
-              tc_mma_nvfp4(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_nvfp4(kBN),
-                           tmem_base + Tr::kTmemSfa + 4 * kb, tmem_base + Tr::kTmemSfb + (kBN / 32) * kb,
-                           (kt | kb) != 0 ? 1u : 0u);
+              tc_mma_nvfp4(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_nvfp4(kBN), sfa + 4 * kb,
+                           sfb + (kBN / 32) * kb, (kt | kb) != 0 ? 1u : 0u);
             }
           } else {
-            tc_cp_sf_atom(tmem_base + Tr::kTmemSfa, make_desc_sf(st + Tr::kSfaOff));
-#pragma unroll
-            for (int h = 0; h < kBN / 128; ++h)
-              tc_cp_sf_atom(tmem_base + Tr::kTmemSfb + 4 * h, make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128));
             for (int kb = 0; kb < kb_here; ++kb) {
               const uint32_t sel = static_cast<uint32_t>(kb) << 30;
-              tc_mma_mxfp8(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_mxfp8(kBN, kb),
-                           (tmem_base + Tr::kTmemSfa) | sel, (tmem_base + Tr::kTmemSfb) | sel,
+              tc_mma_mxfp8(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_mxfp8(kBN, kb), sfa | sel, sfb | sel,
                            (kt | kb) != 0 ? 1u : 0u);
             }
           }
@@ -273,6 +221,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_phase ^= 1u;
       }
     }
+  } else if (warp == kThreads / 32) {
+    // ------------------------------------------------------------ scale copier
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        bool ok = true;
+        for (int kt = 0; kt < k_tiles; ++kt) {
+          // The stage's TMEM scale columns were last read by the MMAs of the
+          // same stage one ring turn ago; those completed before the stage
+          // was released and refilled, i.e. before this wait returns.
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+            fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
+          const uint32_t st = smem_u32(smem + stage * Tr::kStageBytes);
+          const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kSfColsPerStage<FMT>;
+          const uint32_t sfb = sfa + Tr::kSfaCols;
+          if (FMT == MOE_NVFP4) {
+            for (int kb = 0; kb < kb_here; ++kb) {
+              tc_cp_sf_atom(sfa + 4 * kb, make_desc_sf(st + Tr::kSfaOff + 512 * kb));
+#pragma unroll
+              for (int h = 0; h < kBN / 128; ++h)
+                tc_cp_sf_atom(sfb + (kBN / 32) * kb + 4 * h,
+                              make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
+            }
+          } else {
+            tc_cp_sf_atom(sfa, make_desc_sf(st + Tr::kSfaOff));
+#pragma unroll
+            for (int h = 0; h < kBN / 128; ++h)
+              tc_cp_sf_atom(sfb + 4 * h, make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128));
+          }
+          tc_commit(&sf_bar[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     // Warps 2..9: quarter q = warp % 4 of the TMEM lanes (rows), half of the
@@ -284,8 +276,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_l = q * 32 + lane;
     const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + half * (kBN / 2);
     uint32_t acc_phase = 0;
-    const int I = args.n_rows_b / 2;  // gate/up: channels; unused for down
-    const int H = args.n_rows_b;      // down: output channels
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
       const TileCoord tc = tile_coord(tile, s_offsets, E, n_tiles);
       const int mt = tc.mt, nt = tc.nt, e = tc.e;
@@ -305,80 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(tempty_bar);
       acc_phase ^= 1u;
       if (!valid) continue;
-      if (GATEUP) {
-        // columns of this half: [gate 32 | up 32] x 2, channels ch0 + [0, 64)
-        const int ch0 = nt * (kBN / 2) + half * (kBN / 4);
-        const float sa = (FMT == MOE_NVFP4) ? __ldg(args.a_scale) : 1.0f;
-        const float sg = (FMT == MOE_NVFP4) ? __fmul_rn(sa, __ldg(args.w_scales + 3 * e + 0)) : 1.0f;
-        const float su = (FMT == MOE_NVFP4) ? __fmul_rn(sa, __ldg(args.w_scales + 3 * e + 1)) : 1.0f;
-        const float sh = (FMT == MOE_NVFP4) ? __ldg(args.h_scale) : 1.0f;
-#pragma unroll
-        for (int j = 0; j < kBN / 128; ++j) {
-          float* g = acc + 64 * j;
-          float* u = acc + 64 * j + 32;
-          const int ch = ch0 + 32 * j;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            g[i] *= sg;
-            u[i] *= su;
-          }
-          if (args.dbg != nullptr) {
-            float4* dg = reinterpret_cast<float4*>(args.dbg + row * (2 * I) + ch);
-            float4* du = reinterpret_cast<float4*>(args.dbg + row * (2 * I) + I + ch);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              dg[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
-              du[i] = make_float4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
-            }
-          }
-          // h = silu(g) * u, written over g
-#pragma unroll
-          for (int i = 0; i < 32; ++i) g[i] = __fdividef(g[i] * u[i], 1.0f + __expf(-g[i]));
-        }
-        // h of this thread: acc[0..32) channels ch0 + [0, 32), acc[64..96) ch0 + [32, 64)
-        if (FMT == MOE_NVFP4) {
-#pragma unroll 1
-          for (int b = 0; b < 4; ++b) {
-            float blk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              blk[i] = (b == 0) ? acc[i] : (b == 1) ? acc[16 + i] : (b == 2) ? acc[64 + i] : acc[80 + i];
-            const Nvfp4Block qb = nvfp4_quantize16(blk, sh);
-            const int ch = ch0 + 16 * b;
-            *reinterpret_cast<uint2*>(args.h_codes + tile_offset(row, ch / 2, args.h_kb, kActTileRows)) =
-                make_uint2(static_cast<uint32_t>(qb.codes), static_cast<uint32_t>(qb.codes >> 32));
-            args.h_sf[sf_offset(row, ch / 16, I / 16)] = static_cast<uint8_t>(qb.sf);
-          }
-        } else {
-#pragma unroll 1
-          for (int b = 0; b < 2; ++b) {
-            float blk[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) blk[i] = (b == 0) ? acc[i] : acc[64 + i];
-            uint32_t w[8];
-            const uint32_t ex = mxfp8_quantize32(blk, w);
-            const int ch = ch0 + 32 * b;
-            *reinterpret_cast<uint4*>(args.h_codes + tile_offset(row, ch, args.h_kb, kActTileRows)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4*>(args.h_codes + tile_offset(row, ch + 16, args.h_kb, kActTileRows)) =
-                make_uint4(w[4], w[5], w[6], w[7]);
-            args.h_sf[sf_offset(row, ch / 32, I / 32)] = static_cast<uint8_t>(ex);
-          }
-        }
-      } else {
-        const float s = (FMT == MOE_NVFP4) ? __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scales + 3 * e + 2)) : 1.0f;
-        uint4* dst = reinterpret_cast<uint4*>(args.out + row * H + nt * kBN + half * (kBN / 2));
-#pragma unroll
-        for (int i = 0; i < kBN / 16; ++i) {
-          uint32_t p[4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const __nv_bfloat162 b = __floats2bfloat162_rn(acc[8 * i + 2 * c] * s, acc[8 * i + 2 * c + 1] * s);
-            p[c] = *reinterpret_cast<const uint32_t*>(&b);
-          }
-          dst[i] = make_uint4(p[0], p[1], p[2], p[3]);
-        }
-      }
+      epilogue_rows<FMT, GATEUP>(args, acc, row, e, nt, half);
     }
   }
 
@@ -396,15 +313,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int FMT, bool GATEUP>
 static cudaError_t launch_one(const GemmArgs& a, cudaStream_t stream) {
-  using Tr = GemmTraits<FMT>;
-  const size_t smem = 1024 + kStages * Tr::kStageBytes + (2 * kStages + 2) * 8 + 16 + (a.E + 1) * 4;
+  using Tr = GemmTraits<FMT, kBN, kStages>;
+  const size_t smem = 1024 + kStages * Tr::kStageBytes + (3 * kStages + 2) * 8 + 16 + (a.E + 1) * 4;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   static int configured[64] = {0};
   if (dev >= 64 || !configured[dev]) {
     // the largest size any supported E needs (E <= 1024)
-    const size_t smem_max = 1024 + kStages * Tr::kStageBytes + (2 * kStages + 2) * 8 + 16 + 1025 * 4;
+    const size_t smem_max = 1024 + kStages * Tr::kStageBytes + (3 * kStages + 2) * 8 + 16 + 1025 * 4;
     err = cudaFuncSetAttribute(moe_gemm_kernel<FMT, GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem_max));
     if (err != cudaSuccess) return err;
@@ -413,12 +330,13 @@ static cudaError_t launch_one(const GemmArgs& a, cudaStream_t stream) {
   int sms = 0;
   err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (err != cudaSuccess) return err;
-  return launch_pdl(moe_gemm_kernel<FMT, GATEUP>, dim3(sms), dim3(kThreads), smem, stream, a);
+  return launch_pdl(moe_gemm_kernel<FMT, GATEUP>, dim3(sms), dim3(kThreadsOne), smem, stream, a);
 }
 
 size_t gemm_smem_bytes(int fmt, int E) {
-  const int sb = (fmt == MOE_NVFP4) ? GemmTraits<MOE_NVFP4>::kStageBytes : GemmTraits<MOE_MXFP8>::kStageBytes;
-  return 1024 + kStages * sb + (2 * kStages + 2) * 8 + 16 + (E + 1) * 4;
+  const int sb = (fmt == MOE_NVFP4) ? GemmTraits<MOE_NVFP4, kBN, kStages>::kStageBytes
+                                    : GemmTraits<MOE_MXFP8, kBN, kStages>::kStageBytes;
+  return 1024 + kStages * sb + (3 * kStages + 2) * 8 + 16 + (E + 1) * 4;
 }
 
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
@@ -447,6 +365,7 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
   a.n_rows_b = g.n_rows_b;
   a.sf_rb_stride = static_cast<int64_t>(g.K / sfvec) * 128;
   a.b_sf_expert_stride = static_cast<int64_t>(g.n_rows_b) * (g.K / sfvec);
+  if (g.pair) return launch_gemm_pair(g, a, stream);
   if (g.fmt == MOE_NVFP4)
     return g.gateup ? launch_one<MOE_NVFP4, true>(a, stream) : launch_one<MOE_NVFP4, false>(a, stream);
   return g.gateup ? launch_one<MOE_MXFP8, true>(a, stream) : launch_one<MOE_MXFP8, false>(a, stream);

@@ -50,15 +50,27 @@ def to_rows_bytes(fmt, codes):
     return pack_nvfp4(codes) if fmt == "nvfp4" else codes
 
 
+# Expert row counts and token counts: a decode-like case (T * k <= 128 * E)
+# and a prefill-like one (T * k > 128 * E, the shape class that may run on SM
+# pairs with 256-row tiles), with odd row-block counts so that a pair would
+# end past an expert's rows and past the last expert.
+CASES = {
+    "one_sm": (np.array([130, 0, 5, 256], dtype=np.int32), 391),
+    "sm_pair": (np.array([200, 50, 300], dtype=np.int32), 550),
+}
+
+
 @pytest.mark.gpu
 @pytest.mark.parametrize("fmt", ["nvfp4", "mxfp8"])
 @pytest.mark.parametrize("H,I", [(256, 128), (512, 256), (1024, 384)])
-def test_gemm_integer_exact(cuda_device, fmt, H, I):
-    rng = np.random.default_rng(H * 7 + I + (1 if fmt == "mxfp8" else 0))
-    E, k = 4, 1
-    counts = np.array([130, 0, 5, 256], dtype=np.int32)
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_gemm_integer_exact(cuda_device, fmt, H, I, case):
+    rng = np.random.default_rng(H * 7 + I + (1 if fmt == "mxfp8" else 0) + (3 if case == "sm_pair" else 0))
+    counts, T = CASES[case]
+    E, k = len(counts), 1
+    assert (T * k > 128 * E) == (case == "sm_pair")
+    assert counts.sum() == T
     offsets = np.concatenate([[0], np.cumsum((counts + 127) // 128 * 128)]).astype(np.int32)
-    T = 391                                      # R_max(T) >= offsets[E] for k = 1
     cfg = B.make_config(E, k, H, I, fmt)
     R = B.moe_max_rows(cfg, T)
     assert R >= offsets[-1]

@@ -25,6 +25,9 @@ from helpers import ACT_TR, rel_fro, sfvec, tiled_codes, unswizzle_sf
 
 TINY = inputs.WORKLOADS["tiny_nvfp4"]
 TINY_MX = dataclasses.replace(TINY, name="tiny_mxfp8", fmt=inputs.MXFP8)
+# T * k > 128 * E: the prefill shape class (several 128-row blocks per expert)
+TINY_PAIR = dataclasses.replace(TINY, name="tiny_nvfp4_pair", T=1024)
+TINY_PAIR_MX = dataclasses.replace(TINY_PAIR, name="tiny_mxfp8_pair", fmt=inputs.MXFP8)
 
 _layers = {}
 
@@ -98,7 +101,7 @@ def test_weights_bit_exact(cuda_device, wl):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("wl", [TINY, TINY_MX], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [TINY, TINY_MX, TINY_PAIR, TINY_PAIR_MX], ids=lambda w: w.name)
 def test_layer_seeded_inputs(cuda_device, wl):
     layer = get_layer(wl, cuda_device)
     x, lg = inputs.make_x(wl), inputs.make_logits(wl)
@@ -125,6 +128,23 @@ def test_layer_edge_cases(cuda_device, wl, case):
         lg[:, [0, 1, 6]] -= 100.0
     else:                                # T not a multiple of anything
         x, lg = inputs.make_x(wl, T=37, seed=19), inputs.make_logits(wl, T=37, seed=20)
+    run_and_compare(layer, wl, x, lg, oracle_experts(wl))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl", [TINY_PAIR, TINY_PAIR_MX], ids=lambda w: w.name)
+@pytest.mark.parametrize("case", ["hot_experts", "empty_experts", "ragged"])
+def test_pair_layer_edge_cases(cuda_device, wl, case):
+    """Prefill-shaped layer with skewed routing, empty experts and a ragged batch."""
+    layer = get_layer(wl, cuda_device)
+    if case == "hot_experts":
+        x, lg = inputs.make_x(wl, seed=23), inputs.make_logits(wl, seed=24)
+        lg[:, 3] += 50.0
+    elif case == "empty_experts":
+        x, lg = inputs.make_x(wl, seed=25), inputs.make_logits(wl, seed=26)
+        lg[:, [0, 6]] -= 100.0
+    else:
+        x, lg = inputs.make_x(wl, T=777, seed=27), inputs.make_logits(wl, T=777, seed=28)
     run_and_compare(layer, wl, x, lg, oracle_experts(wl))
 
 
