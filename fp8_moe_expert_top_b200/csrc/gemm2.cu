@@ -15,7 +15,9 @@
 // the MMA warp's commits arrive on the "empty" and "accumulator full"
 // barriers of both CTAs (tcgen05.commit multicast); both CTAs' epilogue
 // threads release the accumulator on the even CTA's "accumulator empty"
-// barrier.  Waits are bounded as in gemm.cu.
+// barrier.  A scale-copier warp in the even CTA moves both CTAs' scale atoms
+// into TMEM (tcgen05.cp.cta_group::2, per-stage columns) and signals the MMA
+// thread, as in gemm.cu.  Waits are bounded as in gemm.cu.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -29,6 +31,10 @@
 namespace moe {
 
 constexpr int kPairStages = 5;
+constexpr int kPairThreads = kThreads + 32;  // + the scale-copier warp
+template <int FMT>
+constexpr uint32_t kPairSfCols = (FMT == MOE_NVFP4) ? 48u : 12u;  // TMEM scale columns per stage
+static_assert(kBN + kPairStages * 48 <= kTmemCols, "scale buffers do not fit in TMEM");
 
 // Every operand buffer is viewed as a 2-D array of lines (no swizzle: the
 // codes are stored pre-swizzled), so that each copy below is one box of whole
@@ -52,7 +58,7 @@ struct PairCoord {
 };
 
 template <int FMT, bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     moe_gemm_pair_kernel(const __grid_constant__ PairMaps maps, const GemmArgs args) {
   using Tr = GemmTraits<FMT, 128, kPairStages>;
   extern __shared__ uint8_t smem_raw[];
@@ -61,7 +67,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty_bar = full_bar + kPairStages;
   uint64_t* tfull_bar = empty_bar + kPairStages;
   uint64_t* tempty_bar = tfull_bar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 1);
+  uint64_t* sf_bar = tempty_bar + 1;  // a stage's scales are in both CTAs' TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_bar + kPairStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_offsets = reinterpret_cast<int32_t*>(tmem_slot + 4);
   int32_t* s_pstart = s_offsets + args.E + 1;  // first pair-tile of each expert
@@ -75,6 +82,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kPairStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
+      mbar_init(&sf_bar[s], 1);
     }
     mbar_init(tfull_bar, 1);
     mbar_init(tempty_bar, 2 * 32 * kEpiWarps);
@@ -97,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();
   pdl_trigger();
   const int n_tiles = args.n_rows_b / kBN;
-  for (int i = threadIdx.x; i <= E; i += kThreads) s_offsets[i] = args.offsets[i];
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) s_offsets[i] = args.offsets[i];
   __syncthreads();
   if (warp == 0) {  // s_pstart[e] = sum over e' < e of pairs(e') * n_tiles
     int32_t carry = 0;
@@ -235,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         bool ok = true;
         for (int kt = 0; kt < k_tiles; ++kt) {
-          if (!mbar_wait<true>(&full_bar[stage], phase, abort_flag)) {
+          if (!mbar_wait<true>(&sf_bar[stage], phase, abort_flag) ||
+              !mbar_wait<true>(&full_bar[stage], phase, abort_flag)) {
             fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
             ok = false;
             break;
@@ -245,30 +254,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t st = smem_u32(smem + stage * Tr::kStageBytes);
           const uint64_t adesc = make_desc_sw128(st);
           const uint64_t bdesc = make_desc_sw128(st + Tr::kABytes);
+          const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kPairSfCols<FMT>;
+          const uint32_t sfb = sfa + Tr::kSfaCols;
           if (FMT == MOE_NVFP4) {
             for (int kb = 0; kb < kb_here; ++kb) {
-              tc_cp_sf_atom_pair(tmem_base + Tr::kTmemSfa + 4 * kb, make_desc_sf(st + Tr::kSfaOff + 512 * kb));
-#pragma unroll
-              for (int h = 0; h < kBN / 128; ++h)
-                tc_cp_sf_atom_pair(tmem_base + Tr::kTmemSfb + (kBN / 32) * kb + 4 * h,
-                                   make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
-            }
-            for (int kb = 0; kb < kb_here; ++kb) {
-              tc_mma_nvfp4_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_nvfp4(kBN, 2 * kBM),
-                                tmem_base + Tr::kTmemSfa + 4 * kb, tmem_base + Tr::kTmemSfb + (kBN / 32) * kb,
-                                (kt | kb) != 0 ? 1u : 0u);
+              tc_mma_nvfp4_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_nvfp4(kBN, 2 * kBM), sfa + 4 * kb,
+                                sfb + (kBN / 32) * kb, (kt | kb) != 0 ? 1u : 0u);
             }
           } else {
-            tc_cp_sf_atom_pair(tmem_base + Tr::kTmemSfa, make_desc_sf(st + Tr::kSfaOff));
-#pragma unroll
-            for (int h = 0; h < kBN / 128; ++h)
-              tc_cp_sf_atom_pair(tmem_base + Tr::kTmemSfb + 4 * h,
-                                 make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128));
             for (int kb = 0; kb < kb_here; ++kb) {
               const uint32_t sel = static_cast<uint32_t>(kb) << 30;
-              tc_mma_mxfp8_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_mxfp8(kBN, kb, 2 * kBM),
-                                (tmem_base + Tr::kTmemSfa) | sel, (tmem_base + Tr::kTmemSfb) | sel,
-                                (kt | kb) != 0 ? 1u : 0u);
+              tc_mma_mxfp8_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_mxfp8(kBN, kb, 2 * kBM), sfa | sel,
+                                sfb | sel, (kt | kb) != 0 ? 1u : 0u);
             }
           }
           tc_commit_pair(&empty_bar[stage], 0x3);
@@ -280,6 +277,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_commit_pair(tfull_bar, 0x3);
         acc_phase ^= 1u;
+      }
+    }
+  } else if (warp == kThreads / 32) {
+    // ------------------------------------------------------------ scale copier (even CTA)
+    // Copies each CTA's scale atoms into its own TMEM (cta_group::2), into the
+    // stage's own columns, and signals the MMA thread.  The columns were last
+    // read by the MMAs of the same stage one ring turn ago, which completed
+    // before the stage was released and refilled.
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = cid; tile < total && !*abort_flag; tile += ncl) {
+        bool ok = true;
+        for (int kt = 0; kt < k_tiles; ++kt) {
+          if (!mbar_wait<true>(&full_bar[stage], phase, abort_flag)) {
+            fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
+          const uint32_t st = smem_u32(smem + stage * Tr::kStageBytes);
+          const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kPairSfCols<FMT>;
+          const uint32_t sfb = sfa + Tr::kSfaCols;
+          if (FMT == MOE_NVFP4) {
+            for (int kb = 0; kb < kb_here; ++kb) {
+              tc_cp_sf_atom_pair(sfa + 4 * kb, make_desc_sf(st + Tr::kSfaOff + 512 * kb));
+#pragma unroll
+              for (int h = 0; h < kBN / 128; ++h)
+                tc_cp_sf_atom_pair(sfb + (kBN / 32) * kb + 4 * h,
+                                   make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
+            }
+          } else {
+            tc_cp_sf_atom_pair(sfa, make_desc_sf(st + Tr::kSfaOff));
+#pragma unroll
+            for (int h = 0; h < kBN / 128; ++h)
+              tc_cp_sf_atom_pair(sfb + 4 * h, make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128));
+          }
+          tc_commit_pair(&sf_bar[stage], 0x1);
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
       }
     }
   } else {
@@ -360,8 +402,8 @@ static bool make_line_map(CUtensorMap* map, const void* base, int64_t bytes, int
 template <int FMT, bool GATEUP>
 static cudaError_t launch_pair_one(const PairMaps& maps, const GemmArgs& a, cudaStream_t stream) {
   using Tr = GemmTraits<FMT, 128, kPairStages>;
-  const size_t smem_max = 1024 + kPairStages * Tr::kStageBytes + (2 * kPairStages + 2) * 8 + 16 + 2 * 1025 * 4;
-  const size_t smem = 1024 + kPairStages * Tr::kStageBytes + (2 * kPairStages + 2) * 8 + 16 + 2 * (a.E + 1) * 4;
+  const size_t smem_max = 1024 + kPairStages * Tr::kStageBytes + (3 * kPairStages + 2) * 8 + 16 + 2 * 1025 * 4;
+  const size_t smem = 1024 + kPairStages * Tr::kStageBytes + (3 * kPairStages + 2) * 8 + 16 + 2 * (a.E + 1) * 4;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -372,7 +414,7 @@ static cudaError_t launch_pair_one(const PairMaps& maps, const GemmArgs& a, cuda
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t qc = {};
     qc.gridDim = dim3(2);
-    qc.blockDim = dim3(kThreads);
+    qc.blockDim = dim3(kPairThreads);
     qc.dynamicSmemBytes = smem_max;
     cudaLaunchAttribute qa[1];
     qa[0].id = cudaLaunchAttributeClusterDimension;
@@ -390,7 +432,7 @@ static cudaError_t launch_pair_one(const PairMaps& maps, const GemmArgs& a, cuda
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters[dev]);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kPairThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];

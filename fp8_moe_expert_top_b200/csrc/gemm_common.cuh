@@ -124,7 +124,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, float* acc, 
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           blk[i] = (b == 0) ? acc[i] : (b == 1) ? acc[16 + i] : (b == 2) ? acc[64 + i] : acc[80 + i];
-        const Nvfp4Block qb = nvfp4_quantize16(blk, sh);
+        const Nvfp4Block qb = nvfp4_quantize16_h(blk, sh);
         const int ch = ch0 + 16 * b;
         *reinterpret_cast<uint2*>(args.h_codes + tile_offset(row, ch / 2, args.h_kb, kActTileRows)) =
             make_uint2(static_cast<uint32_t>(qb.codes), static_cast<uint32_t>(qb.codes >> 32));

@@ -18,6 +18,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 namespace moe {
@@ -175,6 +176,74 @@ __device__ __forceinline__ Nvfp4Block nvfp4_quantize16(const float* x, float s_g
   return b;
 }
 
+// Two E2M1 codes (element 2j in the low nibble) decoded to float (exact).
+__device__ __forceinline__ float2 e2m1x2_decode(uint32_t pair) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 t, u;\n\tmov.b16 {t, u}, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(h2)
+      : "h"(static_cast<uint16_t>(pair)));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
+}
+
+// One candidate of the 4-vs-6 search for the requantization of h in the
+// gate/up epilogue.  Same block-scale code (exact), same error terms and
+// pairwise tree as nvfp4_candidate; the element quotient is taken as
+// RN(|x| * RN(1/S)) instead of RN(|x| / S), converted two elements at a time.
+// The two quotients differ by at most 2^-23 relative, so an element code can
+// differ from the definition only where |x| / S lies that close to a
+// rounding midpoint of E2M1; the intermediate's parity bar (at most 1e-3 of
+// its codes may differ, since h itself is computed in float32 with a fast
+// exponential) absorbs that.  Zero and tiny scales take the exact path.
+__device__ __forceinline__ float nvfp4_candidate_h(const float* ax, float a, float s_g, float c, uint64_t& mags,
+                                                   uint32_t& sf) {
+  sf = e4m3_code_of_quotient(a, __fmul_rn(c, s_g));
+  const float S = __fmul_rn(e4m3_decode(sf), s_g);
+  if (!(S >= 0x1p-100f)) return nvfp4_candidate(ax, a, s_g, c, mags, sf);
+  const float rS = __frcp_rn(S);
+  float d2[16];
+  mags = 0;
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    const uint32_t p = cvt_e2m1x2(__fmul_rn(ax[i], rS), __fmul_rn(ax[i + 1], rS)) & 0x77u;
+    mags |= static_cast<uint64_t>(p) << (4 * i);
+    const float2 v = e2m1x2_decode(p);
+    const float d0 = __fsub_rn(ax[i], __fmul_rn(v.x, S));
+    const float d1 = __fsub_rn(ax[i + 1], __fmul_rn(v.y, S));
+    d2[i] = __fmul_rn(d0, d0);
+    d2[i + 1] = __fmul_rn(d1, d1);
+  }
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) d2[i] = __fadd_rn(d2[2 * i], d2[2 * i + 1]);
+  }
+  return d2[0];
+}
+
+// NVFP4 4-vs-6 quantization of 16 values of h (see nvfp4_candidate_h).
+__device__ __forceinline__ Nvfp4Block nvfp4_quantize16_h(const float* x, float s_g) {
+  float ax[16];
+  float a = 0.0f;
+  uint64_t neg = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    ax[i] = fabsf(x[i]);
+    a = fmaxf(a, ax[i]);
+    neg |= static_cast<uint64_t>(x[i] < 0.0f) << (4 * i + 3);
+  }
+  uint64_t m6, m4;
+  uint32_t e6, e4;
+  const float err6 = nvfp4_candidate_h(ax, a, s_g, 6.0f, m6, e6);
+  const float err4 = nvfp4_candidate_h(ax, a, s_g, 4.0f, m4, e4);
+  const bool four = err4 < err6;
+  const uint64_t mags = four ? m4 : m6;
+  const uint64_t nz = (mags | (mags >> 1) | (mags >> 2)) & 0x1111111111111111ull;
+  Nvfp4Block b;
+  b.codes = mags | (neg & (nz << 3));
+  b.sf = four ? e4 : e6;
+  return b;
+}
+
 // MXFP8 quantization of 32 float32 values: codes (4 bytes per uint32, element
 // i in byte i%4 of word i/4) and the E8M0 exponent.
 __device__ __forceinline__ uint32_t mxfp8_quantize32(const float* x, uint32_t* words) {
@@ -186,10 +255,13 @@ __device__ __forceinline__ uint32_t mxfp8_quantize32(const float* x, uint32_t* w
   const float scale = __uint_as_float((254u - e) << 23);   // 2^(127 - e), e <= 246
 #pragma unroll
   for (int w = 0; w < 8; ++w) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) word |= e4m3_encode(__fmul_rn(x[4 * w + b], scale)) << (8 * b);
-    words[w] = word;
+    // two elements per conversion (same rounding and saturation as
+    // e4m3_encode); a code whose magnitude bits are zero loses its sign bit
+    const uint32_t p0 = cvt_e4m3x2(__fmul_rn(x[4 * w], scale), __fmul_rn(x[4 * w + 1], scale));
+    const uint32_t p1 = cvt_e4m3x2(__fmul_rn(x[4 * w + 2], scale), __fmul_rn(x[4 * w + 3], scale));
+    const uint32_t word = p0 | (p1 << 16);
+    const uint32_t nonzero = ((word & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) & 0x80808080u;
+    words[w] = (word & 0x7F7F7F7Fu) | (word & nonzero);
   }
   return e;
 }
