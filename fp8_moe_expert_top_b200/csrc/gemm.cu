@@ -20,7 +20,7 @@
 // K tile fastest, the 128-byte swizzle applied in memory), so every stage is
 // one contiguous 1-D bulk copy per operand.
 //
-// Warp roles (352 threads):
+// Warp roles (384 threads):
 //   warp 0      producer: bulk copies of A, B and their scale atoms into a
 //               4-stage ring
 //   warp 1      MMA issuer: TMEM allocation, tcgen05.mma block-scaled
@@ -28,11 +28,13 @@
 //   warps 2-9   epilogue: tcgen05.ld of the 128x256 fp32 accumulator (two
 //               warps per TMEM lane quarter, 128 columns each), tensor scales,
 //               SwiGLU + requantization (gate/up) or bf16 store (down)
-//   warp 10     scale copier: moves a stage's scale atoms SMEM -> TMEM with
-//               tcgen05.cp into that stage's own TMEM columns.  Copies take
-//               as long as the MMAs in the tensor pipe; issued from their own
-//               thread they run ahead of and overlap the MMA stream instead
-//               of sitting in front of every stage's MMAs.
+//   warps 10-11 scale copiers: the stage's scale atoms SMEM -> TMEM
+//               (tcgen05.cp), alternate k blocks each, into per-stage TMEM
+//               columns.
+// A tcgen05.cp holds its issuing thread for about 50 cycles, copies from
+// different threads overlap, and copies issued by the MMA thread queue behind
+// its MMAs; so the MMA thread issues none and each stage's 12 (NVFP4) copies
+// are spread over two threads of their own.
 // Every mbarrier wait is bounded; a wait that runs out raises a CTA-wide
 // abort flag, every role stops issuing, TMEM is freed and a status bit is
 // set.
@@ -48,7 +50,8 @@
 namespace moe {
 
 constexpr int kStages = 4;
-constexpr int kThreadsOne = kThreads + 32;  // + the scale-copier warp
+constexpr int kCopierWarps = 2;  // scale-copier warps
+constexpr int kThreadsOne = kThreads + 32 * kCopierWarps;
 // TMEM columns of one stage's scales: NVFP4 4 (A) + 8 (B) per 64-element k
 // block x 4 k blocks; MXFP8 4 + 8 (one 32-bit column holds 4 k blocks)
 template <int FMT>
@@ -94,7 +97,7 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&sf_bar[s], 1);
+      mbar_init(&sf_bar[s], kCopierWarps);
     }
     mbar_init(tfull_bar, 1);
     mbar_init(tempty_bar, 32 * kEpiWarps);
@@ -184,8 +187,8 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
         tc_fence_after();
         bool ok = true;
         for (int kt = 0; kt < k_tiles; ++kt) {
-          // the scale copier has seen the stage's operands land and its
-          // scale copies have completed (the operand wait then returns at once)
+          // the scale copiers have seen the stage's operands land and their
+          // copies have completed (the operand wait then returns at once)
           if (!mbar_wait(&sf_bar[stage], phase, abort_flag) || !mbar_wait(&full_bar[stage], phase, abort_flag)) {
             fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
             ok = false;
@@ -221,8 +224,9 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
         acc_phase ^= 1u;
       }
     }
-  } else if (warp == kThreads / 32) {
-    // ------------------------------------------------------------ scale copier
+  } else if (warp >= kThreads / 32) {
+    // ------------------------------------------------------------ scale copiers
+    const int part = warp - kThreads / 32;  // copies the scales of k blocks part, part + kCopierWarps, ...
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -243,17 +247,19 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
           const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kSfColsPerStage<FMT>;
           const uint32_t sfb = sfa + Tr::kSfaCols;
           if (FMT == MOE_NVFP4) {
-            for (int kb = 0; kb < kb_here; ++kb) {
+            for (int kb = part; kb < kb_here; kb += kCopierWarps) {
               tc_cp_sf_atom(sfa + 4 * kb, make_desc_sf(st + Tr::kSfaOff + 512 * kb));
 #pragma unroll
               for (int h = 0; h < kBN / 128; ++h)
                 tc_cp_sf_atom(sfb + (kBN / 32) * kb + 4 * h,
-                              make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
+                      make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
             }
-          } else {
+          } else if (part == 0) {
             tc_cp_sf_atom(sfa, make_desc_sf(st + Tr::kSfaOff));
+            tc_cp_sf_atom(sfb, make_desc_sf(st + Tr::kSfbOff));
+          } else {
 #pragma unroll
-            for (int h = 0; h < kBN / 128; ++h)
+            for (int h = 1; h < kBN / 128; ++h)
               tc_cp_sf_atom(sfb + 4 * h, make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128));
           }
           tc_commit(&sf_bar[stage]);

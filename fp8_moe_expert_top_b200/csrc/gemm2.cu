@@ -15,9 +15,9 @@
 // the MMA warp's commits arrive on the "empty" and "accumulator full"
 // barriers of both CTAs (tcgen05.commit multicast); both CTAs' epilogue
 // threads release the accumulator on the even CTA's "accumulator empty"
-// barrier.  A scale-copier warp in the even CTA moves both CTAs' scale atoms
-// into TMEM (tcgen05.cp.cta_group::2, per-stage columns) and signals the MMA
-// thread, as in gemm.cu.  Waits are bounded as in gemm.cu.
+// barrier.  Scale atoms reach TMEM as in gemm.cu (per-stage columns, copied
+// by two copier warps of the even CTA with tcgen05.cp.cta_group::2).  Waits
+// are bounded as in gemm.cu.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -31,7 +31,8 @@
 namespace moe {
 
 constexpr int kPairStages = 5;
-constexpr int kPairThreads = kThreads + 32;  // + the scale-copier warp
+constexpr int kCopierWarps = 2;  // scale-copier warps (even CTA)
+constexpr int kPairThreads = kThreads + 32 * kCopierWarps;
 template <int FMT>
 constexpr uint32_t kPairSfCols = (FMT == MOE_NVFP4) ? 48u : 12u;  // TMEM scale columns per stage
 static_assert(kBN + kPairStages * 48 <= kTmemCols, "scale buffers do not fit in TMEM");
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     for (int s = 0; s < kPairStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&sf_bar[s], 1);
+      mbar_init(&sf_bar[s], kCopierWarps);
     }
     mbar_init(tfull_bar, 1);
     mbar_init(tempty_bar, 2 * 32 * kEpiWarps);
@@ -279,12 +280,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         acc_phase ^= 1u;
       }
     }
-  } else if (warp == kThreads / 32) {
-    // ------------------------------------------------------------ scale copier (even CTA)
-    // Copies each CTA's scale atoms into its own TMEM (cta_group::2), into the
-    // stage's own columns, and signals the MMA thread.  The columns were last
-    // read by the MMAs of the same stage one ring turn ago, which completed
-    // before the stage was released and refilled.
+  } else if (warp >= kThreads / 32) {
+    // ------------------------------------------------------------ scale copiers (even CTA)
+    // Copy each CTA's scale atoms of every kCopierWarps-th k block into its
+    // own TMEM (cta_group::2), into the stage's own columns, and signal the MMA
+    // thread.  The columns were last read by the MMAs of the same stage one
+    // ring turn ago, which completed before the stage was released and refilled.
+    const int part = warp - kThreads / 32;
     if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
@@ -302,17 +304,19 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kPairSfCols<FMT>;
           const uint32_t sfb = sfa + Tr::kSfaCols;
           if (FMT == MOE_NVFP4) {
-            for (int kb = 0; kb < kb_here; ++kb) {
+            for (int kb = part; kb < kb_here; kb += kCopierWarps) {
               tc_cp_sf_atom_pair(sfa + 4 * kb, make_desc_sf(st + Tr::kSfaOff + 512 * kb));
 #pragma unroll
               for (int h = 0; h < kBN / 128; ++h)
                 tc_cp_sf_atom_pair(sfb + (kBN / 32) * kb + 4 * h,
-                                   make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
+                      make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
             }
-          } else {
+          } else if (part == 0) {
             tc_cp_sf_atom_pair(sfa, make_desc_sf(st + Tr::kSfaOff));
+            tc_cp_sf_atom_pair(sfb, make_desc_sf(st + Tr::kSfbOff));
+          } else {
 #pragma unroll
-            for (int h = 0; h < kBN / 128; ++h)
+            for (int h = 1; h < kBN / 128; ++h)
               tc_cp_sf_atom_pair(sfb + 4 * h, make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128));
           }
           tc_commit_pair(&sf_bar[stage], 0x1);
