@@ -125,11 +125,6 @@ class ClockSampler:
                 "samples": len(sms)}
 
 
-def file_sha(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
-
-
 # --------------------------------------------------------------------------- workload
 
 def build_layer(wl, device, T):
@@ -322,7 +317,8 @@ def run_ours(args, wl, ws, rank, local):
         "e2e": {"value": ws * T * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": int(x_h.numel() * 2 + lg_h.numel() * 4),
                 "d2h_bytes_per_step": int(T * wl.d_model * 2)},
-        "gpu_launches": (7 if T > 1024 else 5) * args.steps,
+        # per step: route top-k, scan, scatter; permute; gate/up; down; combine
+        "gpu_launches": 7 * args.steps,
         "clocks": clk,
     }
     return out, layer
@@ -339,10 +335,18 @@ def measured_traffic(workload, phase):
     ent = d.get(workload, {}).get(phase)
     if not ent:
         return None
-    src = os.path.join(ROOT, "fp8_moe_expert_top_b200", "csrc", "gemm.cu")
-    if ent.get("gemm_sha") != file_sha(src):
+    if ent.get("gemm_sha") != gemm_source_sha():
         return None
     return ent.get("bytes")
+
+
+def gemm_source_sha():
+    """Hash of the sources the one-SM GEMM kernel is compiled from."""
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "gemm_common.cuh", "common.cuh", "quant.cuh"):
+        with open(os.path.join(ROOT, "fp8_moe_expert_top_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -442,13 +446,18 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=None,
                     help="profiling only: override the number of experts (smaller device footprint for ncu)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="profiling only: override the number of tokens (with --experts, keeps rows per expert)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = inputs.WORKLOADS[args.workload]
-    if args.experts is not None:
+    if args.experts is not None or args.tokens is not None:
         import dataclasses
-        wl = dataclasses.replace(wl, name=f"{wl.name}_e{args.experts}", num_experts=args.experts)
+        if args.experts is not None:
+            wl = dataclasses.replace(wl, name=f"{wl.name}_e{args.experts}", num_experts=args.experts)
+        if args.tokens is not None:
+            wl = dataclasses.replace(wl, name=f"{wl.name}_t{args.tokens}", T=args.tokens)
     ws, rank, local = dist_env()
     if ws != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {ws}", file=sys.stderr)
