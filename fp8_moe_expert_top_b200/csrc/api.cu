@@ -34,15 +34,6 @@ moe_status check_T(int64_t T) { return (T < 0 || T > kMaxTokens) ? MOE_ERR_UNSUP
 
 moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// GEMMs on SM pairs (256-row tiles) are built and tested but not selected:
-// the one-SM kernel with its separate scale-copier warp is faster at every
-// measured size.
-bool use_pair(const moe_config* c, int64_t T) {
-  (void)c;
-  (void)T;
-  return false;
-}
-
 int64_t max_rows(const moe_config* c, int64_t T) {
   const int64_t slots = T * c->top_k;
   const int64_t touched = slots < c->num_experts ? slots : c->num_experts;
@@ -179,7 +170,6 @@ moe_status moe_forward_gateup(const moe_config* cfg, int64_t T, const void* pack
   moe::GemmLaunch g{};
   g.fmt = cfg->fmt;
   g.gateup = true;
-  g.pair = use_pair(cfg, T);
   g.E = cfg->num_experts;
   g.K = cfg->d_model;
   g.n_rows_b = 2 * cfg->d_ffn;
@@ -216,7 +206,6 @@ moe_status moe_forward_down(const moe_config* cfg, int64_t T, const void* packed
   moe::GemmLaunch g{};
   g.fmt = cfg->fmt;
   g.gateup = false;
-  g.pair = use_pair(cfg, T);
   g.E = cfg->num_experts;
   g.K = cfg->d_ffn;
   g.n_rows_b = cfg->d_model;

@@ -371,7 +371,6 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
   a.n_rows_b = g.n_rows_b;
   a.sf_rb_stride = static_cast<int64_t>(g.K / sfvec) * 128;
   a.b_sf_expert_stride = static_cast<int64_t>(g.n_rows_b) * (g.K / sfvec);
-  if (g.pair) return launch_gemm_pair(g, a, stream);
   if (g.fmt == MOE_NVFP4)
     return g.gateup ? launch_one<MOE_NVFP4, true>(a, stream) : launch_one<MOE_NVFP4, false>(a, stream);
   return g.gateup ? launch_one<MOE_MXFP8, true>(a, stream) : launch_one<MOE_MXFP8, false>(a, stream);

@@ -1,6 +1,6 @@
-// Pieces shared by the 1-SM and 2-SM persistent block-scaled GEMM kernels:
-// tile constants, kernel arguments, the expert lookup and the epilogue that
-// turns a 128-column slice of one accumulator row into outputs.
+// Pieces of the persistent block-scaled GEMM kernel: tile constants, kernel
+// arguments, the expert lookup and the epilogue that turns a 128-column slice
+// of one accumulator row into outputs.
 #pragma once
 
 #include <cstdint>
@@ -18,7 +18,7 @@ constexpr int kEpiWarps = 8;             // two warps per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 
-// B_ROWS: weight rows a CTA loads per stage (256 on one SM, 128 per SM of a pair).
+// B_ROWS: weight rows a CTA loads per stage.
 template <int FMT, int B_ROWS, int STAGES>
 struct GemmTraits {
   static constexpr int kStages = STAGES;

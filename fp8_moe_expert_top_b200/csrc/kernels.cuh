@@ -26,7 +26,6 @@ cudaError_t launch_quantize_weights(int fmt, int E, int H, int I, int expert_beg
 struct GemmLaunch {
   int fmt;
   bool gateup;
-  bool pair;              // run on SM pairs (M = 256 tiles): experts average more than one row block
   int E, K, n_rows_b;     // K in elements, rows of B per expert (2I or H)
   int64_t R_max;
   const uint8_t* a_codes;
@@ -45,7 +44,5 @@ struct GemmLaunch {
   uint32_t* status;
 };
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream);
-struct GemmArgs;
-cudaError_t launch_gemm_pair(const GemmLaunch& g, const GemmArgs& a, cudaStream_t stream);
 
 }  // namespace moe

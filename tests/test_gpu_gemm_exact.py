@@ -51,12 +51,11 @@ def to_rows_bytes(fmt, codes):
 
 
 # Expert row counts and token counts: a decode-like case (T * k <= 128 * E)
-# and a prefill-like one (T * k > 128 * E, the shape class that may run on SM
-# pairs with 256-row tiles), with odd row-block counts so that a pair would
-# end past an expert's rows and past the last expert.
+# and a prefill-like one (several 128-row blocks per expert, odd block counts,
+# partly filled last blocks).
 CASES = {
-    "one_sm": (np.array([130, 0, 5, 256], dtype=np.int32), 391),
-    "sm_pair": (np.array([200, 50, 300], dtype=np.int32), 550),
+    "decode_like": (np.array([130, 0, 5, 256], dtype=np.int32), 391),
+    "prefill_like": (np.array([200, 50, 300], dtype=np.int32), 550),
 }
 
 
@@ -65,10 +64,10 @@ CASES = {
 @pytest.mark.parametrize("H,I", [(256, 128), (512, 256), (1024, 384)])
 @pytest.mark.parametrize("case", sorted(CASES))
 def test_gemm_integer_exact(cuda_device, fmt, H, I, case):
-    rng = np.random.default_rng(H * 7 + I + (1 if fmt == "mxfp8" else 0) + (3 if case == "sm_pair" else 0))
+    rng = np.random.default_rng(H * 7 + I + (1 if fmt == "mxfp8" else 0) + (3 if case == "prefill_like" else 0))
     counts, T = CASES[case]
     E, k = len(counts), 1
-    assert (T * k > 128 * E) == (case == "sm_pair")
+    assert (T * k > 128 * E) == (case == "prefill_like")
     assert counts.sum() == T
     offsets = np.concatenate([[0], np.cumsum((counts + 127) // 128 * 128)]).astype(np.int32)
     cfg = B.make_config(E, k, H, I, fmt)

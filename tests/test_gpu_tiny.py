@@ -26,8 +26,8 @@ from helpers import ACT_TR, rel_fro, sfvec, tiled_codes, unswizzle_sf
 TINY = inputs.WORKLOADS["tiny_nvfp4"]
 TINY_MX = dataclasses.replace(TINY, name="tiny_mxfp8", fmt=inputs.MXFP8)
 # T * k > 128 * E: the prefill shape class (several 128-row blocks per expert)
-TINY_PAIR = dataclasses.replace(TINY, name="tiny_nvfp4_pair", T=1024)
-TINY_PAIR_MX = dataclasses.replace(TINY_PAIR, name="tiny_mxfp8_pair", fmt=inputs.MXFP8)
+TINY_PREFILL = dataclasses.replace(TINY, name="tiny_nvfp4_prefill", T=1024)
+TINY_PREFILL_MX = dataclasses.replace(TINY_PREFILL, name="tiny_mxfp8_prefill", fmt=inputs.MXFP8)
 
 _layers = {}
 
@@ -101,7 +101,7 @@ def test_weights_bit_exact(cuda_device, wl):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("wl", [TINY, TINY_MX, TINY_PAIR, TINY_PAIR_MX], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [TINY, TINY_MX, TINY_PREFILL, TINY_PREFILL_MX], ids=lambda w: w.name)
 def test_layer_seeded_inputs(cuda_device, wl):
     layer = get_layer(wl, cuda_device)
     x, lg = inputs.make_x(wl), inputs.make_logits(wl)
@@ -132,9 +132,9 @@ def test_layer_edge_cases(cuda_device, wl, case):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("wl", [TINY_PAIR, TINY_PAIR_MX], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [TINY_PREFILL, TINY_PREFILL_MX], ids=lambda w: w.name)
 @pytest.mark.parametrize("case", ["hot_experts", "empty_experts", "ragged"])
-def test_pair_layer_edge_cases(cuda_device, wl, case):
+def test_prefill_layer_edge_cases(cuda_device, wl, case):
     """Prefill-shaped layer with skewed routing, empty experts and a ragged batch."""
     layer = get_layer(wl, cuda_device)
     if case == "hot_experts":
