@@ -74,55 +74,105 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and throttle-reason samples during the timed region.
 
+    NVML is polled from a thread every ~2 ms (the timed regions of the short
+    layers last a few tens of milliseconds); start() returns once the first
+    sample is in.  Falls back to `nvidia-smi -lms` when NVML is unavailable.
+    Only reads the GPU's state.
+    """
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.samples = []
+        self.thread = None
         self.proc = None
-        self.path = os.path.join("/tmp", f"moe_clocks_{os.getpid()}.csv")
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except pynvml.NVMLError:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.dev)
 
     def start(self):
+        import threading
+        try:
+            nv, h = self._nvml_handle()
+        except Exception:  # no NVML: nvidia-smi at its shortest interval
+            self._start_smi()
+            return
+        self.stop_flag = threading.Event()
+        first = threading.Event()
+        max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+
+        def run():
+            while True:
+                try:
+                    self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), max_mhz,
+                                         nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                except nv.NVMLError:
+                    pass
+                first.set()
+                if self.stop_flag.wait(0.002):
+                    break
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+        first.wait(5.0)
+
+    def _start_smi(self):
+        self.path = os.path.join("/tmp", f"moe_clocks_{os.getpid()}.csv")
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            samples = self.samples
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+            samples = []
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) < 9:
+                        continue
+                    try:
+                        mask = sum(bit for (_, bit), v in zip(self.REASONS, parts[5:9])
+                                   if v.lower().startswith("active"))
+                        samples.append((float(parts[1]), float(parts[2]), mask))
+                    except ValueError:
+                        continue
+            os.unlink(self.path)
+        else:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.f.close()
-        sms, maxs, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sms.append(float(parts[1]))
-                    maxs.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower().startswith("active"):
-                        reasons.add(n)
-        os.unlink(self.path)
-        if not sms:
+        if not samples:
             return None
-        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
-                "samples": len(sms)}
+        reasons = sorted({n for _, _, m in samples for n, bit in self.REASONS if m & bit})
+        return {"sm_mhz": statistics.median(s[0] for s in samples), "sm_max_mhz": max(s[1] for s in samples),
+                "reasons": reasons, "samples": len(samples),
+                "source": "nvml, 2 ms" if self.thread is not None else "nvidia-smi, 50 ms"}
 
 
 # --------------------------------------------------------------------------- workload

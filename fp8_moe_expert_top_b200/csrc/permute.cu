@@ -32,36 +32,41 @@ __device__ __forceinline__ void load16_bf16(const __nv_bfloat16* p, float* f) {
   }
 }
 
-// One thread per (token, scale block): 16 elements for NVFP4, 32 for MXFP8.
-// The block is read once, quantized once, and its codes and scale are written
-// to each of the token's k rows.
+// One thread per (token, 32 elements): two NVFP4 blocks or one MXFP8 block.
+// The elements are read once, quantized once, and their codes (one 16-byte
+// chunk for NVFP4, two for MXFP8) and scale byte(s) are written to each of
+// the token's k rows.
 template <int FMT>
 __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const __nv_bfloat16* __restrict__ x,
                                                       const float* __restrict__ act_scale,
                                                       const int32_t* __restrict__ slot_to_row,
                                                       uint8_t* __restrict__ a_codes, uint8_t* __restrict__ a_sf) {
-  constexpr int kBlock = (FMT == MOE_NVFP4) ? 16 : 32;
-  const int nsf = H / kBlock;
+  constexpr int kSfVec = (FMT == MOE_NVFP4) ? 16 : 32;
+  const int nsf = H / kSfVec;
+  const int n32 = H / 32;  // 32-element groups per token
   const int64_t id = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   pdl_wait();
   pdl_trigger();
-  if (id >= static_cast<int64_t>(T) * nsf) return;
-  const int t = static_cast<int>(id / nsf);
-  const int b = static_cast<int>(id % nsf);
-  const __nv_bfloat16* src = x + static_cast<int64_t>(t) * H + kBlock * b;
-  float f[kBlock];
-#pragma unroll
-  for (int i = 0; i < kBlock / 16; ++i) load16_bf16(src + 16 * i, f + 16 * i);
+  if (id >= static_cast<int64_t>(T) * n32) return;
+  const int t = static_cast<int>(id / n32);
+  const int g = static_cast<int>(id % n32);
+  float f[32];
+  load16_bf16(x + static_cast<int64_t>(t) * H + 32 * g, f);
+  load16_bf16(x + static_cast<int64_t>(t) * H + 32 * g + 16, f + 16);
   const int64_t kb = kb_padded(H, FMT == MOE_NVFP4 ? 4 : 8);
   if (FMT == MOE_NVFP4) {
-    const Nvfp4Block q = nvfp4_quantize16(f, __ldg(act_scale));
-    const uint2 c = make_uint2(static_cast<uint32_t>(q.codes), static_cast<uint32_t>(q.codes >> 32));
+    const float s_x = __ldg(act_scale);
+    const Nvfp4Block q0 = nvfp4_quantize16(f, s_x);
+    const Nvfp4Block q1 = nvfp4_quantize16(f + 16, s_x);
+    const uint4 c = make_uint4(static_cast<uint32_t>(q0.codes), static_cast<uint32_t>(q0.codes >> 32),
+                               static_cast<uint32_t>(q1.codes), static_cast<uint32_t>(q1.codes >> 32));
+    const uint16_t sf = static_cast<uint16_t>(q0.sf | (q1.sf << 8));
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (j >= k) break;
       const int64_t r = __ldg(slot_to_row + static_cast<int64_t>(t) * k + j);
-      *reinterpret_cast<uint2*>(a_codes + tile_offset(r, 8 * b, kb, kActTileRows)) = c;
-      a_sf[sf_offset(r, b, nsf)] = static_cast<uint8_t>(q.sf);
+      *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 16 * g, kb, kActTileRows)) = c;
+      *reinterpret_cast<uint16_t*>(a_sf + sf_offset(r, 2 * g, nsf)) = sf;  // blocks 2g, 2g + 1: adjacent bytes
     }
   } else {
     uint32_t w[8];
@@ -70,10 +75,10 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
     for (int j = 0; j < 8; ++j) {
       if (j >= k) break;
       const int64_t r = __ldg(slot_to_row + static_cast<int64_t>(t) * k + j);
-      *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 32 * b, kb, kActTileRows)) = make_uint4(w[0], w[1], w[2], w[3]);
-      *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 32 * b + 16, kb, kActTileRows)) =
+      *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 32 * g, kb, kActTileRows)) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 32 * g + 16, kb, kActTileRows)) =
           make_uint4(w[4], w[5], w[6], w[7]);
-      a_sf[sf_offset(r, b, nsf)] = static_cast<uint8_t>(e);
+      a_sf[sf_offset(r, g, nsf)] = static_cast<uint8_t>(e);
     }
   }
 }
@@ -81,7 +86,7 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
 cudaError_t launch_permute(int fmt, int T, int H, int k, const void* x, const float* act_scale,
                            const int32_t* slot_to_row, uint8_t* a_codes, uint8_t* a_sf, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  const int64_t n = static_cast<int64_t>(T) * (H / (fmt == MOE_NVFP4 ? 16 : 32));
+  const int64_t n = static_cast<int64_t>(T) * (H / 32);
   const dim3 grid(static_cast<unsigned>((n + 255) / 256)), block(256);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (fmt == MOE_NVFP4)

@@ -92,15 +92,6 @@ static __device__ __noinline__ uint32_t e4m3_code_exact(float num, float den) {
   return e4m3_encode(__fdiv_rn(num, den));
 }
 
-// E2M1 magnitude code of RN(num / den), num >= 0, den > 0, with 1/den given.
-__device__ __forceinline__ uint32_t e2m1_code_of_quotient(float num, float den, float rden) {
-  const float q = __fmul_rn(num, rden);
-  const uint32_t pair = cvt_e2m1x2(__fmul_rn(q, kBracketLo), __fmul_rn(q, kBracketHi));
-  const uint32_t lo = pair & 0x7u, hi = (pair >> 4) & 0x7u;
-  if (lo == hi) return lo;
-  return e2m1_code_exact(num, den);
-}
-
 // E4M3 code of RN(num / den), num >= 0, den > 0.
 __device__ __forceinline__ uint32_t e4m3_code_of_quotient(float num, float den) {
   if (num == 0.0f) return 0u;
@@ -109,6 +100,15 @@ __device__ __forceinline__ uint32_t e4m3_code_of_quotient(float num, float den) 
   const uint32_t lo = pair & 0xFFu, hi = pair >> 8;
   if (lo == hi) return lo;
   return e4m3_code_exact(num, den);
+}
+
+// Two E2M1 codes (element 2j in the low nibble) decoded to float (exact).
+__device__ __forceinline__ float2 e2m1x2_decode(uint32_t pair) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 t, u;\n\tmov.b16 {t, u}, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(h2)
+      : "h"(static_cast<uint16_t>(pair)));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
 }
 
 // One candidate of the 4-vs-6 search on magnitudes ax[16] (block maximum a
@@ -128,11 +128,23 @@ __device__ __forceinline__ float nvfp4_candidate(const float* ax, float a, float
   } else if (S >= 0x1p-100f) {
     const float rS = __frcp_rn(S);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t m = e2m1_code_of_quotient(ax[i], S, rS);
-      mags |= static_cast<uint64_t>(m) << (4 * i);
-      const float d = __fsub_rn(ax[i], __fmul_rn(e2m1_mag_value(m), S));
-      d2[i] = __fmul_rn(d, d);
+    for (int i = 0; i < 16; i += 2) {
+      // both ends of both elements' brackets, two elements per conversion
+      const float q0 = __fmul_rn(ax[i], rS), q1 = __fmul_rn(ax[i + 1], rS);
+      const uint32_t lo = cvt_e2m1x2(__fmul_rn(q0, kBracketLo), __fmul_rn(q1, kBracketLo));
+      const uint32_t hi = cvt_e2m1x2(__fmul_rn(q0, kBracketHi), __fmul_rn(q1, kBracketHi));
+      uint32_t p = lo & 0x77u;
+      if (lo != hi) {  // an end differs: settle that element by the exact division
+        const uint32_t m0 = ((lo ^ hi) & 0x7u) ? e2m1_code_exact(ax[i], S) : (lo & 0x7u);
+        const uint32_t m1 = ((lo ^ hi) & 0x70u) ? e2m1_code_exact(ax[i + 1], S) : ((lo >> 4) & 0x7u);
+        p = m0 | (m1 << 4);
+      }
+      mags |= static_cast<uint64_t>(p) << (4 * i);
+      const float2 v = e2m1x2_decode(p);
+      const float d0 = __fsub_rn(ax[i], __fmul_rn(v.x, S));
+      const float d1 = __fsub_rn(ax[i + 1], __fmul_rn(v.y, S));
+      d2[i] = __fmul_rn(d0, d0);
+      d2[i + 1] = __fmul_rn(d1, d1);
     }
   } else {  // tiny scales: exact division throughout
 #pragma unroll 1
@@ -176,14 +188,6 @@ __device__ __forceinline__ Nvfp4Block nvfp4_quantize16(const float* x, float s_g
   return b;
 }
 
-// Two E2M1 codes (element 2j in the low nibble) decoded to float (exact).
-__device__ __forceinline__ float2 e2m1x2_decode(uint32_t pair) {
-  uint32_t h2;
-  asm("{\n\t.reg .b8 t, u;\n\tmov.b16 {t, u}, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
-      : "=r"(h2)
-      : "h"(static_cast<uint16_t>(pair)));
-  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
-}
 
 // One candidate of the 4-vs-6 search for the requantization of h in the
 // gate/up epilogue.  Same block-scale code (exact), same error terms and
