@@ -83,7 +83,8 @@ class ClockSampler:
     """
 
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
-               ("sw_power_cap", 0x4))
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80), ("gpu_idle", 0x1),
+               ("applications_clocks_setting", 0x2), ("sync_boost", 0x10), ("display_clock_setting", 0x100))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -119,7 +120,8 @@ class ClockSampler:
             while True:
                 try:
                     self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), max_mhz,
-                                         nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                                         nv.nvmlDeviceGetCurrentClocksEventReasons(h),
+                                         nv.nvmlDeviceGetPowerUsage(h) / 1000.0))
                 except nv.NVMLError:
                     pass
                 first.set()
@@ -159,9 +161,9 @@ class ClockSampler:
                     if len(parts) < 9:
                         continue
                     try:
-                        mask = sum(bit for (_, bit), v in zip(self.REASONS, parts[5:9])
+                        mask = sum(bit for (_, bit), v in zip(self.REASONS[:4], parts[5:9])
                                    if v.lower().startswith("active"))
-                        samples.append((float(parts[1]), float(parts[2]), mask))
+                        samples.append((float(parts[1]), float(parts[2]), mask, float(parts[3])))
                     except ValueError:
                         continue
             os.unlink(self.path)
@@ -169,9 +171,11 @@ class ClockSampler:
             return None
         if not samples:
             return None
-        reasons = sorted({n for _, _, m in samples for n, bit in self.REASONS if m & bit})
-        return {"sm_mhz": statistics.median(s[0] for s in samples), "sm_max_mhz": max(s[1] for s in samples),
-                "reasons": reasons, "samples": len(samples),
+        reasons = sorted({n for s_ in samples for n, bit in self.REASONS if s_[2] & bit})
+        clk = [s_[0] for s_ in samples]
+        return {"sm_mhz": statistics.median(clk), "sm_max_mhz": max(s_[1] for s_ in samples),
+                "sm_mhz_min": min(clk), "sm_mhz_max_seen": max(clk),
+                "power_w_max": round(max(s_[3] for s_ in samples), 1), "reasons": reasons, "samples": len(samples),
                 "source": "nvml, 2 ms" if self.thread is not None else "nvidia-smi, 50 ms"}
 
 
