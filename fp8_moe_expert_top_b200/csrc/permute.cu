@@ -7,6 +7,7 @@
 // separate quantization pass.  Here the producer of the GEMM1 operand is the
 // permute-gather: each token row is read once, quantized once (NVFP4 4-vs-6
 // or MXFP8) and written to each of its k expert rows.
+#include <algorithm>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -32,29 +33,41 @@ __device__ __forceinline__ void load16_bf16(const __nv_bfloat16* p, float* f) {
   }
 }
 
-// One thread per (token, 32 elements): two NVFP4 blocks or one MXFP8 block.
-// The elements are read once, quantized once, and their codes (one 16-byte
-// chunk for NVFP4, two for MXFP8) and scale byte(s) are written to each of
-// the token's k rows.
-template <int FMT>
+// One thread per (token, G elements): G = 32 (two NVFP4 blocks or one MXFP8
+// block) for large batches, G = 16 (one NVFP4 block) for small ones, where
+// more threads in flight matter more than fewer, wider stores.  The elements
+// are read once, quantized once, and their codes and scale byte(s) are
+// written to each of the token's k rows.
+template <int FMT, int G>
 __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const __nv_bfloat16* __restrict__ x,
                                                       const float* __restrict__ act_scale,
                                                       const int32_t* __restrict__ slot_to_row,
                                                       uint8_t* __restrict__ a_codes, uint8_t* __restrict__ a_sf) {
+  static_assert(G == 32 || (G == 16 && FMT == MOE_NVFP4), "group size");
   constexpr int kSfVec = (FMT == MOE_NVFP4) ? 16 : 32;
   const int nsf = H / kSfVec;
-  const int n32 = H / 32;  // 32-element groups per token
+  const int ng = H / G;  // groups per token
   const int64_t id = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   pdl_wait();
   pdl_trigger();
-  if (id >= static_cast<int64_t>(T) * n32) return;
-  const int t = static_cast<int>(id / n32);
-  const int g = static_cast<int>(id % n32);
-  float f[32];
-  load16_bf16(x + static_cast<int64_t>(t) * H + 32 * g, f);
-  load16_bf16(x + static_cast<int64_t>(t) * H + 32 * g + 16, f + 16);
+  if (id >= static_cast<int64_t>(T) * ng) return;
+  const int t = static_cast<int>(id / ng);
+  const int g = static_cast<int>(id % ng);
+  float f[G];
+#pragma unroll
+  for (int i = 0; i < G / 16; ++i) load16_bf16(x + static_cast<int64_t>(t) * H + G * g + 16 * i, f + 16 * i);
   const int64_t kb = kb_padded(H, FMT == MOE_NVFP4 ? 4 : 8);
-  if (FMT == MOE_NVFP4) {
+  if (FMT == MOE_NVFP4 && G == 16) {
+    const Nvfp4Block q = nvfp4_quantize16(f, __ldg(act_scale));
+    const uint2 c = make_uint2(static_cast<uint32_t>(q.codes), static_cast<uint32_t>(q.codes >> 32));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) break;
+      const int64_t r = __ldg(slot_to_row + static_cast<int64_t>(t) * k + j);
+      *reinterpret_cast<uint2*>(a_codes + tile_offset(r, 8 * g, kb, kActTileRows)) = c;
+      a_sf[sf_offset(r, g, nsf)] = static_cast<uint8_t>(q.sf);
+    }
+  } else if (FMT == MOE_NVFP4) {
     const float s_x = __ldg(act_scale);
     const Nvfp4Block q0 = nvfp4_quantize16(f, s_x);
     const Nvfp4Block q1 = nvfp4_quantize16(f + 16, s_x);
@@ -86,22 +99,32 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
 cudaError_t launch_permute(int fmt, int T, int H, int k, const void* x, const float* act_scale,
                            const int32_t* slot_to_row, uint8_t* a_codes, uint8_t* a_sf, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  const int64_t n = static_cast<int64_t>(T) * (H / 32);
-  const dim3 grid(static_cast<unsigned>((n + 255) / 256)), block(256);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  if (fmt == MOE_NVFP4)
-    return launch_pdl(permute_kernel<MOE_NVFP4>, grid, block, 0, stream, T, H, k, xb, act_scale, slot_to_row, a_codes,
-                      a_sf);
-  return launch_pdl(permute_kernel<MOE_MXFP8>, grid, block, 0, stream, T, H, k, xb, act_scale, slot_to_row, a_codes,
-                    a_sf);
+  const dim3 block(256);
+  // small batches (fewer 32-element groups than 256 per SM): one 16-element
+  // NVFP4 block per thread doubles the threads in flight
+  const bool small = fmt == MOE_NVFP4 && static_cast<int64_t>(T) * (H / 32) < 148 * 256;
+  const int G = small ? 16 : 32;
+  const dim3 grid(static_cast<unsigned>((static_cast<int64_t>(T) * (H / G) + 255) / 256));
+  if (fmt == MOE_NVFP4) {
+    if (small)
+      return launch_pdl(permute_kernel<MOE_NVFP4, 16>, grid, block, 0, stream, T, H, k, xb, act_scale, slot_to_row,
+                        a_codes, a_sf);
+    return launch_pdl(permute_kernel<MOE_NVFP4, 32>, grid, block, 0, stream, T, H, k, xb, act_scale, slot_to_row,
+                      a_codes, a_sf);
+  }
+  return launch_pdl(permute_kernel<MOE_MXFP8, 32>, grid, block, 0, stream, T, H, k, xb, act_scale, slot_to_row,
+                    a_codes, a_sf);
 }
 
 // y[t] = sum_j w[t][j] * out[row(t, j)], float32 in rank order, then bf16.
-// One CTA per token; each thread owns 8 consecutive channels per step.
-__global__ void __launch_bounds__(256) combine_kernel(int H, int k, const __nv_bfloat16* __restrict__ down_out,
-                                                      const float* __restrict__ topk_w,
-                                                      const int32_t* __restrict__ slot_to_row,
-                                                      __nv_bfloat16* __restrict__ y) {
+// One CTA per token, one thread per 8 consecutive channels (a block of
+// min(H / 8, 1024) threads, looping when H > 8192): the thread's k row loads
+// are all issued before the arithmetic.
+__global__ void __launch_bounds__(1024) combine_kernel(int H, int k, const __nv_bfloat16* __restrict__ down_out,
+                                                       const float* __restrict__ topk_w,
+                                                       const int32_t* __restrict__ slot_to_row,
+                                                       __nv_bfloat16* __restrict__ y) {
   const int t = blockIdx.x;
   pdl_wait();
   pdl_trigger();
@@ -113,14 +136,17 @@ __global__ void __launch_bounds__(256) combine_kernel(int H, int k, const __nv_b
     rows[j] = (j < k) ? __ldg(slot_to_row + static_cast<int64_t>(t) * k + j) : 0;
   }
   for (int c8 = threadIdx.x; c8 < H / 8; c8 += blockDim.x) {
+    uint4 u[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      u[j] = (j < k) ? __ldg(reinterpret_cast<const uint4*>(down_out + rows[j] * H) + c8) : make_uint4(0u, 0u, 0u, 0u);
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (j >= k) break;
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(down_out + rows[j] * H) + c8);
-      const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+      const uint32_t q[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(w[j], __uint_as_float(q[i] << 16)));
@@ -140,7 +166,8 @@ __global__ void __launch_bounds__(256) combine_kernel(int H, int k, const __nv_b
 cudaError_t launch_combine(int T, int H, int k, const void* down_out, const float* topk_w,
                            const int32_t* slot_to_row, void* y, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  return launch_pdl(combine_kernel, dim3(T), dim3(256), 0, stream, H, k,
+  const int threads = std::min(1024, (H / 8 + 31) / 32 * 32);
+  return launch_pdl(combine_kernel, dim3(T), dim3(static_cast<unsigned>(threads)), 0, stream, H, k,
                     static_cast<const __nv_bfloat16*>(down_out), topk_w, slot_to_row, static_cast<__nv_bfloat16*>(y));
 }
 

@@ -156,8 +156,9 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
 }
 
 // One CTA of 1024 threads.  Warp w scans the bitmaps of experts w, w + 32, ...:
-// prefix[e][i] = sum of popc over words 0..i-1 of expert e; then the padded
-// offsets over experts.
+// prefix[e][i] = sum of popc over words 0..i-1 of expert e, 32 words (one per
+// lane, coalesced) per warp scan, with the loads of up to 8 such chunks
+// issued before their scans; then the padded offsets over experts.
 __global__ void __launch_bounds__(1024) route_scan_kernel(int E, int W, const uint32_t* __restrict__ bitmap,
                                                            int32_t* __restrict__ prefix,
                                                            int32_t* __restrict__ expert_counts,
@@ -171,17 +172,27 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int E, int W, const ui
     const uint32_t* bm = bitmap + static_cast<int64_t>(e) * W;
     int32_t* pf = prefix + static_cast<int64_t>(e) * W;
     int32_t base = 0;
-    for (int w0 = 0; w0 < W; w0 += 32) {
-      const int i = w0 + lane;
-      const int32_t c = (i < W) ? __popc(bm[i]) : 0;
-      int32_t incl = c;
+    for (int w0 = 0; w0 < W; w0 += 256) {
+      const int chunks = min(8, (W - w0 + 31) / 32);  // the same for the whole warp
+      int32_t c[8];
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-        if (lane >= off) incl += o;
+      for (int j = 0; j < 8; ++j) {
+        const int i = w0 + 32 * j + lane;
+        c[j] = (j < chunks && i < W) ? __popc(bm[i]) : 0;
       }
-      if (i < W) pf[i] = base + incl - c;
-      base += __shfl_sync(0xFFFFFFFFu, incl, 31);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j >= chunks) break;
+        int32_t incl = c[j];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+          if (lane >= off) incl += o;
+        }
+        const int i = w0 + 32 * j + lane;
+        if (i < W) pf[i] = base + incl - c[j];
+        base += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      }
     }
     if (lane == 0) s_count[e] = base;
   }
