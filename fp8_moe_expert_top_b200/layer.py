@@ -86,15 +86,17 @@ class ExpertLayer:
         B.moe_forward_down(self.cfg, T, self.packed, self.h_codes, self.h_sf, self.inter_scale,
                            self.expert_offsets, self.expert_counts, self.down_out, self.status)
 
-    def combine(self, T):
-        B.moe_unpermute_combine(self.cfg, T, self.down_out, self.topk_w, self.slot_to_row, self.y)
+    def combine(self, T, y=None):
+        B.moe_unpermute_combine(self.cfg, T, self.down_out, self.topk_w, self.slot_to_row,
+                                self.y if y is None else y)
 
     # ------------------------------------------------------------- graphs
-    def capture(self, T, events=None):
+    def capture(self, T, events=None, x_in=None, logits_in=None, y_out=None):
         """Capture the whole layer for T tokens as a CUDA graph.
 
-        The graph reads its inputs from self.x_in [T_max, H] (bf16) and
-        self.logits_in [T_max, E] (float32) and writes self.y.  `events`, if
+        The graph reads its inputs from x_in [>= T, H] (bf16) and logits_in
+        [>= T, E] (float32) and writes y_out [>= T, H] (bf16); by default
+        self.x_in, self.logits_in (allocated here) and self.y.  `events`, if
         given, is a list of six timing events created with external=True; they
         are recorded before the layer and after each of its five steps.  Run
         one eager forward first so that every kernel is set up.
@@ -102,11 +104,14 @@ class ExpertLayer:
         if getattr(self, "x_in", None) is None:
             self.x_in = torch.zeros(self.T_max, self.H, dtype=torch.bfloat16, device=self.device)
             self.logits_in = torch.zeros(self.T_max, self.E, dtype=torch.float32, device=self.device)
+        x_in = self.x_in if x_in is None else x_in
+        logits_in = self.logits_in if logits_in is None else logits_in
+        y_out = self.y if y_out is None else y_out
         g = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(device=self.device)
         side.wait_stream(torch.cuda.current_stream(self.device))
-        steps = (lambda: self.route(self.logits_in, T), lambda: self.permute(self.x_in, T),
-                 lambda: self.gateup(T), lambda: self.down(T), lambda: self.combine(T))
+        steps = (lambda: self.route(logits_in, T), lambda: self.permute(x_in, T),
+                 lambda: self.gateup(T), lambda: self.down(T), lambda: self.combine(T, y_out))
         with torch.cuda.graph(g, stream=side):
             if events is not None:
                 events[0].record()
@@ -139,3 +144,59 @@ class ExpertLayer:
         self.down(T)
         self.combine(T)
         return self.y[:T]
+
+
+class HostPipeline:
+    """The layer over a sequence of host batches of T tokens each, with the
+    host <-> device copies of neighbouring batches overlapping its kernels.
+
+    Two CUDA graphs of the layer alternate, each with its own device input and
+    output buffers.  Batch i's x and logits go up on an upload stream while
+    batch i - 1 computes, and each batch's y comes down on a download stream
+    while the next one computes.  Events order every reuse of a buffer: a
+    slot's inputs are overwritten only after the graph that read them has
+    finished, and its output only after it has been copied out.  The graphs
+    share the layer's intermediate buffers, so they run one after the other on
+    the current stream.
+    """
+
+    def __init__(self, layer, T):
+        self.layer, self.T = layer, T
+        dev = layer.device
+        self.x = [torch.zeros(T, layer.H, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.logits = [torch.zeros(T, layer.E, dtype=torch.float32, device=dev) for _ in range(2)]
+        self.y = [torch.zeros(T, layer.H, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.graphs = [layer.capture(T, x_in=self.x[s], logits_in=self.logits[s], y_out=self.y[s])
+                       for s in range(2)]
+        self.up = torch.cuda.Stream(device=dev)
+        self.down = torch.cuda.Stream(device=dev)
+        self.uploaded = [torch.cuda.Event() for _ in range(2)]
+        self.computed = [torch.cuda.Event() for _ in range(2)]
+        self.downloaded = [torch.cuda.Event() for _ in range(2)]
+
+    def run(self, xs, logits, ys):
+        """y_i = layer(x_i, logits_i) for pinned host tensors xs[i] [T, H] bf16,
+        logits[i] [T, E] float32, into pinned host ys[i] [T, H] bf16.  Returns
+        once all work is queued; the current stream waits for the last copy."""
+        comp = torch.cuda.current_stream(self.layer.device)
+        self.up.wait_stream(comp)
+        self.down.wait_stream(comp)
+        for i in range(len(xs)):
+            s = i % 2
+            with torch.cuda.stream(self.up):
+                if i >= 2:
+                    self.up.wait_event(self.computed[s])  # slot s's inputs were read by batch i - 2
+                self.x[s].copy_(xs[i], non_blocking=True)
+                self.logits[s].copy_(logits[i], non_blocking=True)
+                self.uploaded[s].record(self.up)
+            comp.wait_event(self.uploaded[s])
+            if i >= 2:
+                comp.wait_event(self.downloaded[s])  # slot s's output of batch i - 2 is out
+            self.graphs[s].replay()
+            self.computed[s].record(comp)
+            with torch.cuda.stream(self.down):
+                self.down.wait_event(self.computed[s])
+                ys[i].copy_(self.y[s], non_blocking=True)
+                self.downloaded[s].record(self.down)
+        comp.wait_stream(self.up)
+        comp.wait_stream(self.down)

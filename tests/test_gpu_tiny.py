@@ -175,3 +175,27 @@ def test_cuda_graph_replay_matches_eager(cuda_device, wl):
         torch.cuda.synchronize()
         assert torch.equal(y_graph.view(torch.int16), y_eager.view(torch.int16))
     assert torch.equal(layer.h_codes, h_eager)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl", [TINY, TINY_MX], ids=lambda w: w.name)
+def test_host_pipeline_matches_eager(cuda_device, wl):
+    """Five host batches through HostPipeline (uploads and downloads of
+    neighbouring batches overlapping the layer) give, batch by batch, the
+    eager results bit for bit."""
+    from fp8_moe_expert_top_b200.layer import HostPipeline
+
+    layer = get_layer(wl, cuda_device)
+    n = 5
+    xs = [inputs.make_x(wl, seed=40 + 2 * i).pin_memory() for i in range(n)]
+    lgs = [inputs.make_logits(wl, seed=41 + 2 * i).pin_memory() for i in range(n)]
+    ref = []
+    for i in range(n):
+        ref.append(layer.forward(xs[i].to(cuda_device), lgs[i].to(cuda_device)).cpu())
+    pipe = HostPipeline(layer, wl.T)
+    ys = [torch.full((wl.T, wl.d_model), float("nan"), dtype=torch.bfloat16).pin_memory() for _ in range(n)]
+    pipe.run(xs, lgs, ys)
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0
+    for i in range(n):
+        assert torch.equal(ys[i].view(torch.int16), ref[i].view(torch.int16)), i
