@@ -41,6 +41,11 @@ UNIT = "tokens/s"
 
 # --------------------------------------------------------------------------- helpers
 
+def pct(values, q):
+    """q-th percentile (linear interpolation) of a non-empty list."""
+    return float(np.percentile(np.asarray(values, dtype=np.float64), q))
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -345,6 +350,9 @@ def run_ours(args, wl, ws, rank, local):
     roof["traffic"] = measured_traffic(wl.name, dom)
     # whole-layer roofline (slower of bytes at HBM peak and FLOPs at tensor peak)
     layer_t = max(bytes_["layer"] / (peaks["hbm_gbs"] * 1e9), slots * flops_slot / (tensor_peak * 1e12))
+    # nominal B200 peaks for context: 8 TB/s HBM, 9 / 4.5 PFLOP/s dense NVFP4 / FP8
+    nominal_tensor = 9000.0 if wl.fmt == inputs.NVFP4 else 4500.0
+    layer_t_nominal = max(bytes_["layer"] / 8.0e12, slots * flops_slot / (nominal_tensor * 1e12))
     value = ws * T * args.steps / (total_ms * 1e-3)
     out = {
         "metric": METRIC,
@@ -365,6 +373,8 @@ def run_ours(args, wl, ws, rank, local):
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
         "roofline": roof,
         "layer_roofline_frac": layer_t / (total_ms * 1e-3 / args.steps),
+        "layer_roofline_frac_nominal": layer_t_nominal / (total_ms * 1e-3 / args.steps),
+        "step_ms_pct": {"p10": pct(step_ms, 10), "p50": pct(step_ms, 50), "p90": pct(step_ms, 90)},
         "phase_ms": {p: round(mean_ms[p], 4) for p in PHASES},
         "eager_ms_per_step": eager_ms,
         "timing": "CUDA graph of the five calls replayed per step; external CUDA events between the steps",

@@ -63,6 +63,8 @@ WORKLOADS = {
         Workload("decode_mxfp8", 256, 4096, 2560, 384, 8, MXFP8),
         Workload("prefill_nvfp4", 8192, 4096, 2560, 384, 8, NVFP4),
         Workload("prefill_nvfp4_skewed", 16384, 4096, 2560, 384, 8, NVFP4, skewed=True),
+        # the MXFP8 layers (40-47) at the prefill batch of the NVFP4 layer
+        Workload("prefill_mxfp8", 8192, 4096, 2560, 384, 8, MXFP8),
     ]
 }
 

@@ -1,9 +1,9 @@
-"""GPU parity at the full sizes of the four named layers (GPU).
+"""GPU parity at the full sizes of the named layers (GPU).
 
 Layers (d_model 4096, expert ffn 2560, 384 experts, top-8): decode NVFP4
-(T = 64), decode MXFP8 (T = 256), prefill NVFP4 (T = 8192) and prefill NVFP4
-with Zipf-skewed routing (T = 16384), run with the same ExpertLayer the
-benchmark times.  Checked against the oracle:
+(T = 64), decode MXFP8 (T = 256), prefill NVFP4 (T = 8192), prefill NVFP4
+with Zipf-skewed routing (T = 16384) and prefill MXFP8 (T = 8192), run with
+the same ExpertLayer the benchmark times.  Checked against the oracle:
   * routing of every token: top-k ids, softmax weights, counts, offsets and
     the slot permutation, bit-exact;
   * on sampled tokens (the oracle is too slow for all of them): the weight
@@ -29,7 +29,7 @@ from oracle import route as ort
 from gpu_common import assert_expert_equal, build_layer, gpu_expert
 from helpers import ACT_TR, kb_padded, rel_fro, sfvec, sf_index, tile_offsets, unpack_codes
 
-FULL = ["decode_nvfp4", "decode_mxfp8", "prefill_nvfp4", "prefill_nvfp4_skewed"]
+FULL = ["decode_nvfp4", "decode_mxfp8", "prefill_nvfp4", "prefill_nvfp4_skewed", "prefill_mxfp8"]
 
 
 def _quantize_job(job):
