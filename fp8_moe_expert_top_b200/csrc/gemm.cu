@@ -38,6 +38,7 @@
 // Every mbarrier wait is bounded; a wait that runs out raises a CTA-wide
 // abort flag, every role stops issuing, TMEM is freed and a status bit is
 // set.
+#include <atomic>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -324,18 +325,20 @@ static cudaError_t launch_one(const GemmArgs& a, cudaStream_t stream) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  static int configured[64] = {0};
-  if (dev >= 64 || !configured[dev]) {
+  // per device: the kernel's shared-memory limit is raised once and the SM
+  // count read once (host threads may launch concurrently; both are idempotent)
+  static std::atomic<int> sm_count[64];
+  int sms = (dev < 64) ? sm_count[dev].load(std::memory_order_relaxed) : 0;
+  if (sms == 0) {
     // the largest size any supported E needs (E <= 1024)
     const size_t smem_max = 1024 + kStages * Tr::kStageBytes + (3 * kStages + 2) * 8 + 16 + 1025 * 4;
     err = cudaFuncSetAttribute(moe_gemm_kernel<FMT, GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem_max));
     if (err != cudaSuccess) return err;
-    if (dev < 64) configured[dev] = 1;
+    err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 64) sm_count[dev].store(sms, std::memory_order_relaxed);
   }
-  int sms = 0;
-  err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (err != cudaSuccess) return err;
   return launch_pdl(moe_gemm_kernel<FMT, GATEUP>, dim3(sms), dim3(kThreadsOne), smem, stream, a);
 }
 
