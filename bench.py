@@ -416,6 +416,75 @@ def gemm_source_sha():
     return h.hexdigest()[:16]
 
 
+# --------------------------------------------------------------------------- expert stack
+
+def run_depth(args, local, n_nv, n_mx):
+    """The expert layers of the whole model depth applied to one batch: n_nv
+    NVFP4 passes then n_mx MXFP8 passes, each fed the previous pass's output
+    and its own seeded logits (the router is outside the layer), captured as
+    one CUDA graph.  Two weight sets (one NVFP4 and one MXFP8 layer, each larger
+    than L2) serve all passes, so every pass streams its weights from HBM."""
+    import dataclasses
+    from fp8_moe_expert_top_b200.layer import capture_stack
+    T = args.tokens if args.tokens is not None else 64
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl_n = dataclasses.replace(inputs.WORKLOADS["decode_nvfp4"], T=T)
+    wl_m = dataclasses.replace(inputs.WORKLOADS["decode_mxfp8"], T=T)
+    ln, lm = build_layer(wl_n, device, T), build_layer(wl_m, device, T)
+    passes = []
+    for p in range(n_nv + n_mx):
+        wl = wl_n if p < n_nv else wl_m
+        passes.append((ln if p < n_nv else lm, wl,
+                       inputs.make_logits(wl, seed=inputs.BASE_SEED + 100 + p).to(device)))
+    x = inputs.make_x(wl_n).to(device)
+    # eager pass: sets up every kernel and gives each pass's touched experts
+    layer_bytes, cur = 0.0, x
+    for layer, wl, lg in passes:
+        cur = layer.forward(cur, lg).clone()
+        n_touched = int((layer.expert_counts.cpu() > 0).sum())
+        layer_bytes += phase_bytes(wl, n_touched, T * wl.top_k)["layer"]
+    y_bufs = [torch.zeros(T, wl_n.d_model, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    graph, _ = capture_stack([(l, lg) for l, _, lg in passes], x, y_bufs, T)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(device)
+    clocks = ClockSampler(local)
+    clocks.start()
+    step_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
+    clk = clocks.stop()
+    for layer in (ln, lm):
+        if int(layer.status.item()) != 0:
+            raise RuntimeError(f"device status word {int(layer.status.item()):#x}")
+    peaks, _ = load_peaks()
+    ms = statistics.mean(step_ms)
+    return {
+        "metric": f"expert-layer stack ({n_nv} NVFP4 + {n_mx} MXFP8 layers) tokens/s on 1 B200",
+        "value": T / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4+mxfp8",
+        "data": "synthetic (seeded N(0,1) x and per-layer logits, N(0,1/fan_in) weights, random init)",
+        "config": {"workload": f"expert_stack_{n_nv}x_nvfp4_{n_mx}x_mxfp8_t{T}", "T": T, "d_model": wl_n.d_model,
+                   "d_ffn": wl_n.d_ffn, "num_experts": wl_n.num_experts, "top_k": wl_n.top_k,
+                   "l2": "flushed between timed steps (512 MiB write)", "parallelism": "single GPU"},
+        "stack_roofline_frac": (layer_bytes / (peaks["hbm_gbs"] * 1e9)) / (ms * 1e-3),
+        "ms_per_layer": ms / (n_nv + n_mx),
+        "step_ms_pct": {"p10": pct(step_ms, 10), "p50": pct(step_ms, 50), "p90": pct(step_ms, 90)},
+        "gpu_launches": 7 * (n_nv + n_mx) * args.steps,
+        "clocks": clk,
+    }
+
+
 # --------------------------------------------------------------------------- CPU oracle
 
 def _oracle_quantize(args_):
@@ -515,6 +584,9 @@ def main(argv=None):
                     help="profiling only: override the number of experts (smaller device footprint for ncu)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="profiling only: override the number of tokens (with --experts, keeps rows per expert)")
+    ap.add_argument("--depth", default=None, metavar="N_NVFP4,N_MXFP8",
+                    help="time the expert layers of a whole model depth on one batch (e.g. 40,8), "
+                         "--tokens tokens (default 64)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -528,6 +600,12 @@ def main(argv=None):
     ws, rank, local = dist_env()
     if ws != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {ws}", file=sys.stderr)
+    if args.depth is not None:
+        if ws > 1 or args.impl != "ours":
+            ap.error("--depth runs the library on one GPU")
+        n_nv, n_mx = (int(v) for v in args.depth.split(","))
+        print(json.dumps(run_depth(args, local, n_nv, n_mx)))
+        return 0
     if args.impl == "reference":
         out = run_reference(args, wl, ws, rank)
         if out is not None:

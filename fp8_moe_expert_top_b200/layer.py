@@ -200,3 +200,31 @@ class HostPipeline:
                 self.downloaded[s].record(self.down)
         comp.wait_stream(self.up)
         comp.wait_stream(self.down)
+
+
+def capture_stack(passes, x_in, y_bufs, T):
+    """One CUDA graph of expert layers applied one after another to the same T
+    tokens, as in a stack of decoder layers: passes = [(layer, logits), ...],
+    logits [>= T, E] float32 on the device.  Pass 0 reads x_in [>= T, H]
+    (bf16); pass p > 0 reads the output of pass p - 1; pass p writes
+    y_bufs[p % 2].  A layer object may appear in several passes (its
+    intermediate buffers are reused, the passes run in order).  Run each
+    distinct layer eagerly once before capturing.  Returns (graph, y) with y
+    the buffer that holds the last pass's output.
+    """
+    dev = x_in.device
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.graph(g, stream=side):
+        x = x_in
+        for p, (layer, logits) in enumerate(passes):
+            y = y_bufs[p % 2]
+            layer.route(logits, T)
+            layer.permute(x, T)
+            layer.gateup(T)
+            layer.down(T)
+            layer.combine(T, y)
+            x = y
+    torch.cuda.current_stream(dev).wait_stream(side)
+    return g, y_bufs[(len(passes) - 1) % 2]

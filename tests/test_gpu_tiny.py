@@ -199,3 +199,28 @@ def test_host_pipeline_matches_eager(cuda_device, wl):
     assert int(layer.status.item()) == 0
     for i in range(n):
         assert torch.equal(ys[i].view(torch.int16), ref[i].view(torch.int16)), i
+
+
+@pytest.mark.gpu
+def test_layer_stack_graph_matches_eager(cuda_device):
+    """Three NVFP4 and two MXFP8 passes chained in one CUDA graph (each pass
+    fed the previous one's output, fresh logits per pass) give the eager
+    sequence's output bit for bit."""
+    from fp8_moe_expert_top_b200.layer import capture_stack
+
+    ln, lm = get_layer(TINY, cuda_device), get_layer(TINY_MX, cuda_device)
+    T = TINY.T
+    passes = [(ln if p < 3 else lm, inputs.make_logits(TINY, seed=60 + p).to(cuda_device)) for p in range(5)]
+    x = inputs.make_x(TINY, seed=59).to(cuda_device)
+    cur = x
+    for layer, lg in passes:
+        cur = layer.forward(cur, lg).clone()
+    ref = cur.cpu()
+    y_bufs = [torch.zeros(T, TINY.d_model, dtype=torch.bfloat16, device=cuda_device) for _ in range(2)]
+    g, y = capture_stack(passes, x, y_bufs, T)
+    for _ in range(2):
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y.cpu().view(torch.int16), ref.view(torch.int16))
+    assert int(ln.status.item()) == 0 and int(lm.status.item()) == 0
