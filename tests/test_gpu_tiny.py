@@ -224,3 +224,48 @@ def test_layer_stack_graph_matches_eager(cuda_device):
         torch.cuda.synchronize()
         assert torch.equal(y.cpu().view(torch.int16), ref.view(torch.int16))
     assert int(ln.status.item()) == 0 and int(lm.status.item()) == 0
+
+
+def _crafted_weights(wl, seed):
+    """float32 weights of every expert, with crafted blocks in experts 0-3."""
+    g = torch.Generator().manual_seed(seed)
+    E, H, I = wl.num_experts, wl.d_model, wl.d_ffn
+    wg = torch.randn(E, I, H, generator=g) / H ** 0.5
+    wu = torch.randn(E, I, H, generator=g) / H ** 0.5
+    wd = torch.randn(E, H, I, generator=g) / I ** 0.5
+    wg[0].zero_()                                     # an all-zero matrix: tensor scale 1, zero codes
+    wu[1].view(I, H // 16, 16)[:, ::2] = 0.0          # every other 16-element block all zero
+    amax = wd[2].abs().max()                          # blocks whose maxima lie in [0.7, 1] of the
+    mag = amax * (0.7 + 0.3 * torch.rand(8, I, generator=g))  # tensor max: the 4-candidate scale
+    wd[2, :8, :] = mag * torch.sign(torch.randn(8, I, generator=g))  # saturates at 448
+    wg[3, :, :16] = 0.25                              # a block of equal elements (tied errors)
+    return wg.contiguous(), wu.contiguous(), wd.contiguous()
+
+
+def _crafted_x(wl, seed):
+    x = inputs.make_x(wl, seed=seed).float()
+    x[0] = 0.0                                        # an all-zero token
+    x[1, :16] = 0.0                                   # a zero block
+    x[2] = 20.0 * torch.sign(x[2])                    # beyond the static scale's range: saturating codes
+    x[3, 32:64] = x[3, 32:64] * 1e-30                 # values that round to zero codes
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl", [TINY, TINY_MX], ids=lambda w: w.name)
+def test_crafted_blocks(cuda_device, wl):
+    """All-zero matrices and blocks, saturating 4-candidate scales, tied block
+    errors, saturating and underflowing activations: weight codes, routing and
+    activation codes bit-exact, the rest within the bars."""
+    from fp8_moe_expert_top_b200.layer import ExpertLayer
+
+    wg, wu, wd = _crafted_weights(wl, 70)
+    layer = ExpertLayer(wl.num_experts, wl.top_k, wl.d_model, wl.d_ffn, wl.fmt, wl.T, cuda_device,
+                        s_x=inputs.S_X, s_h=inputs.S_H, debug=True)
+    layer.quantize_experts(0, wg.to(cuda_device), wu.to(cuda_device), wd.to(cuda_device))
+    torch.cuda.synchronize()
+    experts = {e: omoe.quantize_expert(wg[e].numpy(), wu[e].numpy(), wd[e].numpy(), wl.fmt)
+               for e in range(wl.num_experts)}
+    for e in range(4):
+        assert_expert_equal(gpu_expert(layer, wl, e), experts[e], e)
+    run_and_compare(layer, wl, _crafted_x(wl, 71), inputs.make_logits(wl, seed=72), experts)
