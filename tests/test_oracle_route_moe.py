@@ -65,6 +65,20 @@ def test_softmax_weights():
     assert np.all(np.diff(w, axis=1) <= 0)             # rank order
 
 
+def test_softmax_weights_of_large_logits():
+    """Softmax is defined for any finite logits: rows offset far from zero
+    (where exp of a raw logit overflows float32) still give the float64 weights."""
+    rng = np.random.default_rng(12)
+    lg = (rng.standard_normal((40, 16)) * 3 + rng.choice([-300.0, 150.0, 1000.0], (40, 1))).astype(np.float32)
+    ids = rt.topk_select(lg, 8)
+    w = rt.topk_softmax(lg, ids)
+    sel = np.take_along_axis(lg.astype(np.float64), ids.astype(np.int64), axis=1)
+    ref = np.exp(sel - sel.max(1, keepdims=True))
+    ref /= ref.sum(1, keepdims=True)
+    assert np.all(np.isfinite(w))
+    np.testing.assert_allclose(w, ref, rtol=4e-7, atol=1e-30)
+
+
 # ---------------------------------------------------------------- slot sort
 
 def test_sort_slots_matches_library_sort():
@@ -175,6 +189,23 @@ def test_layer_equals_per_token_loop(fmt):
     np.testing.assert_allclose(res["y"], ref["y"], rtol=2 ** -7, atol=1e-6)
     diff = np.mean(res["y"] != ref["y"])
     assert diff < 0.02       # only float64 summation order differs, then bf16 rounding
+
+
+def test_weight_tensor_scale_maps_largest_magnitude_to_top_of_range():
+    """NVFP4 weights: the element of largest magnitude lands on the top of the
+    two-level range (code +-6 at block scale 448) and is reproduced, whatever
+    its sign; every other element stays inside the range."""
+    rng = np.random.default_rng(13)
+    for sign in (-1.0, 1.0):
+        w = (rng.standard_normal((32, 64)) * 0.02).astype(np.float32)
+        w[5, 17] = sign * 0.5                           # the extreme element, either sign
+        q = moe.quantize_expert(w, w, w.T.copy(), moe.NVFP4)
+        codes, sf, s_g = q["gate"]
+        deq = fm.nvfp4_dequantize_rows(codes, sf, s_g)
+        assert sf[5, 17 // 16] == 0x7E
+        assert codes[5, 17] == (15 if sign < 0 else 7)
+        assert abs(deq[5, 17] - w[5, 17]) <= 2.0 ** -22 * 0.5
+        assert np.max(np.abs(deq)) <= 0.5 * (1 + 2.0 ** -22)
 
 
 def test_swiglu_closed_form():
