@@ -110,7 +110,7 @@ def test_layer_seeded_inputs(cuda_device, wl):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("wl", [TINY, TINY_MX], ids=lambda w: w.name)
-@pytest.mark.parametrize("case", ["one_token", "hot_experts", "ties", "empty_experts", "ragged"])
+@pytest.mark.parametrize("case", ["one_token", "hot_experts", "ties", "empty_experts", "ragged", "large_logits"])
 def test_layer_edge_cases(cuda_device, wl, case):
     layer = get_layer(wl, cuda_device)
     E = wl.num_experts
@@ -126,6 +126,10 @@ def test_layer_edge_cases(cuda_device, wl, case):
     elif case == "empty_experts":        # experts 0, 1 and 6 never chosen
         x, lg = inputs.make_x(wl, seed=17), inputs.make_logits(wl, seed=18)
         lg[:, [0, 1, 6]] -= 100.0
+    elif case == "large_logits":         # rows offset far from zero: exp of a raw logit would overflow
+        x, lg = inputs.make_x(wl, seed=21), inputs.make_logits(wl, seed=22)
+        offs = torch.tensor([-300.0, 150.0, 1000.0])[torch.arange(wl.T) % 3]
+        lg = (lg * 3.0 + offs[:, None]).to(torch.float32)
     else:                                # T not a multiple of anything
         x, lg = inputs.make_x(wl, T=37, seed=19), inputs.make_logits(wl, T=37, seed=20)
     run_and_compare(layer, wl, x, lg, oracle_experts(wl))
