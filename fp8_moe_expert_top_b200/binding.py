@@ -92,15 +92,26 @@ def make_config(num_experts, top_k, d_model, d_ffn, fmt):
     return moe_config(int(num_experts), int(top_k), int(d_model), int(d_ffn), int(fmt))
 
 
-def _p(t):
-    if t is None:
-        return None
-    return ctypes.c_void_p(t.data_ptr())
+def _marshal(name, stream, *tensors):
+    """Device pointers of `tensors` (None stays NULL) and the stream handle.
 
-
-def _stream(stream=None):
+    Every tensor must be a contiguous CUDA tensor on the stream's device (the
+    current stream of the current device when `stream` is None): the library
+    takes raw device pointers, so a host tensor, a strided view or another
+    GPU's memory is refused here, before anything is enqueued.
+    """
+    for i, t in enumerate(tensors):
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name}: argument {i} is on {t.device}, a CUDA tensor is required")
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: argument {i} is not contiguous")
     s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+    for i, t in enumerate(tensors):
+        if t is not None and t.device != s.device:
+            raise ValueError(f"{name}: argument {i} is on {t.device}, the stream on {s.device}")
+    return [None if t is None else ctypes.c_void_p(t.data_ptr()) for t in tensors], ctypes.c_void_p(s.cuda_stream)
 
 
 def _check(name, status):
@@ -143,61 +154,59 @@ def moe_route_workspace_bytes(cfg, T):
 # ----------------------------------------------------------------- calls
 
 def moe_quantize_weights(cfg, expert_begin, expert_count, w_gate, w_up, w_down, packed, stream=None):
+    (wg, wu, wd, pk), st = _marshal("moe_quantize_weights", stream, w_gate, w_up, w_down, packed)
     _check("moe_quantize_weights", lib().moe_quantize_weights(
-        ctypes.byref(cfg), int(expert_begin), int(expert_count), _p(w_gate), _p(w_up), _p(w_down), _p(packed),
-        _stream(stream)))
+        ctypes.byref(cfg), int(expert_begin), int(expert_count), wg, wu, wd, pk, st))
 
 
 def moe_route_topk(cfg, T, logits, topk_ids, topk_w, expert_counts, expert_offsets, sorted_slots, slot_to_row,
                    workspace, stream=None):
+    p, st = _marshal("moe_route_topk", stream, logits, topk_ids, topk_w, expert_counts, expert_offsets,
+                     sorted_slots, slot_to_row, workspace)
     _check("moe_route_topk", lib().moe_route_topk(
-        ctypes.byref(cfg), int(T), _p(logits), _p(topk_ids), _p(topk_w), _p(expert_counts), _p(expert_offsets),
-        _p(sorted_slots), _p(slot_to_row), _p(workspace), int(workspace.numel() * workspace.element_size()),
-        _stream(stream)))
+        ctypes.byref(cfg), int(T), *p, int(workspace.numel() * workspace.element_size()), st))
 
 
 def moe_route_topk_noalloc(cfg, T, logits, topk_ids, topk_w, expert_counts, expert_offsets, sorted_slots,
                            slot_to_row, stream=None):
     """moe_route_topk without a workspace, for callers that cannot allocate
     device memory (the library's fixed 4 MiB scratch array is used instead)."""
-    _check("moe_route_topk_noalloc", lib().moe_route_topk_noalloc(
-        ctypes.byref(cfg), int(T), _p(logits), _p(topk_ids), _p(topk_w), _p(expert_counts), _p(expert_offsets),
-        _p(sorted_slots), _p(slot_to_row), _stream(stream)))
+    p, st = _marshal("moe_route_topk_noalloc", stream, logits, topk_ids, topk_w, expert_counts, expert_offsets,
+                     sorted_slots, slot_to_row)
+    _check("moe_route_topk_noalloc", lib().moe_route_topk_noalloc(ctypes.byref(cfg), int(T), *p, st))
 
 
 def moe_permute(cfg, T, x, act_scale, slot_to_row, a_codes, a_sf, stream=None):
-    _check("moe_permute", lib().moe_permute(
-        ctypes.byref(cfg), int(T), _p(x), _p(act_scale), _p(slot_to_row), _p(a_codes), _p(a_sf), _stream(stream)))
+    p, st = _marshal("moe_permute", stream, x, act_scale, slot_to_row, a_codes, a_sf)
+    _check("moe_permute", lib().moe_permute(ctypes.byref(cfg), int(T), *p, st))
 
 
 def moe_forward(cfg, T, packed, a_codes, a_sf, act_scale, inter_scale, expert_offsets, expert_counts, h_codes, h_sf,
                 down_out, gateup_debug=None, status_word=None, stream=None):
-    _check("moe_forward", lib().moe_forward(
-        ctypes.byref(cfg), int(T), _p(packed), _p(a_codes), _p(a_sf), _p(act_scale), _p(inter_scale),
-        _p(expert_offsets), _p(expert_counts), _p(h_codes), _p(h_sf), _p(down_out), _p(gateup_debug),
-        _p(status_word), _stream(stream)))
+    p, st = _marshal("moe_forward", stream, packed, a_codes, a_sf, act_scale, inter_scale, expert_offsets,
+                     expert_counts, h_codes, h_sf, down_out, gateup_debug, status_word)
+    _check("moe_forward", lib().moe_forward(ctypes.byref(cfg), int(T), *p, st))
 
 
 def moe_forward_gateup(cfg, T, packed, a_codes, a_sf, act_scale, inter_scale, expert_offsets, expert_counts,
                        h_codes, h_sf, gateup_debug=None, status_word=None, stream=None):
-    _check("moe_forward_gateup", lib().moe_forward_gateup(
-        ctypes.byref(cfg), int(T), _p(packed), _p(a_codes), _p(a_sf), _p(act_scale), _p(inter_scale),
-        _p(expert_offsets), _p(expert_counts), _p(h_codes), _p(h_sf), _p(gateup_debug), _p(status_word),
-        _stream(stream)))
+    p, st = _marshal("moe_forward_gateup", stream, packed, a_codes, a_sf, act_scale, inter_scale, expert_offsets,
+                     expert_counts, h_codes, h_sf, gateup_debug, status_word)
+    _check("moe_forward_gateup", lib().moe_forward_gateup(ctypes.byref(cfg), int(T), *p, st))
 
 
 def moe_forward_down(cfg, T, packed, h_codes, h_sf, inter_scale, expert_offsets, expert_counts, down_out,
                      status_word=None, stream=None):
-    _check("moe_forward_down", lib().moe_forward_down(
-        ctypes.byref(cfg), int(T), _p(packed), _p(h_codes), _p(h_sf), _p(inter_scale), _p(expert_offsets),
-        _p(expert_counts), _p(down_out), _p(status_word), _stream(stream)))
+    p, st = _marshal("moe_forward_down", stream, packed, h_codes, h_sf, inter_scale, expert_offsets, expert_counts,
+                     down_out, status_word)
+    _check("moe_forward_down", lib().moe_forward_down(ctypes.byref(cfg), int(T), *p, st))
 
 
 def moe_unpermute_combine(cfg, T, down_out, topk_w, slot_to_row, y, stream=None):
-    _check("moe_unpermute_combine", lib().moe_unpermute_combine(
-        ctypes.byref(cfg), int(T), _p(down_out), _p(topk_w), _p(slot_to_row), _p(y), _stream(stream)))
+    p, st = _marshal("moe_unpermute_combine", stream, down_out, topk_w, slot_to_row, y)
+    _check("moe_unpermute_combine", lib().moe_unpermute_combine(ctypes.byref(cfg), int(T), *p, st))
 
 
 def moe_selftest_bounded_wait(status_word, limit_ns, stream=None):
-    _check("moe_selftest_bounded_wait", lib().moe_selftest_bounded_wait(_p(status_word), int(limit_ns),
-                                                                        _stream(stream)))
+    (sw,), st = _marshal("moe_selftest_bounded_wait", stream, status_word)
+    _check("moe_selftest_bounded_wait", lib().moe_selftest_bounded_wait(sw, int(limit_ns), st))

@@ -24,6 +24,12 @@ class ExpertLayer:
         self.fmt = self.cfg.fmt
         self.T_max = int(T_max)
         self.device = torch.device(device)
+        if self.device.type != "cuda":
+            raise ValueError(f"ExpertLayer runs on a CUDA device, not {self.device}")
+        if self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
+        if self.T_max < 0:
+            raise ValueError(f"T_max must be >= 0, got {self.T_max}")
         dev = self.device
         self.layout = B.moe_get_weights_layout(self.cfg)
         self.packed = torch.empty(self.layout.total_bytes, dtype=torch.uint8, device=dev)
@@ -60,11 +66,30 @@ class ExpertLayer:
     def quantize_experts(self, expert_begin, w_gate, w_up, w_down):
         """Quantize float32 weights of experts [begin, begin + n) into self.packed."""
         n = w_gate.shape[0]
-        for t in (w_gate, w_up, w_down):
-            assert t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+        shapes = ((n, self.I, self.H), (n, self.I, self.H), (n, self.H, self.I))
+        for name, t, shape in zip(("w_gate", "w_up", "w_down"), (w_gate, w_up, w_down), shapes):
+            if t.dtype != torch.float32 or tuple(t.shape) != shape:
+                raise ValueError(f"{name}: float32 {shape} expected, got {t.dtype} {tuple(t.shape)}")
         B.moe_quantize_weights(self.cfg, expert_begin, n, w_gate, w_up, w_down, self.packed)
 
     # ------------------------------------------------------------- steps
+    def _check_T(self, T):
+        if not 0 <= T <= self.T_max:
+            raise ValueError(f"T = {T} tokens, this layer's buffers hold 0..{self.T_max}")
+
+    def _check_io(self, T, x=None, logits=None, y=None):
+        """Shapes, dtypes and device of step inputs / outputs holding >= T rows."""
+        self._check_T(T)
+        args = [(name, t, cols, dtype) for name, t, cols, dtype in (
+            ("x", x, self.H, torch.bfloat16), ("logits", logits, self.E, torch.float32),
+            ("y", y, self.H, torch.bfloat16)) if t is not None]
+        for name, t, cols, dtype in args:
+            if t.dim() != 2 or t.shape[0] < T or t.shape[1] != cols or t.dtype != dtype:
+                raise ValueError(f"{name}: {dtype} [>= {T}, {cols}] expected, got {t.dtype} {tuple(t.shape)}")
+        for name, t, _, _ in args:
+            if t.device != self.device:
+                raise ValueError(f"{name} is on {t.device}, the layer on {self.device}")
+
     def route(self, logits, T):
         B.moe_route_topk(self.cfg, T, logits, self.topk_ids, self.topk_w, self.expert_counts,
                          self.expert_offsets, self.sorted_slots, self.slot_to_row, self.route_ws)
@@ -107,6 +132,7 @@ class ExpertLayer:
         x_in = self.x_in if x_in is None else x_in
         logits_in = self.logits_in if logits_in is None else logits_in
         y_out = self.y if y_out is None else y_out
+        self._check_io(T, x_in, logits_in, y_out)
         g = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(device=self.device)
         side.wait_stream(torch.cuda.current_stream(self.device))
@@ -120,24 +146,31 @@ class ExpertLayer:
                 if events is not None:
                     events[i + 1].record()
         torch.cuda.current_stream(self.device).wait_stream(side)
-        self._graph_T = T
+        g.moe_layer_io = (self, T, x_in, logits_in, y_out)
         return g
 
     def forward_graph(self, graph, x, logits):
-        """Copy x / logits into the graph's input buffers and replay it."""
-        T = self._graph_T
-        assert x.shape[0] == T and logits.shape[0] == T
-        self.x_in[:T].copy_(x, non_blocking=True)
-        self.logits_in[:T].copy_(logits, non_blocking=True)
+        """Copy x [T, H] / logits [T, E] into the input buffers `graph` was
+        captured with (by this layer's capture), replay it, and return its
+        output rows y[:T]."""
+        io = getattr(graph, "moe_layer_io", None)
+        if io is None or io[0] is not self:
+            raise ValueError("the graph was not captured by this layer's capture()")
+        _, T, x_in, logits_in, y_out = io
+        if x.shape[0] != T or logits.shape[0] != T:
+            raise ValueError(f"the graph was captured for T = {T}, got {x.shape[0]} / {logits.shape[0]} rows")
+        self._check_io(T, x, logits)
+        x_in[:T].copy_(x, non_blocking=True)
+        logits_in[:T].copy_(logits, non_blocking=True)
         graph.replay()
-        return self.y[:T]
+        return y_out[:T]
 
     def forward(self, x, logits):
         """y[:T] for bf16 x [T, H] and float32 logits [T, E] already on the device."""
         T = x.shape[0]
-        assert T <= self.T_max and logits.shape == (T, self.E)
-        assert x.dtype == torch.bfloat16 and logits.dtype == torch.float32
-        assert x.is_contiguous() and logits.is_contiguous()
+        self._check_io(T, x, logits)
+        if logits.shape[0] != T:
+            raise ValueError(f"x has {T} rows, logits {logits.shape[0]}")
         self.route(logits, T)
         self.permute(x, T)
         self.gateup(T)
@@ -212,6 +245,10 @@ def capture_stack(passes, x_in, y_bufs, T):
     distinct layer eagerly once before capturing.  Returns (graph, y) with y
     the buffer that holds the last pass's output.
     """
+    if not passes:
+        raise ValueError("capture_stack needs at least one pass")
+    for p, (layer, logits) in enumerate(passes):
+        layer._check_io(T, x_in if p == 0 else None, logits, y_bufs[p % 2])
     dev = x_in.device
     g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream(device=dev)

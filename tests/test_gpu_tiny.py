@@ -182,6 +182,65 @@ def test_cuda_graph_replay_matches_eager(cuda_device, wl):
 
 
 @pytest.mark.gpu
+def test_graphs_of_two_batch_sizes_replay_independently(cuda_device):
+    """Each graph remembers its own token count and buffers: a graph captured
+    earlier still replays correctly after another one has been captured."""
+    wl = TINY
+    layer = get_layer(wl, cuda_device)
+    x, lg = inputs.make_x(wl, seed=33).to(cuda_device), inputs.make_logits(wl, seed=34).to(cuda_device)
+    y_full = layer.forward(x, lg).clone()
+    y_part = layer.forward(x[:37], lg[:37]).clone()
+    g_full = layer.capture(wl.T)
+    g_part = layer.capture(37)
+    for _ in range(2):
+        y = layer.forward_graph(g_full, x, lg).clone()
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y_full.view(torch.int16))
+        y = layer.forward_graph(g_part, x[:37], lg[:37]).clone()
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y_part.view(torch.int16))
+    with pytest.raises(ValueError, match="captured for T = 37"):
+        layer.forward_graph(g_part, x, lg)
+    with pytest.raises(ValueError, match="not captured by this layer"):
+        get_layer(TINY_MX, cuda_device).forward_graph(g_full, x, lg)
+
+
+@pytest.mark.gpu
+def test_layer_and_binding_refuse_bad_arguments(cuda_device):
+    """Wrong sizes, dtypes, devices or strides raise on the host before any
+    launch (the library takes raw pointers and cannot check them)."""
+    wl = TINY
+    layer = get_layer(wl, cuda_device)
+    T, H, E = wl.T, wl.d_model, wl.num_experts
+    x, lg = inputs.make_x(wl, seed=35).to(cuda_device), inputs.make_logits(wl, seed=36).to(cuda_device)
+    big_x = torch.zeros(T + 1, H, dtype=torch.bfloat16, device=cuda_device)
+    big_lg = torch.zeros(T + 1, E, dtype=torch.float32, device=cuda_device)
+    with pytest.raises(ValueError, match="buffers hold"):
+        layer.forward(big_x, big_lg)
+    with pytest.raises(ValueError, match="^logits: "):
+        layer.forward(x, lg.double())
+    with pytest.raises(ValueError, match="^logits: "):
+        layer.forward(x, lg[:, :E - 1].contiguous())
+    with pytest.raises(ValueError, match="^x: "):
+        layer.forward(x.float(), lg)
+    with pytest.raises(ValueError, match="is on cpu"):
+        layer.forward(x.cpu(), lg.cpu())
+    with pytest.raises(ValueError, match="^logits: "):
+        layer.forward(x, lg[:T - 1])
+    with pytest.raises(ValueError, match="buffers hold"):
+        layer.capture(T + 1)
+    with pytest.raises(ValueError, match="not contiguous"):
+        B.moe_permute(layer.cfg, T, torch.zeros(H, T, dtype=torch.bfloat16, device=cuda_device).t(),
+                      layer.act_scale, layer.slot_to_row, layer.a_codes, layer.a_sf)
+    with pytest.raises(ValueError, match="float32"):
+        layer.quantize_experts(0, *(torch.zeros(1, 3, 3, device=cuda_device) for _ in range(3)))
+    # the layer still works afterwards
+    y = layer.forward(x, lg)
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0 and y.shape == (T, H)
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("wl", [TINY, TINY_MX], ids=lambda w: w.name)
 def test_host_pipeline_matches_eager(cuda_device, wl):
     """Five host batches through HostPipeline (uploads and downloads of
