@@ -96,9 +96,14 @@ def permute_quantize(x, sorted_slots, k, fmt, s_x=None):
 
 
 def swiglu(g, u):
-    """silu(g) * u = g * u / (1 + exp(-g)) in float64."""
+    """silu(g) * u = g * u / (1 + exp(-g)) in float64.
+
+    For g below about -709 exp(-g) overflows to inf and the quotient is the
+    limit, a signed zero; numpy's overflow warning is silenced for that case.
+    """
     g = np.asarray(g, dtype=np.float64)
-    return g * u / (1.0 + np.exp(-g))
+    with np.errstate(over="ignore"):
+        return g * u / (1.0 + np.exp(-g))
 
 
 def expert_ffn(a_deq, wq_deq, fmt, s_h):

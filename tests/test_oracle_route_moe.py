@@ -208,6 +208,37 @@ def test_weight_tensor_scale_maps_largest_magnitude_to_top_of_range():
         assert np.max(np.abs(deq)) <= 0.5 * (1 + 2.0 ** -22)
 
 
+def test_expert_ffn_gemms_against_exact_sums():
+    """Brute force on a tiny expert: with operands on the E2M1 grid times
+    powers of two (so every product and partial sum is exact in float64) the
+    oracle's gate and up outputs equal the exact rational sums element by
+    element, and its down output is within float64 rounding of the exact sum
+    over its own dequantized intermediate."""
+    from fractions import Fraction
+    rng = np.random.default_rng(21)
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+    m, H, I = 3, 32, 32
+
+    def rand(shape):
+        return rng.choice(grid, shape) * rng.choice([-1, 1], shape) * np.exp2(rng.integers(-3, 4, shape))
+
+    a, wg, wu, wd = rand((m, H)), rand((I, H)), rand((I, H)), rand((H, I))
+
+    def exact(A, W):                       # A [m, K] times W [n, K] transposed, in rationals
+        return [[sum(Fraction(float(A[i, c])) * Fraction(float(W[j, c])) for c in range(A.shape[1]))
+                 for j in range(W.shape[0])] for i in range(A.shape[0])]
+
+    f = moe.expert_ffn(a, dict(gate=wg, up=wu, down=wd), moe.MXFP8, None)
+    assert f["gate"].tolist() == [[float(v) for v in row] for row in exact(a, wg)]
+    assert f["up"].tolist() == [[float(v) for v in row] for row in exact(a, wu)]
+    h_deq = fm.mxfp8_dequantize_rows(f["h_codes"], f["h_sf"])
+    o = exact(h_deq, wd)
+    bound = I * 2.0 ** -52 * (np.abs(h_deq) @ np.abs(wd).T)
+    for i in range(m):
+        for j in range(H):
+            assert abs(Fraction(float(f["out"][i, j])) - o[i][j]) <= Fraction(float(bound[i, j]))
+
+
 def test_swiglu_closed_form():
     g = np.array([0.0, 1.0, -1.0, 10.0, -30.0])
     u = np.array([2.0, 3.0, 1.0, 1.0, 1.0])
