@@ -94,6 +94,7 @@ def test_sizes():
         assert off % 256 == 0
 
 
+@pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder pointers: run only where nothing can launch")
 def test_invalid_arguments_are_rejected_before_any_launch():
     """Null or misaligned pointers and small workspaces return a status, with no
     CUDA call made (these run on a machine without a GPU)."""

@@ -95,3 +95,27 @@ def test_capture_stack_refuses_an_empty_stack():
     from fp8_moe_expert_top_b200.layer import capture_stack
     with pytest.raises(ValueError, match="at least one pass"):
         capture_stack([], _host(4, 256, dtype=torch.bfloat16), [None, None], 4)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder pointers: run only where nothing can launch")
+@pytest.mark.parametrize("T", [-1, (1 << 20) + 1])
+def test_token_count_out_of_range_is_refused_before_any_launch(T):
+    """T outside 0..2^20 returns MOE_ERR_UNSUPPORTED from every call that takes
+    T; the pointers (placeholders, never dereferenced) are not looked at."""
+    import ctypes
+    L = B.lib()
+    cfg = ctypes.byref(CFG)
+    p = ctypes.c_void_p(0x10000)
+    calls = {
+        "moe_route_topk": lambda: L.moe_route_topk(cfg, T, p, p, p, p, p, p, p, p, 1 << 30, None),
+        "moe_route_topk_noalloc": lambda: L.moe_route_topk_noalloc(cfg, T, p, p, p, p, p, p, p, None),
+        "moe_permute": lambda: L.moe_permute(cfg, T, p, p, p, p, p, None),
+        "moe_forward": lambda: L.moe_forward(cfg, T, p, p, p, p, p, p, p, p, p, p, None, None, None),
+        "moe_forward_gateup": lambda: L.moe_forward_gateup(cfg, T, p, p, p, p, p, p, p, p, p, None, None, None),
+        "moe_forward_down": lambda: L.moe_forward_down(cfg, T, p, p, p, p, p, p, p, None, None),
+        "moe_unpermute_combine": lambda: L.moe_unpermute_combine(cfg, T, p, p, p, p, None),
+    }
+    for name, call in calls.items():
+        assert call() == 2, name                      # MOE_ERR_UNSUPPORTED
+    assert B.moe_max_rows(CFG, T) == -1
+    assert B.moe_route_workspace_bytes(CFG, T) == -1
