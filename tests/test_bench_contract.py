@@ -71,3 +71,32 @@ def test_gpu_arm_fails_loudly_without_gpu():
                        capture_output=True, text=True, timeout=300)
     assert r.returncode != 0
     assert _json_lines(r.stdout) == []
+
+
+def _bench_module():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_algorithmic_bytes_match_the_published_sizes():
+    """The roofline's numerators: packed weights of all 384 experts are 6.795
+    GB (NVFP4, 0.5625 B per element) and 12.457 GB (MXFP8, 1.03125 B) per
+    layer, 31,457,280 elements per expert; the layer's other compulsory bytes
+    are x and y in bf16 and the float32 logits."""
+    bench = _bench_module()
+    from fp8_moe_expert_top_b200 import inputs
+    for name, per_layer in (("prefill_nvfp4", 6.795e9), ("prefill_mxfp8", 12.457e9)):
+        wl = inputs.WORKLOADS[name]
+        H, I, E, T = wl.d_model, wl.d_ffn, wl.num_experts, wl.T
+        assert 3 * H * I == 31_457_280
+        b = bench.phase_bytes(wl, E, T * wl.top_k)
+        weights = b["layer"] - (T * H * 2 + T * E * 4 + T * H * 2)
+        assert abs(weights - per_layer) <= 0.0005 * per_layer, (name, weights)
+        assert b["gateup"] - (2 * weights / 3) == pytest.approx(T * wl.top_k * (H + I) * (weights / E / (3 * H * I)))
+        # every phase's bytes are positive and the layer excludes the permuted buffers
+        assert all(v > 0 for v in b.values())
+        assert b["layer"] < sum(b[p] for p in bench.PHASES)
+
