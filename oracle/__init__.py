@@ -25,8 +25,9 @@ Sources (pages, by title and section)
     experts": expert activations are quantized to the layer's weight
     format, inside the kernels that produce them.
   Everything the pages leave open (dimensions, router scoring, tie rules,
-  the error metric, the tensor scale) follows the readings listed in the
-  design notes of this repository; each function states the reading it uses.
+  the error metric, the tensor scale) is a reading, the same one the CUDA
+  library implements; each function states the reading it uses and the page
+  passage it follows.
 
 Parity status: every function here is pinned by a CPU test against a
 library routine, a brute-force search, a closed form or a hand-worked

@@ -42,7 +42,12 @@ E2M1_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
 
 
 def e2m1_decode(codes):
-    """4-bit E2M1 codes (bit 3 = sign) -> float64 values."""
+    """4-bit E2M1 codes (bit 3 = sign) -> float64 values.
+
+    Follows the E2M1 element type of the NVFP4 experts (pages "thinkingmachines/Inkling-2-Small", section
+    Overview; "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section "NVFP4 and MXFP8
+    experts"); values as the OCP MX v1.0 format definition.
+    """
     codes = np.asarray(codes).astype(np.int64)
     mag = np.asarray(E2M1_MAGNITUDES, dtype=np.float64)[codes & 7]
     return np.where((codes >> 3) & 1, -mag, mag)
@@ -55,6 +60,10 @@ def e2m1_encode_magnitude(v):
     0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.  At a midpoint the code with a zero
     mantissa bit wins (0, 1, 1, 2, 2, 4, 4); anything above 5 saturates to 6.
     Returns the 3-bit magnitude code (0..7).
+
+    Follows the E2M1 element type of the NVFP4 experts (pages "thinkingmachines/Inkling-2-Small", section
+    Overview; "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section "NVFP4 and MXFP8
+    experts"); rounding as the OCP MX v1.0 conversion rule.
     """
     v = np.asarray(v, dtype=np.float64)
     code = np.zeros(v.shape, dtype=np.int64)
@@ -76,7 +85,12 @@ E4M3_MAX = 448.0
 
 
 def e4m3_decode(codes):
-    """8-bit E4M3FN codes -> float64 values (NaN for 0x7F and 0xFF)."""
+    """8-bit E4M3FN codes -> float64 values (NaN for 0x7F and 0xFF).
+
+    Follows E4M3, the element type of the MXFP8 experts and the block-scale type of NVFP4 (pages
+    "thinkingmachines/Inkling-2-Small", section Overview; "Thinking Machines releases Inkling 2 Small weights
+    under Apache 2.0", section "NVFP4 and MXFP8 experts").
+    """
     codes = np.asarray(codes).astype(np.int64)
     sign = np.where((codes >> 7) & 1, -1.0, 1.0)
     exp = (codes >> 3) & 15
@@ -94,6 +108,10 @@ def e4m3_encode(v):
     Works on the exact value of each input (float32 inputs are exact in
     float64).  Zero results are returned as +0 (code 0x00) whatever the
     sign of the input, the canonical zero of this library.
+
+    Follows E4M3, the element type of the MXFP8 experts and the block-scale type of NVFP4 (pages
+    "thinkingmachines/Inkling-2-Small", section Overview; "Thinking Machines releases Inkling 2 Small weights
+    under Apache 2.0", section "NVFP4 and MXFP8 experts").
     """
     v = np.asarray(v, dtype=np.float64)
     if np.any(np.isnan(v)):
@@ -126,7 +144,11 @@ def e4m3_encode(v):
 # --------------------------------------------------------------------------
 
 def e8m0_decode(codes):
-    """8-bit E8M0 codes -> float64 powers of two (NaN for 0xFF)."""
+    """8-bit E8M0 codes -> float64 powers of two (NaN for 0xFF).
+
+    Follows E8M0, the block-scale type of the MXFP8 experts (page "thinkingmachines/Inkling-2-Small", section
+    Overview).
+    """
     codes = np.asarray(codes).astype(np.int64)
     val = np.exp2(codes.astype(np.float64) - 127.0)
     return np.where(codes == 255, np.nan, val)
@@ -145,6 +167,9 @@ def pairwise_tree_sum_f32(d):
 
     Level by level: (d0+d1), (d2+d3), ... then ((d0+d1)+(d2+d3)), ...; every
     addition is a float32 addition.
+
+    Follows the error sum of the 4-vs-6 pick (page "Thinking Machines releases Inkling 2 Small weights under
+    Apache 2.0", section TL;DR); the pages fix no order, this tree is the order both implementations use.
     """
     s = _f32(d)
     while s.shape[-1] > 1:
@@ -162,7 +187,11 @@ NVFP4_TENSOR_DIVISOR = 2688.0
 
 
 def nvfp4_tensor_scale(amax):
-    """Second-level (tensor) scale s_g = amax / 2688 in float32; 1 when amax == 0."""
+    """Second-level (tensor) scale s_g = amax / 2688 in float32; 1 when amax == 0.
+
+    Follows the NVFP4 two-level scaling (page "Thinking Machines releases Inkling 2 Small weights under Apache
+    2.0", section TL;DR); amax / (6 * 448) is the reading of the tensor scale.
+    """
     amax = F32(amax)
     if amax == 0:
         return F32(1.0)
@@ -180,6 +209,9 @@ def _nvfp4_candidate(x, a, s_g, c):
       err_c = pairwise-tree sum of d_i * d_i
     If S_c is zero every code is zero and err_c is the tree sum of x_i * x_i.
     Returns (codes uint8[..., 16], scale code uint8[...], err float32[...]).
+
+    Follows page "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section TL;DR: each
+    block's maximum is mapped to 4 and to 6.
     """
     denom = (F32(c) * s_g).astype(np.float32)
     ratio = (a / denom).astype(np.float32)
@@ -204,6 +236,9 @@ def nvfp4_quantize_blocks(x, s_g):
     Returns (codes uint8[..., 16] with 4-bit E2M1 codes, scale codes uint8[...]
     in E4M3, chose_four bool[...]).  Candidate 4 is kept only when its error
     is strictly lower than candidate 6's (ties go to 6).
+
+    Follows page "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section TL;DR: the
+    block is quantized both ways and the lower-error result is kept.
     """
     x = _f32(x)
     s_g = F32(s_g)
@@ -223,6 +258,9 @@ def nvfp4_quantize_rows(x, s_g):
     """Quantize a [rows, K] float32 matrix along K (K a multiple of 16).
 
     Returns (codes uint8[rows, K], scale codes uint8[rows, K/16]).
+
+    Follows pages "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section TL;DR and
+    "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section "NVFP4 and MXFP8 experts".
     """
     x = _f32(x)
     rows, K = x.shape
@@ -232,7 +270,11 @@ def nvfp4_quantize_rows(x, s_g):
 
 
 def nvfp4_dequantize_rows(codes, scales, s_g):
-    """Inverse of nvfp4_quantize_rows in float64: code * dec(scale) * s_g."""
+    """Inverse of nvfp4_quantize_rows in float64: code * dec(scale) * s_g.
+
+    Follows pages "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section TL;DR and
+    "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section "NVFP4 and MXFP8 experts".
+    """
     rows, K = codes.shape
     v = e2m1_decode(codes).reshape(rows, K // NVFP4_BLOCK, NVFP4_BLOCK)
     v = v * e4m3_decode(scales)[..., None] * float(F32(s_g))
@@ -252,6 +294,9 @@ def mxfp8_scale_exponent(amax):
 
     floor(log2 amax) is taken exactly from the float32 exponent; amax == 0
     gives 0.  For float32 subnormal amax the result clamps to 0.
+
+    Follows page "thinkingmachines/Inkling-2-Small", section Overview (MXFP8 experts in layers 40-47); the
+    shared exponent as the OCP MX v1.0 rule.
     """
     amax = np.asarray(amax, dtype=np.float64)
     with np.errstate(divide="ignore"):
@@ -267,6 +312,9 @@ def mxfp8_quantize_blocks(x):
     q_i = E4M3(x_i * 2^(127 - e)); multiplying by a power of two is exact
     here (see mxfp8_scale_exponent), and values that land in (448, 512)
     saturate to 448.  Returns (codes uint8[..., 32], scale codes uint8[...]).
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview and "Thinking Machines releases Inkling
+    2 Small weights under Apache 2.0", section "NVFP4 and MXFP8 experts".
     """
     x = _f32(x)
     assert x.shape[-1] == MXFP8_BLOCK
@@ -280,7 +328,11 @@ def mxfp8_quantize_blocks(x):
 
 
 def mxfp8_quantize_rows(x):
-    """Quantize a [rows, K] float32 matrix along K (K a multiple of 32)."""
+    """Quantize a [rows, K] float32 matrix along K (K a multiple of 32).
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview and "Thinking Machines releases Inkling
+    2 Small weights under Apache 2.0", section "NVFP4 and MXFP8 experts".
+    """
     x = _f32(x)
     rows, K = x.shape
     assert K % MXFP8_BLOCK == 0
@@ -289,6 +341,11 @@ def mxfp8_quantize_rows(x):
 
 
 def mxfp8_dequantize_rows(codes, scales):
+    """Inverse of mxfp8_quantize_rows in float64: code * 2^(e - 127).
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview and "Thinking Machines releases Inkling
+    2 Small weights under Apache 2.0", section "NVFP4 and MXFP8 experts".
+    """
     rows, K = codes.shape
     v = e4m3_decode(codes).reshape(rows, K // MXFP8_BLOCK, MXFP8_BLOCK)
     v = v * e8m0_decode(scales)[..., None]
@@ -304,6 +361,9 @@ def bf16_round(v):
 
     Direct rounding of the exact value to 8 significant bits; magnitudes
     below the smallest normal bfloat16 round on the subnormal grid 2^-133.
+
+    Follows the reading that the layer's input x and output y are bf16 (the pages state no activation type);
+    rounding to nearest, ties to even.
     """
     v = np.asarray(v, dtype=np.float64)
     a = np.abs(v)

@@ -36,6 +36,10 @@ def quantize_rows(x, fmt, s_g=None):
 
     NVFP4 uses the 4-vs-6 quantizer with tensor scale s_g; MXFP8 ignores s_g.
     Returns (codes, scales).
+
+    Follows page "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section "NVFP4 and
+    MXFP8 experts": activations are quantized to the layer's weight format; page
+    "thinkingmachines/Inkling-2-Small", section Overview: NVFP4 in layers 0-39, MXFP8 in 40-47.
     """
     if fmt == NVFP4:
         return fm.nvfp4_quantize_rows(x, s_g)
@@ -45,6 +49,11 @@ def quantize_rows(x, fmt, s_g=None):
 
 
 def dequantize_rows(codes, scales, fmt, s_g=None):
+    """Exact float64 values of quantized rows in the layer format (inverse of quantize_rows).
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview and "Thinking Machines releases Inkling
+    2 Small weights under Apache 2.0", section "NVFP4 and MXFP8 experts".
+    """
     if fmt == NVFP4:
         return fm.nvfp4_dequantize_rows(codes, scales, s_g)
     if fmt == MXFP8:
@@ -53,7 +62,11 @@ def dequantize_rows(codes, scales, fmt, s_g=None):
 
 
 def weight_tensor_scale(w, fmt):
-    """Per-(expert, matrix) tensor scale: amax / 2688 for NVFP4, 1 for MXFP8."""
+    """Per-(expert, matrix) tensor scale: amax / 2688 for NVFP4, 1 for MXFP8.
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview and "Thinking Machines releases Inkling
+    2 Small weights under Apache 2.0", section TL;DR.
+    """
     if fmt == NVFP4:
         return fm.nvfp4_tensor_scale(np.max(np.abs(np.asarray(w, dtype=np.float32))))
     return np.float32(1.0)
@@ -64,6 +77,9 @@ def quantize_expert(w_gate, w_up, w_down, fmt):
 
     Returns a dict with, for m in ('gate', 'up', 'down'), the codes
     [rows, K], the block-scale codes [rows, K/block] and the tensor scale.
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview and "Thinking Machines releases Inkling
+    2 Small weights under Apache 2.0", section TL;DR: the experts' weights in NVFP4 (4-vs-6) or MXFP8.
     """
     out = {}
     for name, w in (("gate", w_gate), ("up", w_up), ("down", w_down)):
@@ -74,6 +90,11 @@ def quantize_expert(w_gate, w_up, w_down, fmt):
 
 
 def dequantize_expert(q, fmt):
+    """Exact float64 values of one expert's three quantized matrices.
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview and "Thinking Machines releases Inkling
+    2 Small weights under Apache 2.0", section TL;DR.
+    """
     return {m: dequantize_rows(c, sf, fmt, s) for m, (c, sf, s) in q.items()}
 
 
@@ -87,6 +108,10 @@ def permute_quantize(x, sorted_slots, k, fmt, s_x=None):
     Row r holds token sorted_slots[r] // k; padding rows (slot -1) are left
     out of the result (returned mask is False there).  Every copy of a token
     is the same quantization of x[t], so it is computed once per token.
+
+    Follows page "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section "NVFP4 and
+    MXFP8 experts": the quantization of the expert inputs is part of the kernel that produces them, so every
+    copy of a token is the same quantization.
     """
     x = np.asarray(x, dtype=np.float32)
     codes_t, sf_t = quantize_rows(x, fmt, s_x)
@@ -100,6 +125,8 @@ def swiglu(g, u):
 
     For g below about -709 exp(-g) overflows to inf and the quotient is the
     limit, a signed zero; numpy's overflow warning is silenced for that case.
+
+    Follows the expert FFN; the pages do not print it, SwiGLU without bias is the reading.
     """
     g = np.asarray(g, dtype=np.float64)
     with np.errstate(over="ignore"):
@@ -112,6 +139,9 @@ def expert_ffn(a_deq, wq_deq, fmt, s_h):
     a_deq  float64 [m, H]   dequantized activation rows
     wq_deq dict of float64 dequantized weights
     Returns dict(gate=[m, I], up=[m, I] float64, h_codes, h_sf, out=[m, H]).
+
+    Follows page "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section "NVFP4 and
+    MXFP8 experts": the intermediate is requantized to the layer's format before the down projection.
     """
     g = a_deq @ wq_deq["gate"].T
     u = a_deq @ wq_deq["up"].T
@@ -123,7 +153,10 @@ def expert_ffn(a_deq, wq_deq, fmt, s_h):
 
 
 def combine(out_rows, topk_w, slot_to_row):
-    """y[t] = sum_j w[t, j] * out[slot_to_row[t*k + j]] in float64, then bf16."""
+    """y[t] = sum_j w[t, j] * out[slot_to_row[t*k + j]] in float64, then bf16.
+
+    Follows page "thinkingmachines/Inkling-2-Small", section Overview: routed experts only, no shared expert.
+    """
     T, k = topk_w.shape
     y = np.zeros((T, out_rows.shape[1]), dtype=np.float64)
     for j in range(k):
@@ -142,6 +175,10 @@ def forward(x, logits, experts_q, k, fmt, s_x=None, s_h=None, num_experts=None):
     Returns a dict with every intermediate: the routing tensors, A codes /
     scales per row, gate/up float64 per row, h codes / scales per row, the
     per-row down output and y.
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview, "Thinking Machines releases Inkling 2
+    Small weights under Apache 2.0", section TL;DR and "Thinking Machines releases Inkling 2 Small weights
+    under Apache 2.0", section "NVFP4 and MXFP8 experts".
     """
     x = np.asarray(x, dtype=np.float32)
     T, H = x.shape
@@ -182,6 +219,10 @@ def forward_tokens(x_rows, logits_rows, experts_q, k, fmt, s_x=None, s_h=None):
     The same steps as forward(), applied to each given token on its own:
     top-k, softmax, quantize x[t], the k expert FFNs, weighted sum, bf16.
     experts_q must hold every expert these tokens select.
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview, "Thinking Machines releases Inkling 2
+    Small weights under Apache 2.0", section TL;DR and "Thinking Machines releases Inkling 2 Small weights
+    under Apache 2.0", section "NVFP4 and MXFP8 experts".
     """
     x_rows = np.asarray(x_rows, dtype=np.float32)
     logits_rows = np.asarray(logits_rows, dtype=np.float32)

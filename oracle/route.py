@@ -47,6 +47,11 @@ def exp_own(x):
       p = Horner(1/7!, ..., 1/1!, 1/0!) at r         (multiply, then add)
       exp(x) = p * 2^n
     Arguments below -80 return 0.  Every operation is one float32 rounding.
+
+    Follows the reading that the k selected experts are weighted by a softmax of their logits (the pages route
+    each token to 8 of 384 experts: "thinkingmachines/Inkling-2-Small", section Overview; "Thinking Machines
+    releases Inkling 2 Small weights under Apache 2.0", section "NVFP4 and MXFP8 experts"); the method is Cody
+    and Waite's range reduction (Software Manual for the Elementary Functions, 1980) with a Taylor polynomial.
     """
     x = np.asarray(x, dtype=np.float32)
     n = np.rint((x * LOG2E_F32).astype(np.float32)).astype(np.float32)
@@ -66,6 +71,10 @@ def topk_select(logits, k):
     Selection by definition: k rounds, each taking the largest remaining
     value (numpy argmax returns the first, i.e. lowest, index among equal
     maxima, and compares -0 equal to +0).
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview (384 routed experts, top-8) and
+    "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section "NVFP4 and MXFP8 experts"
+    (8 of 384 experts per token).
     """
     logits = np.asarray(logits, dtype=np.float32)
     if np.any(np.isnan(logits)):
@@ -81,7 +90,12 @@ def topk_select(logits, k):
 
 
 def topk_softmax(logits, ids):
-    """Softmax over the selected logits (float32, sequential sum in rank order)."""
+    """Softmax over the selected logits (float32, sequential sum in rank order).
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview and "Thinking Machines releases Inkling
+    2 Small weights under Apache 2.0", section "NVFP4 and MXFP8 experts"; the softmax over the k selected
+    logits is the reading of the router's weights.
+    """
     logits = np.asarray(logits, dtype=np.float32)
     T, k = ids.shape
     sel = np.take_along_axis(logits, ids.astype(np.int64), axis=1).astype(np.float32)
@@ -94,6 +108,7 @@ def topk_softmax(logits, ids):
 
 
 def round_up(v, m):
+    """Smallest multiple of m that is >= v (v >= 0, m > 0)."""
     return (v + m - 1) // m * m
 
 
@@ -107,6 +122,9 @@ def sort_slots(ids, num_experts):
       sorted_slots  int32[R]     slot stored in each row, -1 for padding,
                                  R = offsets[E]
       slot_to_row   int32[T*k]   inverse map
+
+    Follows page "Thinking Machines releases Inkling 2 Small weights under Apache 2.0", section "NVFP4 and
+    MXFP8 experts": each token's 8 expert slots, grouped by expert for the per-expert GEMMs.
     """
     ids = np.asarray(ids, dtype=np.int64)
     T, k = ids.shape
@@ -132,7 +150,11 @@ def sort_slots(ids, num_experts):
 
 
 def route(logits, k, num_experts):
-    """Whole routing step: top-k ids, softmax weights and the slot sort."""
+    """Whole routing step: top-k ids, softmax weights and the slot sort.
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview and "Thinking Machines releases Inkling
+    2 Small weights under Apache 2.0", section "NVFP4 and MXFP8 experts".
+    """
     ids = topk_select(logits, k)
     w = topk_softmax(logits, ids)
     counts, offsets, sorted_slots, slot_to_row = sort_slots(ids, num_experts)
