@@ -245,3 +245,29 @@ def test_swiglu_closed_form():
     ref = np.array([0.0, 3.0 / (1 + math.exp(-1.0)), -1.0 / (1 + math.e), 10.0 / (1 + math.exp(-10.0)),
                     -30.0 / (1 + math.exp(30.0))])
     np.testing.assert_allclose(moe.swiglu(g, u), ref, rtol=1e-15)
+
+
+@pytest.mark.parametrize("fmt", [moe.NVFP4, moe.MXFP8])
+def test_degenerate_batches(fmt):
+    """An empty batch gives an empty output and no rows; k = E sends every
+    token to every expert (weights a softmax over all E logits, every segment
+    holding all T tokens in order); a single token equals its per-token
+    evaluation."""
+    x, lg, experts, _ = _small_case(fmt, T=5, E=3, k=3, seed=11)
+    s_x, s_h = np.float32(8 / 2688), np.float32(24 / 2688)
+    empty = moe.forward(x[:0], lg[:0], experts, 3, fmt, s_x, s_h)
+    assert empty["y"].shape == (0, x.shape[1])
+    assert empty["offsets"].tolist() == [0, 0, 0, 0] and empty["counts"].tolist() == [0, 0, 0]
+    full = moe.forward(x, lg, experts, 3, fmt, s_x, s_h)
+    assert full["counts"].tolist() == [5, 5, 5]
+    assert full["offsets"].tolist() == [0, 128, 256, 384]
+    for e in range(3):
+        slots = full["sorted_slots"][128 * e:128 * e + 5]
+        assert (slots // 3).tolist() == [0, 1, 2, 3, 4]
+    sel = np.take_along_axis(lg.astype(np.float64), full["topk_ids"].astype(np.int64), axis=1)
+    ref = np.exp(sel - sel[:, :1])
+    np.testing.assert_allclose(full["topk_w"], ref / ref.sum(1, keepdims=True), rtol=4e-7)
+    np.testing.assert_allclose(full["topk_w"].sum(1), 1.0, rtol=1e-6)
+    one = moe.forward(x[2:3], lg[2:3], experts, 3, fmt, s_x, s_h)
+    tok = moe.forward_tokens(x[2:3], lg[2:3], experts, 3, fmt, s_x, s_h)
+    np.testing.assert_array_equal(one["y"], tok["y"])      # same sums in the same order
