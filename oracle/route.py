@@ -149,6 +149,32 @@ def sort_slots(ids, num_experts):
             sorted_slots.astype(np.int32), slot_to_row.astype(np.int32))
 
 
+def router_logits(x, w_router):
+    """Router scores of every token for every routed expert:
+        logits[t, e] = sum_h x[t, h] * W_r[e, h]
+    x [T, H] and W_r [E, H] hold bfloat16 values (passed exactly, widened to
+    float32 or float64).  Each product is exact in float64 (two 8-bit
+    significands); the sum is taken in float64 and rounded once to float32.
+
+    Follows pages "thinkingmachines/Inkling-2-Small", section Overview (each token scored against the 384
+    routed experts, top-8 kept) and "Thinking Machines releases Inkling 2 Small weights under Apache 2.0",
+    section "NVFP4 and MXFP8 experts" (8 of 384 experts per token).  The pages do not print the router; the
+    reading used is a bias-free linear projection of the layer input, bfloat16 weights, one float32 score per
+    expert.
+    """
+    x64 = np.asarray(x, dtype=np.float64)
+    w64 = np.asarray(w_router, dtype=np.float64)
+    return (x64 @ w64.T).astype(np.float32)
+
+
+def router_route(x, w_router, k, num_experts):
+    """Routing of tokens from their layer input: the router scores, then route().
+
+    Follows the same passages as router_logits and route.
+    """
+    return route(router_logits(x, w_router), k, num_experts)
+
+
 def route(logits, k, num_experts):
     """Whole routing step: top-k ids, softmax weights and the slot sort.
 

@@ -143,6 +143,12 @@ MUTANTS = [
      "expert_ffn(a_deq, wq, fmt, s_x)"),
     ("weight_tensor_scale_signed_max", moe, "weight_tensor_scale", "np.max(np.abs(np.asarray(w, dtype=np.float32)))",
      "np.max(np.asarray(w, dtype=np.float32))"),
+    # router scores
+    ("router_logits_float32_sum", rt, "router_logits", "(x64 @ w64.T)",
+     "(x64.astype(np.float32) @ w64.astype(np.float32).T)"),
+    ("router_logits_experts_reversed", rt, "router_logits", "w64 = np.asarray(w_router, dtype=np.float64)",
+     "w64 = np.asarray(w_router, dtype=np.float64)[::-1]"),
+    ("router_logits_no_float32_rounding", rt, "router_logits", ".astype(np.float32)", ""),
 ]
 
 

@@ -30,6 +30,75 @@ def test_exp_own_accuracy_against_math_exp():
     assert rt.exp_own(np.float32(-80.5)) == 0.0
 
 
+# ---------------------------------------------------------------- router scores
+
+def _f32_nearest(q):
+    """The float32 nearest to the rational q, ties to the even significand
+    (decided exactly with fractions)."""
+    from fractions import Fraction
+    f = np.float32(float(q))
+    cands = [np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))]
+    return min(cands, key=lambda c: (abs(Fraction(float(c)) - q), int(np.float32(c).view(np.uint32)) & 1))
+
+
+def _bf16_values(rng, shape, scale=1.0):
+    import torch
+    v = torch.from_numpy((rng.standard_normal(shape) * scale).astype(np.float32)).to(torch.bfloat16)
+    return v.float().numpy()
+
+
+@pytest.mark.parametrize("spread", [False, True])
+def test_router_logits_against_exact_rational_sums(spread):
+    """Every score is the float32 rounding of the exact sum of bf16 products
+    (also when the products span many binades, so that a float32 running sum
+    would drop low bits)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    T, E, H = 8, 16, 256
+    x = _bf16_values(rng, (T, H))
+    if spread:
+        x = _bf16_values(rng, (T, H)) * np.exp2(rng.integers(-12, 13, (T, H))).astype(np.float32)
+    w = _bf16_values(rng, (E, H), 1.0 / 16)
+    got = rt.router_logits(x, w)
+    assert got.dtype == np.float32 and got.shape == (T, E)
+    xf = [[Fraction(float(v)) for v in row] for row in x]
+    wf = [[Fraction(float(v)) for v in row] for row in w]
+    for t in range(T):
+        for e in range(E):
+            q = sum(a * b for a, b in zip(xf[t], wf[e]))
+            assert got[t, e] == _f32_nearest(q), (t, e, got[t, e], float(q))
+
+
+def test_router_logits_of_one_hot_rows():
+    """A token that is a scaled unit vector scores each expert with that
+    column of the router weights, exactly."""
+    rng = np.random.default_rng(12)
+    w = _bf16_values(rng, (5, 16))
+    x = np.zeros((3, 16), dtype=np.float32)
+    x[0, 3], x[1, 15], x[2, 0] = 1.0, -2.0, 0.5
+    got = rt.router_logits(x, w)
+    np.testing.assert_array_equal(got[0], w[:, 3])
+    np.testing.assert_array_equal(got[1], -2.0 * w[:, 15])
+    np.testing.assert_array_equal(got[2], 0.5 * w[:, 0])
+
+
+def test_router_route_equal_router_rows_tie_to_lower_index():
+    """Two experts with the same router row score the same on every token;
+    whenever both are selected the lower index comes first."""
+    rng = np.random.default_rng(13)
+    w = _bf16_values(rng, (12, 32))
+    w[9] = w[2]
+    x = _bf16_values(rng, (400, 32))
+    r = rt.router_route(x, w, 4, 12)
+    both = 0
+    for row in r["topk_ids"].tolist():
+        if 2 in row and 9 in row:
+            both += 1
+            assert row.index(2) + 1 == row.index(9)
+        assert 9 not in row or 2 in row
+    assert both > 0
+
+
 # ---------------------------------------------------------------- top-k
 
 @pytest.mark.parametrize("ties", [False, True])
