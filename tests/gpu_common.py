@@ -37,8 +37,10 @@ def oracle_expert(wl, e, device):
 
 
 def gpu_expert(layer, wl, e):
-    packed = layer.packed.cpu().numpy()
-    return decode_expert(packed, layer.layout, wl.fmt, e, wl.d_model, wl.d_ffn)
+    """Expert e's (codes, scales, tensor scale) read back from the device,
+    copying only that expert's byte ranges of the packed buffer."""
+    get = lambda off, n: layer.packed[off:off + n].cpu().numpy()  # noqa: E731
+    return decode_expert(get, layer.layout, wl.fmt, e, wl.d_model, wl.d_ffn)
 
 
 def assert_expert_equal(got, ref, e):

@@ -21,6 +21,14 @@ def sf_index(rows, nsf):
     return atom * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + c % 4
 
 
+def sf_index_rows(rows, nsf):
+    """Byte offset of every (row, col) scale of the given rows, int64 [len(rows), nsf]."""
+    r = np.asarray(rows, dtype=np.int64)[:, None]
+    c = np.arange(nsf, dtype=np.int64)[None, :]
+    atom = (r // 128) * (nsf // 4) + c // 4
+    return atom * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + c % 4
+
+
 def unswizzle_sf(buf, rows, nsf):
     """[rows, nsf] uint8 scales from an atom-layout buffer (rows % 128 == 0)."""
     buf = np.asarray(buf, dtype=np.uint8).reshape(-1)
@@ -116,20 +124,25 @@ def w13_row(m, c):
 def decode_expert(packed, layout, fmt, e, H, I):
     """(codes, scales, tensor scale) of gate, up and down of expert e.
 
-    packed: uint8 numpy array of the whole packed buffer (or a copy of it).
+    packed: uint8 numpy array of the whole packed buffer (or a copy of it),
+    or a function (offset, nbytes) -> uint8 numpy array of that byte range.
     """
     v = sfvec(fmt)
-    p = np.asarray(packed, dtype=np.uint8)
+    if callable(packed):
+        get = packed
+    else:
+        p = np.asarray(packed, dtype=np.uint8)
+        get = lambda off, n: p[off:off + n]  # noqa: E731
     kb13, kb2 = kb_padded(H, fmt), kb_padded(I, fmt)
     n13 = 2 * I * kb13
-    c13 = p[layout.w13_codes + e * n13: layout.w13_codes + (e + 1) * n13]
+    c13 = get(layout.w13_codes + e * n13, n13)
     s13n = 2 * I * H // v
-    s13 = p[layout.w13_sf + e * s13n: layout.w13_sf + (e + 1) * s13n]
+    s13 = get(layout.w13_sf + e * s13n, s13n)
     n2 = H * kb2
-    c2 = p[layout.w2_codes + e * n2: layout.w2_codes + (e + 1) * n2]
+    c2 = get(layout.w2_codes + e * n2, n2)
     s2n = H * I // v
-    s2 = p[layout.w2_sf + e * s2n: layout.w2_sf + (e + 1) * s2n]
-    scales = p[layout.scales + 12 * e: layout.scales + 12 * (e + 1)].view(np.float32)
+    s2 = get(layout.w2_sf + e * s2n, s2n)
+    scales = np.ascontiguousarray(get(layout.scales + 12 * e, 12)).view(np.float32)
     codes13 = tiled_codes(fmt, c13, np.arange(2 * I), H, WEIGHT_TR)
     sf13 = unswizzle_sf(s13, 2 * I, H // v)
     codes2 = tiled_codes(fmt, c2, np.arange(H), I, WEIGHT_TR)

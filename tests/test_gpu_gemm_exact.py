@@ -51,23 +51,30 @@ def to_rows_bytes(fmt, codes):
 
 
 # Expert row counts and token counts: a decode-like case (T * k <= 128 * E)
-# and a prefill-like one (several 128-row blocks per expert, odd block counts,
-# partly filled last blocks).
+# and prefill-like ones (several 128-row blocks per expert, odd block counts,
+# partly filled last blocks, an empty expert).
 CASES = {
     "decode_like": (np.array([130, 0, 5, 256], dtype=np.int32), 391),
     "prefill_like": (np.array([200, 50, 300], dtype=np.int32), 550),
+    "prefill_long": (np.array([300, 0, 1000], dtype=np.int32), 1300),
 }
+
+# (H, I, case): three small shapes, and the model's own d_model 4096 / expert
+# ffn 2560, where the K loop turns the 4-stage ring many times (16 NVFP4 or
+# 32 MXFP8 K tiles in gate/up, 10 or 20 in down), an expert spans up to 8
+# row blocks and every persistent CTA walks several tiles.
+SHAPES = ([(H, I, c) for H, I in [(256, 128), (512, 256), (1024, 384)] for c in ("decode_like", "prefill_like")]
+          + [(4096, 2560, "decode_like"), (4096, 2560, "prefill_long")])
 
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("fmt", ["nvfp4", "mxfp8"])
-@pytest.mark.parametrize("H,I", [(256, 128), (512, 256), (1024, 384)])
-@pytest.mark.parametrize("case", sorted(CASES))
+@pytest.mark.parametrize("H,I,case", SHAPES)
 def test_gemm_integer_exact(cuda_device, fmt, H, I, case):
-    rng = np.random.default_rng(H * 7 + I + (1 if fmt == "mxfp8" else 0) + (3 if case == "prefill_like" else 0))
+    rng = np.random.default_rng(H * 7 + I + (1 if fmt == "mxfp8" else 0) + (3 if case != "decode_like" else 0))
     counts, T = CASES[case]
     E, k = len(counts), 1
-    assert (T * k > 128 * E) == (case == "prefill_like")
+    assert (T * k > 128 * E) == (case != "decode_like")
     assert counts.sum() == T
     offsets = np.concatenate([[0], np.cumsum((counts + 127) // 128 * 128)]).astype(np.int32)
     cfg = B.make_config(E, k, H, I, fmt)
