@@ -28,17 +28,15 @@ constexpr int kMaxDevices = 64;
 void* g_scratch_addr[kMaxDevices] = {nullptr};
 std::mutex g_scratch_mutex;
 
-// Device address of g_route_scratch on the current device (looked up once
-// per device; host code cannot use the symbol itself as a device pointer).
-cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
+// Device address of g_route_scratch on device `dev`, which must be the
+// current device (looked up once per device; host code cannot use the
+// symbol itself as a device pointer).
+cudaError_t scratch_address(int dev, void** out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
   if (g_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
-    err = cudaGetSymbolAddress(&p, g_route_scratch);
+    const cudaError_t err = cudaGetSymbolAddress(&p, g_route_scratch);
     if (err != cudaSuccess) return err;
     g_scratch_addr[dev] = p;
   }
@@ -57,8 +55,18 @@ extern "C" MOE_API moe_status moe_route_topk_noalloc(const moe_config* cfg, int6
   const int64_t need = moe_route_workspace_bytes(cfg, T);
   if (need < 0) return MOE_ERR_UNSUPPORTED;
   if (need > kScratchBytes) return MOE_ERR_WORKSPACE;  // more tokens x experts than the fixed scratch holds
+  // The scratch address is per device: the work must go to the current
+  // device.  A stream of another device is refused before anything is
+  // enqueued (the legacy and per-thread default streams belong to the current
+  // device).
+  int dev = 0, stream_dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (stream != nullptr) {
+    if (cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &stream_dev) != cudaSuccess) return MOE_ERR_INVALID_ARG;
+    if (stream_dev != dev) return MOE_ERR_INVALID_ARG;
+  }
   void* scratch = nullptr;
-  if (scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  if (scratch_address(dev, &scratch) != cudaSuccess) return MOE_ERR_CUDA;
   // Every byte of scratch that the kernels read is written earlier in the
   // same call, so nothing has to be cleared between calls.
   return moe_route_topk(cfg, T, logits, topk_ids, topk_w, expert_counts, expert_offsets, sorted_slots, slot_to_row,

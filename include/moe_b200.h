@@ -247,7 +247,13 @@ MOE_API moe_status moe_unpermute_combine(const moe_config* cfg, int64_t T, const
  *     and enqueue nothing.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) for that device; make that first call outside
- *     any CUDA stream capture.
+ *     any CUDA stream capture.  With CUDA's lazy module loading (the
+ *     default) the array's 4 MiB are only then allocated on that device, so
+ *     the first call can fail with MOE_ERR_CUDA when the device is out of
+ *     memory; later calls reuse the address.
+ *   - The work runs on the current device: `stream` must be NULL (the
+ *     default stream) or a stream of the current device, else the call
+ *     returns MOE_ERR_INVALID_ARG and enqueues nothing.
  *   - All calls share the one array: calls whose work overlaps on the GPU
  *     (different streams, or different host threads) race and may return
  *     wrong results.  Calls on one stream are safe.
