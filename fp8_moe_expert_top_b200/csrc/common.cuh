@@ -143,6 +143,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Wait for the phase with the given parity to complete, ignoring the abort
+// flag; returns false after limit_ns.  Used to drain work already in flight
+// once a CTA has aborted.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u && globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Bulk copies global -> shared (the TMA engine's 1-D mode, no multicast)
 // ---------------------------------------------------------------------------

@@ -36,8 +36,11 @@
 // its MMAs; so the MMA thread issues none and each stage's 12 (NVFP4) copies
 // are spread over two threads of their own.
 // Every mbarrier wait is bounded; a wait that runs out raises a CTA-wide
-// abort flag, every role stops issuing, TMEM is freed and a status bit is
-// set.
+// abort flag and every role stops issuing.  Work already in flight (bulk
+// copies into stages nobody consumed, MMAs, scale copies) is then waited for,
+// again with a time limit, before TMEM is freed; if that wait also runs out,
+// TMEM is left allocated rather than freed under a running tensor-core
+// operation.  A status bit reports the abort.
 #include <atomic>
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -87,8 +90,10 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
   uint64_t* tfull_bar = empty_bar + kStages;
   uint64_t* tempty_bar = tfull_bar + 1;
   uint64_t* sf_bar = tempty_bar + 1;  // a stage's scales are in TMEM
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_bar + kStages);
+  uint64_t* drain_bar = sf_bar + kStages;  // after an abort: in-flight tcgen05 work has finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* drain_failed = reinterpret_cast<volatile int*>(tmem_slot + 2);
   int32_t* s_offsets = reinterpret_cast<int32_t*>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -102,7 +107,9 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
     }
     mbar_init(tfull_bar, 1);
     mbar_init(tempty_bar, 32 * kEpiWarps);
+    mbar_init(drain_bar, 1 + kCopierWarps);
     *abort_flag = 0;
+    *drain_failed = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -123,6 +130,9 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
   const int total = m_tiles * n_tiles;
   const int k_tiles = (args.K + Tr::kElemsPerStage - 1) / Tr::kElemsPerStage;
   uint32_t fail_bits = 0;
+  // producer: stages armed for a bulk copy (bit s) and the full-barrier
+  // phase parity each was armed in; drained after an abort
+  uint32_t armed = 0u, armed_par = 0u;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -167,6 +177,8 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
           for (int h = 0; h < kBN / 128; ++h)
             bulk_load(st + Tr::kSfbOff + h * Tr::kSfBytes128, b_sf + h * args.sf_rb_stride + kt * Tr::kSfBytes128,
                       sf_bytes, &full_bar[stage], pol_w);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
@@ -310,7 +322,29 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) {
+  // Every role has left its loop; the abort flag no longer changes.  After a
+  // normal run nothing is in flight (each stage's copies landed before its
+  // MMAs ran, each scale copy finished before its MMAs ran, the last MMAs
+  // before the epilogue's last wait).  After an abort, wait for what is.
+  if (*abort_flag) {
+    bool drained = true;
+    if (warp == 0 && lane == 0) {
+      // a stage's copies complete its full barrier phase whether or not the
+      // MMA warp consumed it, and a stage is re-armed only after it is freed
+      for (int st = 0; st < kStages; ++st)
+        if ((armed >> st) & 1u) drained = mbar_wait_drain(&full_bar[st], (armed_par >> st) & 1u) && drained;
+    } else if ((warp == 1 || warp >= kThreads / 32) && lane == 0) {
+      // MMAs and scale copies this thread issued: one arrival each on the
+      // drain barrier once they have completed
+      tc_commit(drain_bar);
+      drained = mbar_wait_drain(drain_bar, 0);
+    }
+    if (!drained) *drain_failed = 1;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  if (warp == 1 && !*drain_failed) {
     __syncwarp();
     tmem_dealloc(tmem_base, kTmemCols);
   }
@@ -321,7 +355,7 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
 template <int FMT, bool GATEUP>
 static cudaError_t launch_one(const GemmArgs& a, cudaStream_t stream) {
   using Tr = GemmTraits<FMT, kBN, kStages>;
-  const size_t smem = 1024 + kStages * Tr::kStageBytes + (3 * kStages + 2) * 8 + 16 + (a.E + 1) * 4;
+  const size_t smem = 1024 + kStages * Tr::kStageBytes + (3 * kStages + 3) * 8 + 16 + (a.E + 1) * 4;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -331,7 +365,7 @@ static cudaError_t launch_one(const GemmArgs& a, cudaStream_t stream) {
   int sms = (dev < 64) ? sm_count[dev].load(std::memory_order_relaxed) : 0;
   if (sms == 0) {
     // the largest size any supported E needs (E <= 1024)
-    const size_t smem_max = 1024 + kStages * Tr::kStageBytes + (3 * kStages + 2) * 8 + 16 + 1025 * 4;
+    const size_t smem_max = 1024 + kStages * Tr::kStageBytes + (3 * kStages + 3) * 8 + 16 + 1025 * 4;
     err = cudaFuncSetAttribute(moe_gemm_kernel<FMT, GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem_max));
     if (err != cudaSuccess) return err;
@@ -345,7 +379,7 @@ static cudaError_t launch_one(const GemmArgs& a, cudaStream_t stream) {
 size_t gemm_smem_bytes(int fmt, int E) {
   const int sb = (fmt == MOE_NVFP4) ? GemmTraits<MOE_NVFP4, kBN, kStages>::kStageBytes
                                     : GemmTraits<MOE_MXFP8, kBN, kStages>::kStageBytes;
-  return 1024 + kStages * sb + (3 * kStages + 2) * 8 + 16 + (E + 1) * 4;
+  return 1024 + kStages * sb + (3 * kStages + 3) * 8 + 16 + (E + 1) * 4;
 }
 
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
