@@ -1,15 +1,18 @@
 """Benchmark of the routed MoE expert layer on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--only] [--impl ours|reference]
 
 One step is one pass of the whole layer over one batch of synthetic inputs
 already resident in HBM: route -> permute+quantize -> gate/up GEMM (SwiGLU +
 requantization) -> down GEMM -> weighted combine.  Default workload: the
-decode NVFP4 layer (64 tokens, d_model 4096, expert ffn 2560, 384 experts,
-top-8).  Weights are random-init of that architecture, quantized once by the
-library before timing.  Every timed step is bracketed by CUDA events on the
-launching stream; L2 is flushed (a 512 MiB write) between timed steps,
-outside the events.  With --gpus N > 1 (launched by torchrun) every rank runs
+largest single-GPU layer, NVFP4 with Zipf-skewed routing (16,384 tokens,
+d_model 4096, expert ffn 2560, 384 experts, top-8); on one GPU the same run
+also measures the other four full-size layers (decode NVFP4 T=64, decode
+MXFP8 T=256, prefill NVFP4 T=8192, prefill MXFP8 T=8192) and reports them
+under "workloads" (--only skips them).  Weights are random-init of that
+architecture, quantized once by the library before timing.  Every timed step
+is bracketed by CUDA events on the launching stream; L2 is flushed (a 512 MiB
+write) between timed steps, outside the events.  With --gpus N > 1 (launched by torchrun) every rank runs
 an independent replica of the same workload (the layer has no data-path
 exchange on one node: "replicas only"), the times are max-reduced over ranks
 and `value` counts the tokens of all ranks.
@@ -37,6 +40,9 @@ from fp8_moe_expert_top_b200 import inputs  # noqa: E402
 
 METRIC = "MoE layer tokens/s on 1 B200; % of HBM or NVFP4/FP8 tensor roofline"
 UNIT = "tokens/s"
+# the largest single-GPU layer, and the other full-size layers measured beside it
+HEADLINE = "prefill_nvfp4_skewed"
+FULL_SIZE = ("decode_nvfp4", "decode_mxfp8", "prefill_nvfp4", "prefill_nvfp4_skewed", "prefill_mxfp8")
 
 
 # --------------------------------------------------------------------------- helpers
@@ -344,6 +350,9 @@ def run_ours(args, wl, ws, rank, local):
     else:
         roof = {"bound": "tensor", "achieved": dom_flops / t_dom / 1e12, "peak": tensor_peak, "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    # against the nominal B200 peaks (8 TB/s HBM; 9 / 4.5 PFLOP/s dense NVFP4 / FP8)
+    roof["frac_nominal"] = roof["achieved"] / (8000.0 if roof["bound"] == "hbm" else
+                                               (9000.0 if wl.fmt == inputs.NVFP4 else 4500.0))
     roof["kernel"] = f"moe_gemm_kernel ({dom})"
     roof["peak_source"] = peak_kind + (" hbm_gbs" if roof["bound"] == "hbm" else
                                        f" bf16_tflops x {4 if wl.fmt == inputs.NVFP4 else 2} (nominal ratio)")
@@ -547,7 +556,9 @@ def cpu_baseline(wl, n_tokens=None):
 def run_reference(args, wl, ws, rank):
     if rank != 0:
         return None
-    n = default_sample_tokens(wl)
+    # one token per step at full size (about 4 s of host work each), so a
+    # run of the default 20 + 5 steps ends within a few minutes
+    n = 1 if wl.d_model * wl.d_ffn > (1 << 20) else default_sample_tokens(wl)
     x, lg, experts = oracle_sample(wl, n)
     for _ in range(args.warmup):
         time_oracle(wl, x, lg, experts)
@@ -577,7 +588,8 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode_nvfp4", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--only", action="store_true", help="measure only --workload, not the other full-size layers")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=None,
@@ -620,6 +632,17 @@ def main(argv=None):
         out, layer = run_ours(args, wl, ws, rank, local)
         del layer
         torch.cuda.empty_cache()
+        if ws == 1 and not args.only and args.experts is None and args.tokens is None:
+            out["workloads"] = {}
+            for name in FULL_SIZE:
+                if name == wl.name:
+                    continue
+                o, layer = run_ours(args, inputs.WORKLOADS[name], ws, rank, local)
+                del layer
+                torch.cuda.empty_cache()
+                out["workloads"][name] = {key: o[key] for key in (
+                    "value", "unit", "ms_per_step", "dtype", "config", "roofline", "layer_roofline_frac",
+                    "layer_roofline_frac_nominal", "step_ms_pct", "phase_ms", "e2e", "gpu_launches", "clocks")}
         if rank == 0:
             if ws == 1 and not args.no_cpu_baseline:
                 out["cpu_baseline"] = cpu_baseline(wl)
