@@ -57,6 +57,7 @@ SIGNATURES = {
     "moe_route_workspace_bytes": (_I64, [_CFG, _I64]),
     "moe_quantize_weights": (ctypes.c_int, [_CFG, _I32, _I32, _P, _P, _P, _P, _P]),
     "moe_route_topk": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P]),
+    "moe_router_topk": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P]),
     "moe_permute": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_forward_gateup": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -174,6 +175,17 @@ def moe_route_topk_noalloc(cfg, T, logits, topk_ids, topk_w, expert_counts, expe
     p, st = _marshal("moe_route_topk_noalloc", stream, logits, topk_ids, topk_w, expert_counts, expert_offsets,
                      sorted_slots, slot_to_row)
     _check("moe_route_topk_noalloc", lib().moe_route_topk_noalloc(ctypes.byref(cfg), int(T), *p, st))
+
+
+def moe_router_topk(cfg, T, x, w_router, logits_out, topk_ids, topk_w, expert_counts, expert_offsets, sorted_slots,
+                    slot_to_row, workspace, status_word=None, stream=None):
+    """Routing from bf16 x [T, H] and bf16 router weights [E, H]; logits_out
+    (float32 [T, E]) is an optional copy of the scores."""
+    p, st = _marshal("moe_router_topk", stream, x, w_router, logits_out, topk_ids, topk_w, expert_counts,
+                     expert_offsets, sorted_slots, slot_to_row, workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    status = _marshal("moe_router_topk", stream, status_word)[0][0]
+    _check("moe_router_topk", lib().moe_router_topk(ctypes.byref(cfg), int(T), *p, ws_bytes, status, st))
 
 
 def moe_permute(cfg, T, x, act_scale, slot_to_row, a_codes, a_sf, stream=None):

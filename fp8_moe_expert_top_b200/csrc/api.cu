@@ -129,6 +129,33 @@ moe_status moe_route_topk(const moe_config* cfg, int64_t T, const float* logits,
                                      workspace, static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_router_topk(const moe_config* cfg, int64_t T, const void* x_bf16, const void* w_router_bf16,
+                           float* logits_out, int32_t* topk_ids, float* topk_w, int32_t* expert_counts,
+                           int32_t* expert_offsets, int32_t* sorted_slots, int32_t* slot_to_row, void* workspace,
+                           int64_t workspace_bytes, uint32_t* status_word, void* stream) {
+  moe_status s = check(cfg);
+  if (s != MOE_OK) return s;
+  if ((s = check_T(T)) != MOE_OK) return s;
+  if (cfg->num_experts > 512) return MOE_ERR_UNSUPPORTED;  // all scores of a token in one TMEM accumulator
+  if (!expert_counts || !expert_offsets || !sorted_slots) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x_bf16 || !w_router_bf16 || !topk_ids || !topk_w || !slot_to_row || !workspace))
+    return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < moe::route_workspace_bytes(cfg->num_experts, T)) return MOE_ERR_WORKSPACE;
+  if ((x_bf16 && !aligned16(x_bf16)) || (w_router_bf16 && !aligned16(w_router_bf16)) ||
+      (workspace && !aligned16(workspace)) || (logits_out && !aligned16(logits_out)))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int E = cfg->num_experts, k = cfg->top_k;
+  cudaError_t err = moe::route_prepare(static_cast<int>(T), E, expert_counts, expert_offsets, sorted_slots,
+                                       max_rows(cfg, T), workspace, st);
+  if (err != cudaSuccess || T == 0) return from_cuda(err);
+  err = moe::launch_router_topk(x_bf16, w_router_bf16, logits_out, static_cast<int>(T), E, cfg->d_model, k, topk_ids,
+                                topk_w, workspace, status_word, st);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  return from_cuda(moe::route_finish(static_cast<int>(T), E, k, topk_ids, expert_counts, expert_offsets, sorted_slots,
+                                     slot_to_row, workspace, st));
+}
+
 moe_status moe_permute(const moe_config* cfg, int64_t T, const void* x_bf16, const float* act_scale,
                        const int32_t* slot_to_row, void* a_codes, void* a_sf, void* stream) {
   moe_status s = check(cfg);

@@ -12,6 +12,21 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
                          int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
                          int32_t* slot_to_row, int64_t R_max, void* workspace, cudaStream_t stream);
 
+// The routing steps around the top-k: zero the token bitmaps and mark every
+// row of sorted_slots as padding (prepare), then per-expert counts, padded
+// offsets and the slot scatter from the bitmaps (finish).
+cudaError_t route_prepare(int T, int E, int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
+                          int64_t R_max, void* workspace, cudaStream_t stream);
+cudaError_t route_finish(int T, int E, int k, const int32_t* topk_ids, int32_t* expert_counts,
+                         int32_t* expert_offsets, int32_t* sorted_slots, int32_t* slot_to_row, void* workspace,
+                         cudaStream_t stream);
+
+// Router scores fused with the top-k (logits = x W_r^T on tcgen05, then the
+// same top-k, softmax and bitmaps as route_topk_kernel); E <= 512.
+cudaError_t launch_router_topk(const void* x, const void* w_router, float* logits_out, int T, int E, int H, int k,
+                               int32_t* topk_ids, float* topk_w, void* workspace, uint32_t* status,
+                               cudaStream_t stream);
+
 cudaError_t launch_permute(int fmt, int T, int H, int k, const void* x, const float* act_scale,
                            const int32_t* slot_to_row, uint8_t* a_codes, uint8_t* a_sf, cudaStream_t stream);
 

@@ -22,33 +22,9 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "route_common.cuh"
 
 namespace moe {
-
-// exp(x) for x <= 0 by Cody-Waite reduction and a degree-7 Taylor series,
-// one float32 rounding per operation (see the header for the definition).
-__device__ __forceinline__ float exp_own(float x) {
-  const float kLog2e = 0x1.715476p+0f;      // log2(e) rounded to float32
-  const float kLn2Hi = 0x1.62e4p-1f;        // 0.693145751953125 (16 significant bits)
-  const float kLn2Lo = 0x1.7f7d1cp-20f;     // ln(2) - kLn2Hi rounded to float32
-  // 1/i! rounded to float32, i = 0..7
-  const float c0 = 1.0f, c1 = 1.0f, c2 = 0.5f, c3 = 0x1.555556p-3f, c4 = 0x1.555556p-5f,
-              c5 = 0x1.111112p-7f, c6 = 0x1.6c16c2p-10f, c7 = 0x1.a01a02p-13f;
-  if (x < -80.0f) return 0.0f;
-  const float n = rintf(__fmul_rn(x, kLog2e));
-  float r = __fsub_rn(x, __fmul_rn(n, kLn2Hi));
-  r = __fsub_rn(r, __fmul_rn(n, kLn2Lo));
-  float p = c7;
-  p = __fadd_rn(__fmul_rn(p, r), c6);
-  p = __fadd_rn(__fmul_rn(p, r), c5);
-  p = __fadd_rn(__fmul_rn(p, r), c4);
-  p = __fadd_rn(__fmul_rn(p, r), c3);
-  p = __fadd_rn(__fmul_rn(p, r), c2);
-  p = __fadd_rn(__fmul_rn(p, r), c1);
-  p = __fadd_rn(__fmul_rn(p, r), c0);
-  const float two_n = __uint_as_float(static_cast<uint32_t>(static_cast<int>(n) + 127) << 23);
-  return __fmul_rn(p, two_n);
-}
 
 constexpr int kTopkWarps = 8;  // tokens per CTA of the top-k kernel
 
@@ -230,9 +206,8 @@ int64_t route_workspace_bytes(int E, int64_t T) {
   return static_cast<int64_t>(E) * W * 8 + 256;  // bitmap words + their prefix counts
 }
 
-cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w,
-                         int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
-                         int32_t* slot_to_row, int64_t R_max, void* workspace, cudaStream_t stream) {
+cudaError_t route_prepare(int T, int E, int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
+                          int64_t R_max, void* workspace, cudaStream_t stream) {
   cudaError_t err = cudaMemsetAsync(sorted_slots, 0xFF, static_cast<size_t>(R_max) * sizeof(int32_t), stream);
   if (err != cudaSuccess) return err;
   if (T == 0) {
@@ -241,10 +216,31 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
     return cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), stream);
   }
   const int W = (T + 31) / 32;
-  uint32_t* bitmap = static_cast<uint32_t*>(workspace);
-  int32_t* prefix = reinterpret_cast<int32_t*>(bitmap + static_cast<int64_t>(E) * W);
-  err = cudaMemsetAsync(bitmap, 0, static_cast<size_t>(E) * W * sizeof(uint32_t), stream);
+  return cudaMemsetAsync(workspace, 0, static_cast<size_t>(E) * W * sizeof(uint32_t), stream);
+}
+
+cudaError_t route_finish(int T, int E, int k, const int32_t* topk_ids, int32_t* expert_counts,
+                         int32_t* expert_offsets, int32_t* sorted_slots, int32_t* slot_to_row, void* workspace,
+                         cudaStream_t stream) {
+  const int W = (T + 31) / 32;
+  const uint32_t* bitmap = static_cast<const uint32_t*>(workspace);
+  int32_t* prefix = reinterpret_cast<int32_t*>(static_cast<uint32_t*>(workspace) + static_cast<int64_t>(E) * W);
+  cudaError_t err = launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, stream, E, W, bitmap, prefix,
+                               expert_counts, expert_offsets);
   if (err != cudaSuccess) return err;
+  const int64_t slots = static_cast<int64_t>(T) * k;
+  return launch_pdl(route_scatter_kernel, dim3(static_cast<unsigned>((slots + 255) / 256)), dim3(256), 0, stream, T,
+                    E, k, W, topk_ids, bitmap, static_cast<const int32_t*>(prefix),
+                    static_cast<const int32_t*>(expert_offsets), sorted_slots, slot_to_row);
+}
+
+cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w,
+                         int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
+                         int32_t* slot_to_row, int64_t R_max, void* workspace, cudaStream_t stream) {
+  cudaError_t err = route_prepare(T, E, expert_counts, expert_offsets, sorted_slots, R_max, workspace, stream);
+  if (err != cudaSuccess || T == 0) return err;
+  const int W = (T + 31) / 32;
+  uint32_t* bitmap = static_cast<uint32_t*>(workspace);
   const int npl = (E + 31) / 32;
   const dim3 grid((T + kTopkWarps - 1) / kTopkWarps), block(kTopkWarps * 32);
   const float* lg = logits;
@@ -257,14 +253,7 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
   else
     err = launch_pdl(route_topk_kernel<32>, grid, block, 0, stream, lg, T, E, k, W, topk_ids, topk_w, bitmap);
   if (err != cudaSuccess) return err;
-  err = launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, stream, E, W, static_cast<const uint32_t*>(bitmap),
-                   prefix, expert_counts, expert_offsets);
-  if (err != cudaSuccess) return err;
-  const int64_t slots = static_cast<int64_t>(T) * k;
-  return launch_pdl(route_scatter_kernel, dim3(static_cast<unsigned>((slots + 255) / 256)), dim3(256), 0, stream, T,
-                    E, k, W, static_cast<const int32_t*>(topk_ids), static_cast<const uint32_t*>(bitmap),
-                    static_cast<const int32_t*>(prefix), static_cast<const int32_t*>(expert_offsets), sorted_slots,
-                    slot_to_row);
+  return route_finish(T, E, k, topk_ids, expert_counts, expert_offsets, sorted_slots, slot_to_row, workspace, stream);
 }
 
 }  // namespace moe

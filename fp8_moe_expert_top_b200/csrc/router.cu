@@ -1,0 +1,376 @@
+// Router scores fused with the top-k: logits = x W_r^T on tcgen05, and in
+// the same kernel the per-token top-k, the softmax over the k selected scores
+// and the per-expert token bitmaps that the slot sort counts.
+//
+// Pages: "thinkingmachines/Inkling-2-Small" (vLLM recipe), section Overview,
+// and "Thinking Machines releases Inkling 2 Small weights under Apache 2.0",
+// section "NVFP4 and MXFP8 experts": every token is scored against the 384
+// routed experts and sent to the 8 best.  The scores never reach global
+// memory (unless the caller asks for a debug copy): the accumulator in TMEM
+// is reduced to the k selected experts by the epilogue.
+//
+// One CTA per 128 tokens:
+//   warp 0      producer: TMA tile loads (cp.async.bulk.tensor, 128-byte
+//               swizzle, no multicast) of 64 bf16 of K for the 128 token rows
+//               of x and for all expert rows of W_r, into a ring of stages
+//   warp 1      MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
+//               M = 128, N = 256 and/or 128 per 128-expert block, the
+//               accumulator of all (up to 512) experts in TMEM
+//   warps 2-5   epilogue: one token row per thread: tcgen05.ld 32 scores at
+//               a time, a sorted top-8 kept in registers (strict '>' while
+//               scanning experts in ascending order, so equal scores keep the
+//               lower index), then the same softmax and bitmap update as
+//               route_topk_kernel (bit-identical weights for equal scores).
+// Every wait is bounded; a wait that runs out raises the CTA's abort flag,
+// the roles stop, work in flight is drained and a status bit is set.
+#include <cstdint>
+#include <mutex>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "route_common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRM = 128;           // tokens per CTA (TMEM lanes)
+constexpr int kRKElems = 64;       // bf16 of K per stage (128 bytes per row)
+constexpr int kREpiWarps = 4;
+constexpr int kRThreads = 64 + 32 * kREpiWarps;
+constexpr int kRTileBytes = kRM * 128;  // one 128-row x 128-byte tile
+
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* tmap, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 operands, fp32 accumulator.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, M = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+struct RouterArgs {
+  float* logits_out;  // optional [T][E] debug copy of the scores
+  int32_t* topk_ids;
+  float* topk_w;
+  uint32_t* bitmap;   // [E][W] token bitmaps
+  uint32_t* status;
+  int T, E, H, k, W;
+};
+
+// NB: 128-expert blocks of W_r (1..4); ST: ring stages.
+template <int NB, int ST>
+__global__ void __launch_bounds__(kRThreads, 1)
+    router_topk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                       const RouterArgs args) {
+  constexpr int kStageBytes = kRTileBytes * (1 + NB);
+  constexpr uint32_t kTmemCols = NB == 1 ? 128u : (NB == 2 ? 256u : 512u);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + ST * kStageBytes);
+  uint64_t* empty_bar = full_bar + ST;
+  uint64_t* acc_bar = empty_bar + ST;
+  uint64_t* drain_bar = acc_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* drain_failed = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kRM;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(acc_bar, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *drain_failed = 0;
+    fence_mbar_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  pdl_wait();
+  pdl_trigger();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int k_tiles = args.H / kRKElems;
+  uint32_t fail_bits = 0;
+  uint32_t armed = 0u, armed_par = 0u;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+          fail_bits |= MOE_DEVICE_TIMEOUT_PRODUCER;
+          break;
+        }
+        uint8_t* st = smem + stage * kStageBytes;
+        // a box that reaches past the last token or expert is filled with
+        // zeros and still counts its full size
+        mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
+        tma_load_2d(st, &tmap_x, kt * kRKElems, m0, &full_bar[stage]);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+          tma_load_2d(st + kRTileBytes * (1 + b), &tmap_w, kt * kRKElems, b * 128, &full_bar[stage]);
+        armed |= 1u << stage;
+        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == ST) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+          fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + stage * kStageBytes);
+        const uint64_t adesc = make_desc_sw128(st);
+#pragma unroll
+        for (int kk = 0; kk < kRKElems / 16; ++kk) {
+          const uint32_t acc = (kt | kk) != 0 ? 1u : 0u;
+#pragma unroll
+          for (int b = 0; b < NB; b += 2) {
+            const uint64_t bdesc = make_desc_sw128(st + kRTileBytes * (1 + b));
+            if (b + 1 < NB)
+              tc_mma_bf16(tmem_base + 128 * b, adesc + 2 * kk, bdesc + 2 * kk, idesc_bf16(256), acc);
+            else
+              tc_mma_bf16(tmem_base + 128 * b, adesc + 2 * kk, bdesc + 2 * kk, idesc_bf16(128), acc);
+          }
+        }
+        tc_commit(&empty_bar[stage]);
+        if (++stage == ST) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) tc_commit(acc_bar);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    const int row = q * 32 + lane;
+    const int t = m0 + row;
+    if (mbar_wait(acc_bar, 0, abort_flag)) {
+      tc_fence_after();
+      float tv[8];
+      int ti[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        tv[j] = -INFINITY;
+        ti[j] = 0x7FFFFFFF;
+      }
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < NB * 4; ++c) {
+        float v[32];
+        tmem_ld32(t_row + 32 * c, v);
+        tmem_ld_wait();
+        if (t < args.T) {
+          if (args.logits_out != nullptr) {
+            float* dst = args.logits_out + static_cast<int64_t>(t) * args.E;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (32 * c + i < args.E) dst[32 * c + i] = v[i];
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int e = 32 * c + i;
+            // strictly better than the current 8th (an empty slot loses to
+            // anything); experts arrive in ascending order, so an equal score
+            // already held keeps its lower index ahead
+            if (e < args.E && (v[i] > tv[7] || ti[7] == 0x7FFFFFFF)) {
+              tv[7] = v[i];
+              ti[7] = e;
+#pragma unroll
+              for (int j = 7; j > 0; --j) {
+                if (tv[j] > tv[j - 1] || ti[j - 1] == 0x7FFFFFFF) {
+                  const float fv = tv[j];
+                  tv[j] = tv[j - 1];
+                  tv[j - 1] = fv;
+                  const int fi = ti[j];
+                  ti[j] = ti[j - 1];
+                  ti[j - 1] = fi;
+                }
+              }
+            }
+          }
+        }
+      }
+      if (t < args.T) {
+        // softmax over the k selected scores, as route_topk_kernel computes it
+        const int k = args.k;
+        float ex[8];
+        float s = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          ex[j] = (j < k) ? exp_own(__fsub_rn(tv[j], tv[0])) : 0.0f;
+          if (j == 0) s = ex[0];
+          else if (j < k) s = __fadd_rn(s, ex[j]);
+        }
+        const int64_t o = static_cast<int64_t>(t) * k;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < k) {
+            args.topk_ids[o + j] = ti[j];
+            args.topk_w[o + j] = __fdiv_rn(ex[j], s);
+            atomicOr(&args.bitmap[static_cast<int64_t>(ti[j]) * args.W + (t >> 5)], 1u << (t & 31));
+          }
+        }
+      }
+    } else {
+      fail_bits |= MOE_DEVICE_TIMEOUT_EPILOGUE;
+    }
+  }
+
+  if (fail_bits != 0u && args.status != nullptr) atomicOr(args.status, fail_bits);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (*abort_flag) {
+    // drain what is in flight before TMEM is freed (as in the expert GEMMs)
+    bool drained = true;
+    if (warp == 0 && lane == 0) {
+      for (int st = 0; st < ST; ++st)
+        if ((armed >> st) & 1u) drained = mbar_wait_drain(&full_bar[st], (armed_par >> st) & 1u) && drained;
+    } else if (warp == 1 && lane == 0) {
+      tc_commit(drain_bar);
+      drained = mbar_wait_drain(drain_bar, 0);
+    }
+    if (!drained) *drain_failed = 1;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  if (warp == 1 && !*drain_failed) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template <int NB>
+constexpr int router_stages() {
+  return (kRTileBytes * (1 + NB) * 4 <= 200 * 1024) ? 4 : ((kRTileBytes * (1 + NB) * 3 <= 200 * 1024) ? 3 : 2);
+}
+template <int NB>
+constexpr size_t router_smem() {
+  return 1024 + static_cast<size_t>(router_stages<NB>()) * kRTileBytes * (1 + NB) +
+         (2 * router_stages<NB>() + 2) * 8 + 16;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// A [rows][H] bf16 row-major matrix, loaded in boxes of 64 elements x 128
+// rows with the 128-byte swizzle; rows past the end read as zeros.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t H) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kRKElems), static_cast<cuuint32_t>(kRM)};
+  const cuuint32_t elem[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NB>
+cudaError_t launch_nb(const CUtensorMap& mx, const CUtensorMap& mw, const RouterArgs& a, cudaStream_t stream) {
+  constexpr int ST = router_stages<NB>();
+  constexpr size_t smem = router_smem<NB>();
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(router_topk_kernel<NB, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem));
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const dim3 grid(static_cast<unsigned>((a.T + kRM - 1) / kRM));
+  return launch_pdl(router_topk_kernel<NB, ST>, grid, dim3(kRThreads), smem, stream, mx, mw, a);
+}
+
+}  // namespace
+
+cudaError_t launch_router_topk(const void* x, const void* w_router, float* logits_out, int T, int E, int H, int k,
+                               int32_t* topk_ids, float* topk_w, void* workspace, uint32_t* status,
+                               cudaStream_t stream) {
+  CUtensorMap mx, mw;
+  if (!make_map(&mx, x, T, H) || !make_map(&mw, w_router, E, H)) return cudaErrorInvalidValue;
+  RouterArgs a;
+  a.logits_out = logits_out;
+  a.topk_ids = topk_ids;
+  a.topk_w = topk_w;
+  a.bitmap = static_cast<uint32_t*>(workspace);
+  a.status = status;
+  a.T = T;
+  a.E = E;
+  a.H = H;
+  a.k = k;
+  a.W = (T + 31) / 32;
+  const int nb = (E + 127) / 128;
+  switch (nb) {
+    case 1: return launch_nb<1>(mx, mw, a, stream);
+    case 2: return launch_nb<2>(mx, mw, a, stream);
+    case 3: return launch_nb<3>(mx, mw, a, stream);
+    case 4: return launch_nb<4>(mx, mw, a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace moe

@@ -94,6 +94,21 @@ class ExpertLayer:
         B.moe_route_topk(self.cfg, T, logits, self.topk_ids, self.topk_w, self.expert_counts,
                          self.expert_offsets, self.sorted_slots, self.slot_to_row, self.route_ws)
 
+    def set_router(self, w_router):
+        """bf16 router weights [E, H] (device) for routing from x (route_x)."""
+        if w_router.dtype != torch.bfloat16 or tuple(w_router.shape) != (self.E, self.H):
+            raise ValueError(f"w_router: bfloat16 ({self.E}, {self.H}) expected, got {w_router.dtype} "
+                             f"{tuple(w_router.shape)}")
+        if w_router.device != self.device:
+            raise ValueError(f"w_router is on {w_router.device}, the layer on {self.device}")
+        self.w_router = w_router.contiguous()
+
+    def route_x(self, x, T, logits_out=None):
+        """Routing from the layer input x [>= T, H] bf16: router scores fused
+        with the top-k (moe_router_topk)."""
+        B.moe_router_topk(self.cfg, T, x, self.w_router, logits_out, self.topk_ids, self.topk_w, self.expert_counts,
+                          self.expert_offsets, self.sorted_slots, self.slot_to_row, self.route_ws, self.status)
+
     def permute(self, x, T):
         B.moe_permute(self.cfg, T, x, self.act_scale, self.slot_to_row, self.a_codes, self.a_sf)
 
@@ -165,13 +180,20 @@ class ExpertLayer:
         graph.replay()
         return y_out[:T]
 
-    def forward(self, x, logits):
-        """y[:T] for bf16 x [T, H] and float32 logits [T, E] already on the device."""
+    def forward(self, x, logits=None):
+        """y[:T] for bf16 x [T, H] and float32 logits [T, E] already on the
+        device; with logits None the router weights given to set_router score
+        the tokens (moe_router_topk)."""
         T = x.shape[0]
         self._check_io(T, x, logits)
-        if logits.shape[0] != T:
-            raise ValueError(f"x has {T} rows, logits {logits.shape[0]}")
-        self.route(logits, T)
+        if logits is None:
+            if getattr(self, "w_router", None) is None:
+                raise ValueError("no logits and no router weights (set_router)")
+            self.route_x(x, T)
+        else:
+            if logits.shape[0] != T:
+                raise ValueError(f"x has {T} rows, logits {logits.shape[0]}")
+            self.route(logits, T)
         self.permute(x, T)
         self.gateup(T)
         self.down(T)

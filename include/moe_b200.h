@@ -187,6 +187,30 @@ MOE_API moe_status moe_route_topk(const moe_config* cfg, int64_t T, const float*
                           float* topk_w, int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
                           int32_t* slot_to_row, void* workspace, int64_t workspace_bytes, void* stream);
 
+/* Routing from the layer input, with the router scores fused into the
+ * top-k [P1 Overview; P2 "NVFP4 and MXFP8 experts": each token is scored
+ * against the routed experts and sent to the top_k best].  The scores
+ *     logits[t][e] = sum_h x[t][h] * w_router[e][h]
+ * are computed on the tensor cores (bf16 products, float32 accumulation) and
+ * reduced to the k selected experts in the same kernel; they reach memory only
+ * through the optional logits_out.  Then, exactly as moe_route_topk does for
+ * given logits: top-k (ties to the lower index, rank order), the softmax over
+ * the k selected scores, counts, padded offsets and the slot sort.
+ *   x_bf16         bf16 [T][d_model], row-major (the layer input)
+ *   w_router_bf16  bf16 [num_experts][d_model], row-major (no bias)
+ *   logits_out     optional float32 [T][num_experts]: a copy of the scores
+ *                  (NULL in normal use)
+ *   other outputs and workspace as for moe_route_topk (same sizes)
+ *   status_word    optional uint32 device status word (MOE_DEVICE_*)
+ * Supported: num_experts <= 512 (MOE_ERR_UNSUPPORTED otherwise).  The
+ * float32 sums are taken in the tensor core's order, so a score can differ
+ * from the exactly rounded sum in its last bits; results do not depend on
+ * thread timing. */
+MOE_API moe_status moe_router_topk(const moe_config* cfg, int64_t T, const void* x_bf16, const void* w_router_bf16,
+                                   float* logits_out, int32_t* topk_ids, float* topk_w, int32_t* expert_counts,
+                                   int32_t* expert_offsets, int32_t* sorted_slots, int32_t* slot_to_row,
+                                   void* workspace, int64_t workspace_bytes, uint32_t* status_word, void* stream);
+
 /* Permute-gather with fused activation quantization [P2 "NVFP4 and MXFP8
  * experts": activations quantized to the weight format inside the producing
  * kernel; P2 TL;DR: the 4-vs-6 pick].  Token t's row x[t] (bf16 [T][H]) is

@@ -22,6 +22,7 @@ CALLS = {
     "moe_quantize_weights": lambda h: B.moe_quantize_weights(CFG, 0, 1, h, h, h, h),
     "moe_route_topk": lambda h: B.moe_route_topk(CFG, 4, h, h, h, h, h, h, h, h),
     "moe_route_topk_noalloc": lambda h: B.moe_route_topk_noalloc(CFG, 4, h, h, h, h, h, h, h),
+    "moe_router_topk": lambda h: B.moe_router_topk(CFG, 4, h, h, h, h, h, h, h, h, h, h, h),
     "moe_permute": lambda h: B.moe_permute(CFG, 4, h, h, h, h, h),
     "moe_forward": lambda h: B.moe_forward(CFG, 4, h, h, h, h, h, h, h, h, h, h),
     "moe_forward_gateup": lambda h: B.moe_forward_gateup(CFG, 4, h, h, h, h, h, h, h, h, h),
@@ -109,6 +110,7 @@ def test_token_count_out_of_range_is_refused_before_any_launch(T):
     calls = {
         "moe_route_topk": lambda: L.moe_route_topk(cfg, T, p, p, p, p, p, p, p, p, 1 << 30, None),
         "moe_route_topk_noalloc": lambda: L.moe_route_topk_noalloc(cfg, T, p, p, p, p, p, p, p, None),
+        "moe_router_topk": lambda: L.moe_router_topk(cfg, T, p, p, None, p, p, p, p, p, p, p, 1 << 30, None, None),
         "moe_permute": lambda: L.moe_permute(cfg, T, p, p, p, p, p, None),
         "moe_forward": lambda: L.moe_forward(cfg, T, p, p, p, p, p, p, p, p, p, p, None, None, None),
         "moe_forward_gateup": lambda: L.moe_forward_gateup(cfg, T, p, p, p, p, p, p, p, p, p, None, None, None),
