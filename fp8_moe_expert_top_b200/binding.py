@@ -23,6 +23,7 @@ MOE_DEVICE_TIMEOUT_PRODUCER = 0x1
 MOE_DEVICE_TIMEOUT_MMA = 0x2
 MOE_DEVICE_TIMEOUT_EPILOGUE = 0x4
 MOE_DEVICE_TIMEOUT_SELFTEST = 0x8
+MOE_DEVICE_BAD_GROUP_EXPERT = 0x10
 
 
 class MoeError(RuntimeError):
@@ -62,6 +63,7 @@ SIGNATURES = {
     "moe_forward": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_forward_gateup": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_forward_down": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_forward_grouped": (ctypes.c_int, [_CFG, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_unpermute_combine": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P]),
     "moe_route_topk_noalloc": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_selftest_bounded_wait": (ctypes.c_int, [_P, _I64, _P]),
@@ -212,6 +214,13 @@ def moe_forward_down(cfg, T, packed, h_codes, h_sf, inter_scale, expert_offsets,
     p, st = _marshal("moe_forward_down", stream, packed, h_codes, h_sf, inter_scale, expert_offsets, expert_counts,
                      down_out, status_word)
     _check("moe_forward_down", lib().moe_forward_down(ctypes.byref(cfg), int(T), *p, st))
+
+
+def moe_forward_grouped(cfg, num_groups, packed, a_codes, a_sf, act_scale, inter_scale, group_offsets, group_counts,
+                        group_expert, h_codes, h_sf, down_out, gateup_debug=None, status_word=None, stream=None):
+    p, st = _marshal("moe_forward_grouped", stream, packed, a_codes, a_sf, act_scale, inter_scale, group_offsets,
+                     group_counts, group_expert, h_codes, h_sf, down_out, gateup_debug, status_word)
+    _check("moe_forward_grouped", lib().moe_forward_grouped(ctypes.byref(cfg), int(num_groups), *p, st))
 
 
 def moe_unpermute_combine(cfg, T, down_out, topk_w, slot_to_row, y, stream=None):

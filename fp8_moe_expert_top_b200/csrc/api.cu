@@ -262,6 +262,67 @@ moe_status moe_forward(const moe_config* cfg, int64_t T, const void* packed, con
                           status_word, stream);
 }
 
+moe_status moe_forward_grouped(const moe_config* cfg, int32_t num_groups, const void* packed, const void* a_codes,
+                               const void* a_sf, const float* act_scale, const float* inter_scale,
+                               const int32_t* group_offsets, const int32_t* group_counts,
+                               const int32_t* group_expert, void* h_codes, void* h_sf, void* down_out,
+                               float* gateup_debug, uint32_t* status_word, void* stream) {
+  moe_status s = check(cfg);
+  if (s != MOE_OK) return s;
+  if (num_groups < 0 || num_groups > 1024) return MOE_ERR_UNSUPPORTED;
+  if (num_groups == 0) return MOE_OK;
+  if (!packed || !a_codes || !a_sf || !group_offsets || !group_counts || !group_expert || !h_codes || !h_sf ||
+      !down_out)
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->fmt == MOE_NVFP4 && (!act_scale || !inter_scale)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(a_codes) || !aligned16(a_sf) || !aligned16(h_codes) || !aligned16(h_sf) ||
+      !aligned16(down_out) || (gateup_debug && !aligned16(gateup_debug)))
+    return MOE_ERR_INVALID_ARG;
+  moe_weights_layout L;
+  layout(cfg, &L);
+  const uint8_t* base = static_cast<const uint8_t*>(packed);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  moe::GemmLaunch g{};
+  g.fmt = cfg->fmt;
+  g.E = num_groups;
+  g.offsets = group_offsets;
+  g.counts = group_counts;
+  g.expert_map = group_expert;
+  g.n_weights = cfg->num_experts;
+  g.w_scales = reinterpret_cast<const float*>(base + L.scales);
+  g.status = status_word;
+  // gate/up + SwiGLU + requantized h
+  g.gateup = true;
+  g.K = cfg->d_model;
+  g.n_rows_b = 2 * cfg->d_ffn;
+  g.a_codes = static_cast<const uint8_t*>(a_codes);
+  g.a_sf = static_cast<const uint8_t*>(a_sf);
+  g.b_codes = base + L.w13_codes;
+  g.b_sf = base + L.w13_sf;
+  g.a_scale = act_scale;
+  g.h_scale = inter_scale;
+  g.h_codes = static_cast<uint8_t*>(h_codes);
+  g.h_sf = static_cast<uint8_t*>(h_sf);
+  g.dbg = gateup_debug;
+  cudaError_t err = moe::launch_gemm(g, st);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  // down
+  g.gateup = false;
+  g.K = cfg->d_ffn;
+  g.n_rows_b = cfg->d_model;
+  g.a_codes = static_cast<const uint8_t*>(h_codes);
+  g.a_sf = static_cast<const uint8_t*>(h_sf);
+  g.b_codes = base + L.w2_codes;
+  g.b_sf = base + L.w2_sf;
+  g.a_scale = inter_scale;
+  g.h_scale = nullptr;
+  g.h_codes = nullptr;
+  g.h_sf = nullptr;
+  g.dbg = nullptr;
+  g.out = down_out;
+  return from_cuda(moe::launch_gemm(g, st));
+}
+
 moe_status moe_unpermute_combine(const moe_config* cfg, int64_t T, const void* down_out, const float* topk_w,
                                  const int32_t* slot_to_row, void* y_bf16, void* stream) {
   moe_status s = check(cfg);

@@ -65,10 +65,15 @@ static_assert(kBN + kStages * 48 <= kTmemCols, "scale buffers do not fit in TMEM
 // tile, and the expert's 128-row blocks (mt) fastest.  CTAs running at the same
 // time therefore share one weight tile (read from HBM once, then from L2), and
 // an expert's activation rows are re-read from L2 for each weight tile.
+// A row group is one expert's segment; with an expert map (grouped calls)
+// group e uses the weights of expert map[e] (an index outside the packed
+// weights is clamped to 0 and reported through the status word).
 struct TileCoord {
-  int e, mt, nt, m_blocks;
+  int e, we, mt, nt, m_blocks;
+  bool bad;
 };
-__device__ __forceinline__ TileCoord tile_coord(int tile, const int32_t* offs, int E, int n_tiles) {
+__device__ __forceinline__ TileCoord tile_coord(int tile, const int32_t* offs, int E, int n_tiles,
+                                                const int32_t* emap, int n_weights) {
   TileCoord c;
   c.e = find_expert(offs, E, (tile / n_tiles) * kBM);
   const int mt0 = offs[c.e] / kBM;
@@ -76,6 +81,13 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const int32_t* offs, i
   const int local = tile - mt0 * n_tiles;
   c.nt = local / c.m_blocks;
   c.mt = mt0 + local % c.m_blocks;
+  c.we = c.e;
+  c.bad = false;
+  if (emap != nullptr) {
+    const int w = __ldg(emap + c.e);
+    c.bad = w < 0 || w >= n_weights;
+    c.we = c.bad ? 0 : w;
+  }
   return c;
 }
 
@@ -145,15 +157,15 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-        const TileCoord tc = tile_coord(tile, s_offsets, E, n_tiles);
-        const int mt = tc.mt, nt = tc.nt, e = tc.e;
+        const TileCoord tc = tile_coord(tile, s_offsets, E, n_tiles, args.expert_map, args.n_weights);
+        const int mt = tc.mt, nt = tc.nt, e = tc.e, we = tc.we;
         const uint64_t pol_w = tc.m_blocks > 1 ? pol_keep : pol_stream;
         const uint8_t* a_sf = args.a_sf + static_cast<int64_t>(mt) * args.sf_rb_stride;
-        const uint8_t* b_sf = args.b_sf + static_cast<int64_t>(e) * args.b_sf_expert_stride +
+        const uint8_t* b_sf = args.b_sf + static_cast<int64_t>(we) * args.b_sf_expert_stride +
                               static_cast<int64_t>(nt) * (kBN / 128) * args.sf_rb_stride;
         const int64_t ktiles_row = args.kb >> 7;  // K tiles per code row
         const uint8_t* a_tiles = args.a_codes + static_cast<int64_t>(mt) * ktiles_row * Tr::kABytes;
-        const uint8_t* b_tiles = args.b_codes + static_cast<int64_t>(e) * args.b_expert_stride +
+        const uint8_t* b_tiles = args.b_codes + static_cast<int64_t>(we) * args.b_expert_stride +
                                  static_cast<int64_t>(nt) * ktiles_row * Tr::kBBytes;
         // Only the row block's valid rows are loaded (rounded up to 16); the
         // rest of the A tile keeps stale data, whose output rows are never
@@ -296,9 +308,10 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
     const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + half * (kBN / 2);
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-      const TileCoord tc = tile_coord(tile, s_offsets, E, n_tiles);
+      const TileCoord tc = tile_coord(tile, s_offsets, E, n_tiles, args.expert_map, args.n_weights);
       const int mt = tc.mt, nt = tc.nt, e = tc.e;
       const int valid_rows = s_offsets[e] + __ldg(args.counts + e) - mt * kBM;
+      if (tc.bad && warp == 2 && lane == 0) fail_bits |= MOE_DEVICE_BAD_GROUP_EXPERT;
       const bool valid = row_l < valid_rows;
       const int64_t row = static_cast<int64_t>(mt) * kBM + row_l;
       if (!mbar_wait(tfull_bar, acc_phase, abort_flag)) {
@@ -314,7 +327,7 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
       mbar_arrive(tempty_bar);
       acc_phase ^= 1u;
       if (!valid) continue;
-      epilogue_rows<FMT, GATEUP>(args, acc, row, e, nt, half);
+      epilogue_rows<FMT, GATEUP>(args, acc, row, tc.we, nt, half);
     }
   }
 
@@ -403,6 +416,8 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
   a.dbg = g.dbg;
   a.out = static_cast<__nv_bfloat16*>(g.out);
   a.status = g.status;
+  a.expert_map = g.expert_map;
+  a.n_weights = g.expert_map != nullptr ? g.n_weights : g.E;
   a.E = g.E;
   a.K = g.K;
   a.n_rows_b = g.n_rows_b;

@@ -56,7 +56,9 @@ struct GemmArgs {
   float* dbg;
   __nv_bfloat16* out;
   uint32_t* status;
-  int E;
+  const int32_t* expert_map;  // optional: weights of row group e are expert_map[e]
+  int n_weights;              // experts in the packed weights
+  int E;                      // row groups (experts, or segments with an expert map)
   int K;            // reduction length in elements
   int n_rows_b;     // weight rows per expert (2I for gate/up, H for down)
   int64_t kb;                 // bytes of one code row, padded to a multiple of 128

@@ -57,6 +57,8 @@ struct GemmLaunch {
   float* dbg;
   void* out;              // down: bf16 [R_max][H]
   uint32_t* status;
+  const int32_t* expert_map;  // optional [E]: row group -> expert of the packed weights
+  int n_weights;              // experts in the packed weights (with expert_map)
 };
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream);
 

@@ -95,6 +95,9 @@ typedef struct {
 #define MOE_DEVICE_TIMEOUT_MMA 0x2u
 #define MOE_DEVICE_TIMEOUT_EPILOGUE 0x4u
 #define MOE_DEVICE_TIMEOUT_SELFTEST 0x8u
+/* moe_forward_grouped: a group named an expert outside the packed weights
+ * (expert 0's weights were used for its rows instead). */
+#define MOE_DEVICE_BAD_GROUP_EXPERT 0x10u
 
 /* Layout of the packed expert weights (byte offsets from the buffer start).
  * For NVFP4 (bits = 4, sfvec = 16) and MXFP8 (bits = 8, sfvec = 32), with
@@ -252,6 +255,35 @@ MOE_API moe_status moe_forward_gateup(const moe_config* cfg, int64_t T, const vo
 MOE_API moe_status moe_forward_down(const moe_config* cfg, int64_t T, const void* packed, const void* h_codes,
                             const void* h_sf, const float* inter_scale, const int32_t* expert_offsets,
                             const int32_t* expert_counts, void* down_out, uint32_t* status_word, void* stream);
+
+/* Expert FFN over rows grouped by the expert whose weights they use, for
+ * expert parallelism [P1 Overview: expert parallelism follows the TP group]:
+ * a rank that holds a slice of the experts receives, from every rank, the
+ * rows routed to its experts, each source's rows already grouped by expert
+ * and padded to 128 rows.  Row group g (rows group_offsets[g] ..
+ * group_offsets[g] + group_counts[g] - 1) is computed exactly as moe_forward
+ * computes the rows of expert group_expert[g] of `packed`.
+ *   cfg            num_experts = experts held in `packed` (this rank's slice)
+ *   num_groups     row groups, 0 .. 1024
+ *   group_offsets  int32 [num_groups + 1], device: first row of each group,
+ *                  multiples of 128, non-decreasing, group_offsets[0] = 0
+ *   group_counts   int32 [num_groups], device: rows in use per group,
+ *                  <= group_offsets[g + 1] - group_offsets[g]
+ *   group_expert   int32 [num_groups], device: expert of `packed` per group;
+ *                  an index outside 0 .. num_experts - 1 is replaced by 0 and
+ *                  sets MOE_DEVICE_BAD_GROUP_EXPERT in the status word
+ *   a_codes, a_sf, h_codes, h_sf, down_out, gateup_debug, scales, status
+ *                  as for moe_forward, sized for group_offsets[num_groups]
+ *                  rows (buffers sized by moe_codes_bytes / moe_sf_bytes for a
+ *                  multiple of 128 rows at least that large)
+ * The row layout and the results of each row are independent of the other
+ * groups: a row gives the same bits as in moe_forward. */
+MOE_API moe_status moe_forward_grouped(const moe_config* cfg, int32_t num_groups, const void* packed,
+                                       const void* a_codes, const void* a_sf, const float* act_scale,
+                                       const float* inter_scale, const int32_t* group_offsets,
+                                       const int32_t* group_counts, const int32_t* group_expert, void* h_codes,
+                                       void* h_sf, void* down_out, float* gateup_debug, uint32_t* status_word,
+                                       void* stream);
 
 /* Weighted un-permute and combine [routed experts, no shared expert, P1
  * Overview]: y[t] = sum_{j<k} topk_w[t][j] * down_out[slot_to_row[t*k+j]],

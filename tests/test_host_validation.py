@@ -27,6 +27,7 @@ CALLS = {
     "moe_forward": lambda h: B.moe_forward(CFG, 4, h, h, h, h, h, h, h, h, h, h),
     "moe_forward_gateup": lambda h: B.moe_forward_gateup(CFG, 4, h, h, h, h, h, h, h, h, h),
     "moe_forward_down": lambda h: B.moe_forward_down(CFG, 4, h, h, h, h, h, h, h),
+    "moe_forward_grouped": lambda h: B.moe_forward_grouped(CFG, 2, h, h, h, h, h, h, h, h, h, h, h),
     "moe_unpermute_combine": lambda h: B.moe_unpermute_combine(CFG, 4, h, h, h, h),
     "moe_selftest_bounded_wait": lambda h: B.moe_selftest_bounded_wait(h, 1000),
 }
