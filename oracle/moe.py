@@ -240,3 +240,75 @@ def forward_tokens(x_rows, logits_rows, experts_q, k, fmt, s_x=None, s_h=None):
             f = expert_ffn(a_deq[t:t + 1], cache[e], fmt, s_h)
             y[t] += float(w[t, j]) * f["out"][0]
     return dict(topk_ids=ids, topk_w=w, a_codes=codes, a_sf=sf, y=fm.bf16_round(y))
+
+
+# --------------------------------------------------------------------------
+# BF16 experts with LoRA adapters
+# --------------------------------------------------------------------------
+
+def lora_project(a, w, lora_a, lora_b, scaling):
+    """a W^T + scaling * (a A^T) B^T in float64: a projection with weight
+    W [N, K] and a rank-r adapter A [r, K], B [N, r].
+
+    Follows page "thinkingmachines/Inkling-2-Small", section Configurations, and page "Thinking Machines
+    releases Inkling 2 Small weights under Apache 2.0", section "LoRA and reinforcement learning": adapters on
+    the routed experts need BF16 expert weights (a rank-32 adapter in the pages' validation run).  The adapter
+    form is the usual low-rank update W + scaling * B A, applied without merging.
+    """
+    a = np.asarray(a, dtype=np.float64)
+    out = a @ np.asarray(w, dtype=np.float64).T
+    if lora_a is None:
+        return out
+    z = a @ np.asarray(lora_a, dtype=np.float64).T
+    return out + float(scaling) * (z @ np.asarray(lora_b, dtype=np.float64).T)
+
+
+def expert_ffn_bf16(a, w, lora, scaling):
+    """One BF16 expert with adapters on gate, up and down:
+        g = proj(a, gate), u = proj(a, up), h = bf16(silu(g) * u),
+        out = proj(h, down)
+    a float64 [m, H] (bf16 values); w dict of bf16-valued [I, H] / [H, I]
+    matrices; lora dict m -> (A, B) or None.  The intermediate h is the bf16
+    input of the down projection, as in a BF16 model.
+
+    Follows the same passages as lora_project; SwiGLU as in expert_ffn.
+    """
+    lo = lora or {}
+    g = lora_project(a, w["gate"], *lo.get("gate", (None, None)), scaling)
+    u = lora_project(a, w["up"], *lo.get("up", (None, None)), scaling)
+    h = fm.bf16_round(swiglu(g, u))
+    out = lora_project(h, w["down"], *lo.get("down", (None, None)), scaling)
+    return dict(gate=g, up=u, h=h, out=out)
+
+
+def forward_bf16(x, logits, experts_w, experts_lora, k, scaling, num_experts=None):
+    """Whole layer with BF16 experts and adapters: route -> per-expert FFN on
+    the rows of its tokens (no quantization) -> combine.
+
+    experts_w[e] dict of gate/up/down bf16-valued matrices; experts_lora[e]
+    dict m -> (A, B), or None for an expert without adapters.
+
+    Follows the same passages as lora_project, and route / combine.
+    """
+    x = np.asarray(x, dtype=np.float32)
+    T, H = x.shape
+    E = num_experts if num_experts is not None else logits.shape[1]
+    r = rt.route(logits, k, E)
+    R = r["sorted_slots"].shape[0]
+    out_rows = np.zeros((R, H), dtype=np.float64)
+    gate = up = hb = None
+    for e in range(E):
+        lo, cnt = int(r["offsets"][e]), int(r["counts"][e])
+        if cnt == 0:
+            continue
+        tok = r["sorted_slots"][lo:lo + cnt] // k
+        f = expert_ffn_bf16(x[tok].astype(np.float64), experts_w[e], experts_lora.get(e), scaling)
+        if gate is None:
+            I = f["gate"].shape[1]
+            gate, up, hb = np.zeros((R, I)), np.zeros((R, I)), np.zeros((R, I))
+        gate[lo:lo + cnt], up[lo:lo + cnt], hb[lo:lo + cnt] = f["gate"], f["up"], f["h"]
+        out_rows[lo:lo + cnt] = f["out"]
+    y = combine(out_rows, r["topk_w"], r["slot_to_row"])
+    res = dict(r)
+    res.update(gate=gate, up=up, h=hb, out=out_rows, y=y)
+    return res

@@ -149,6 +149,12 @@ MUTANTS = [
     ("router_logits_experts_reversed", rt, "router_logits", "w64 = np.asarray(w_router, dtype=np.float64)",
      "w64 = np.asarray(w_router, dtype=np.float64)[::-1]"),
     ("router_logits_no_float32_rounding", rt, "router_logits", ".astype(np.float32)", ""),
+    # BF16 experts with adapters
+    ("lora_scaling_dropped", moe, "lora_project", "float(scaling) * ", ""),
+    ("lora_b_not_transposed", moe, "lora_project", "np.asarray(lora_b, dtype=np.float64).T",
+     "np.asarray(lora_b, dtype=np.float64)"),
+    ("lora_down_input_not_bf16", moe, "expert_ffn_bf16", "h = fm.bf16_round(swiglu(g, u))", "h = swiglu(g, u)"),
+    ("lora_up_uses_gate_adapter", moe, "expert_ffn_bf16", 'lo.get("up", (None, None))', 'lo.get("gate", (None, None))'),
 ]
 
 

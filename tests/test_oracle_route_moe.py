@@ -340,3 +340,76 @@ def test_degenerate_batches(fmt):
     one = moe.forward(x[2:3], lg[2:3], experts, 3, fmt, s_x, s_h)
     tok = moe.forward_tokens(x[2:3], lg[2:3], experts, 3, fmt, s_x, s_h)
     np.testing.assert_array_equal(one["y"], tok["y"])      # same sums in the same order
+
+
+
+# ---------------------------------------------------------------- BF16 experts with LoRA adapters
+
+def _grid_vals(rng, shape, step, lim):
+    n = int(round(lim / step))
+    return (rng.integers(-n, n + 1, shape) * step).astype(np.float64)
+
+
+def test_lora_project_against_exact_rational_sums():
+    """a W^T + s (a A^T) B^T against sums of fractions, on grid values."""
+    from fractions import Fraction
+    rng = np.random.default_rng(21)
+    a = _grid_vals(rng, (3, 8), 0.25, 2.0)
+    w = _grid_vals(rng, (5, 8), 0.125, 1.0)
+    la = _grid_vals(rng, (2, 8), 0.5, 1.0)
+    lb = _grid_vals(rng, (5, 2), 0.25, 1.0)
+    s = 0.75
+    got = moe.lora_project(a, w, la, lb, s)
+    for i in range(3):
+        for n in range(5):
+            main = sum(Fraction(a[i, kk]) * Fraction(w[n, kk]) for kk in range(8))
+            z = [sum(Fraction(a[i, kk]) * Fraction(la[j, kk]) for kk in range(8)) for j in range(2)]
+            ref = main + Fraction(s) * sum(z[j] * Fraction(lb[n, j]) for j in range(2))
+            assert got[i, n] == float(ref), (i, n)
+
+
+def test_lora_zero_b_is_the_plain_projection():
+    rng = np.random.default_rng(22)
+    a, w = rng.standard_normal((4, 16)), rng.standard_normal((6, 16))
+    la = rng.standard_normal((3, 16))
+    np.testing.assert_array_equal(moe.lora_project(a, w, la, np.zeros((6, 3)), 2.0), a @ w.T)
+    np.testing.assert_array_equal(moe.lora_project(a, w, None, None, 2.0), a @ w.T)
+
+
+def test_lora_rank_one_closed_form():
+    """A = unit row e_i, B = column c: the update adds s * a[:, i] * c."""
+    rng = np.random.default_rng(23)
+    a = _grid_vals(rng, (4, 10), 0.25, 2.0)
+    w = _grid_vals(rng, (7, 10), 0.25, 1.0)
+    c = _grid_vals(rng, (7, 1), 0.5, 2.0)
+    la = np.zeros((1, 10))
+    la[0, 6] = 1.0
+    got = moe.lora_project(a, w, la, c, 0.5)
+    np.testing.assert_array_equal(got, a @ w.T + 0.5 * a[:, 6:7] * c[:, 0][None, :])
+
+
+def test_bf16_layer_with_adapters_equals_merged_weights_written_out():
+    """One expert, k = 1: the layer equals a per-token SwiGLU FFN with the
+    adapters merged into the weights (W + s B A), written out with math.exp
+    and torch's bf16 rounding of the intermediate."""
+    import torch
+    rng = np.random.default_rng(24)
+    T, H, I, r, s = 12, 16, 8, 2, 0.5
+    x = _grid_vals(rng, (T, H), 0.25, 2.0).astype(np.float32)
+    w = {"gate": _grid_vals(rng, (I, H), 0.125, 0.5), "up": _grid_vals(rng, (I, H), 0.125, 0.5),
+         "down": _grid_vals(rng, (H, I), 0.125, 0.5)}
+    lo = {m: (_grid_vals(rng, (r, w[m].shape[1]), 0.25, 0.5), _grid_vals(rng, (w[m].shape[0], r), 0.25, 0.5))
+          for m in w}
+    lg = np.zeros((T, 1), dtype=np.float32)
+    res = moe.forward_bf16(x, lg, {0: w}, {0: lo}, 1, s, 1)
+    merged = {m: w[m] + s * lo[m][1] @ lo[m][0] for m in w}
+    for t in range(T):
+        g = [float(np.dot(x[t].astype(np.float64), merged["gate"][i])) for i in range(I)]
+        u = [float(np.dot(x[t].astype(np.float64), merged["up"][i])) for i in range(I)]
+        h = torch.tensor([gi * ui / (1.0 + math.exp(-gi)) for gi, ui in zip(g, u)], dtype=torch.float64)
+        h = h.to(torch.bfloat16).double().numpy()
+        o = merged["down"] @ h
+        yt = torch.tensor(o, dtype=torch.float64).to(torch.bfloat16).double().numpy()
+        np.testing.assert_allclose(res["gate"][t], g, rtol=1e-14, atol=1e-14)
+        np.testing.assert_allclose(res["y"][t], yt, rtol=2.0 ** -8, atol=1e-30)
+        assert np.mean(res["y"][t] == yt) >= 0.9
