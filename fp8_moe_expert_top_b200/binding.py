@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_NVFP4 = 0
 MOE_MXFP8 = 1
-FORMATS = {"nvfp4": MOE_NVFP4, "mxfp8": MOE_MXFP8}
+MOE_BF16 = 2
+FORMATS = {"nvfp4": MOE_NVFP4, "mxfp8": MOE_MXFP8, "bf16": MOE_BF16}
 
 MOE_DEVICE_TIMEOUT_PRODUCER = 0x1
 MOE_DEVICE_TIMEOUT_MMA = 0x2
@@ -63,7 +64,10 @@ SIGNATURES = {
     "moe_forward": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_forward_gateup": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_forward_down": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
-    "moe_forward_grouped": (ctypes.c_int, [_CFG, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_forward_grouped": (ctypes.c_int, [_CFG, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                           _P]),
+    "moe_pack_weights_bf16": (ctypes.c_int, [_CFG, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I32,
+                                             ctypes.c_float, _P, _P]),
     "moe_unpermute_combine": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P]),
     "moe_route_topk_noalloc": (ctypes.c_int, [_CFG, _I64, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_selftest_bounded_wait": (ctypes.c_int, [_P, _I64, _P]),
@@ -216,11 +220,24 @@ def moe_forward_down(cfg, T, packed, h_codes, h_sf, inter_scale, expert_offsets,
     _check("moe_forward_down", lib().moe_forward_down(ctypes.byref(cfg), int(T), *p, st))
 
 
-def moe_forward_grouped(cfg, num_groups, packed, a_codes, a_sf, act_scale, inter_scale, group_offsets, group_counts,
-                        group_expert, h_codes, h_sf, down_out, gateup_debug=None, status_word=None, stream=None):
+def moe_forward_grouped(cfg, num_groups, max_rows, packed, a_codes, a_sf, act_scale, inter_scale, group_offsets,
+                        group_counts, group_expert, h_codes, h_sf, down_out, gateup_debug=None, status_word=None,
+                        stream=None):
     p, st = _marshal("moe_forward_grouped", stream, packed, a_codes, a_sf, act_scale, inter_scale, group_offsets,
                      group_counts, group_expert, h_codes, h_sf, down_out, gateup_debug, status_word)
-    _check("moe_forward_grouped", lib().moe_forward_grouped(ctypes.byref(cfg), int(num_groups), *p, st))
+    _check("moe_forward_grouped", lib().moe_forward_grouped(ctypes.byref(cfg), int(num_groups), int(max_rows), *p,
+                                                            st))
+
+
+def moe_pack_weights_bf16(cfg, expert_begin, expert_count, w_gate, w_up, w_down, lora=None, lora_rank=0,
+                          lora_scaling=0.0, packed=None, stream=None):
+    """bf16 weights [n, I, H] / [n, H, I] and optional adapters
+    lora = (a_gate, b_gate, a_up, b_up, a_down, b_down) into packed."""
+    lo = lora if lora is not None else (None,) * 6
+    p, st = _marshal("moe_pack_weights_bf16", stream, w_gate, w_up, w_down, *lo, packed)
+    _check("moe_pack_weights_bf16", lib().moe_pack_weights_bf16(
+        ctypes.byref(cfg), int(expert_begin), int(expert_count), *p[:9], int(lora_rank), float(lora_scaling), p[9],
+        st))
 
 
 def moe_unpermute_combine(cfg, T, down_out, topk_w, slot_to_row, y, stream=None):

@@ -14,12 +14,22 @@ constexpr int64_t kMaxTokens = int64_t(1) << 20;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int bits_of(const moe_config* c) { return c->fmt == MOE_NVFP4 ? 4 : 8; }
-int sfvec_of(const moe_config* c) { return c->fmt == MOE_NVFP4 ? 16 : 32; }
+// A block-scale buffer argument: unused (may be NULL) for BF16, required and
+// aligned for the block-scaled formats.
+bool sf_ok(const moe_config* cfg, const void* sf) {
+  return cfg->fmt == MOE_BF16 ? (sf == nullptr || aligned16(sf)) : (sf != nullptr && aligned16(sf));
+}
+
+int bits_of(const moe_config* c) { return c->fmt == MOE_NVFP4 ? 4 : (c->fmt == MOE_MXFP8 ? 8 : 16); }
+int sfvec_of(const moe_config* c) { return c->fmt == MOE_MXFP8 ? 32 : 16; }
+// bytes of one tiled operand row of K elements (BF16: plus the adapter K tile)
+int64_t row_bytes(const moe_config* c, int64_t K) {
+  return c->fmt == MOE_BF16 ? 2 * K + 128 : moe::kb_padded(K, bits_of(c));
+}
 
 moe_status check(const moe_config* c) {
   if (c == nullptr) return MOE_ERR_INVALID_ARG;
-  if (c->fmt != MOE_NVFP4 && c->fmt != MOE_MXFP8) return MOE_ERR_UNSUPPORTED;
+  if (c->fmt != MOE_NVFP4 && c->fmt != MOE_MXFP8 && c->fmt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (c->num_experts < 1 || c->num_experts > 1024) return MOE_ERR_UNSUPPORTED;
   if (c->top_k < 1 || c->top_k > 8 || c->top_k > c->num_experts) return MOE_ERR_UNSUPPORTED;
   if (c->d_model < 256 || c->d_model % 256 != 0) return MOE_ERR_UNSUPPORTED;
@@ -46,14 +56,16 @@ void layout(const moe_config* c, moe_weights_layout* L) {
   const int b = bits_of(c), v = sfvec_of(c);
   auto up256 = [](int64_t x) { return (x + 255) / 256 * 256; };
   int64_t off = 0;
+  const bool bf16 = c->fmt == MOE_BF16;
+  (void)b;
   L->w13_codes = off;
-  off = up256(off + E * 2 * I * moe::kb_padded(H, b));
-  L->w13_sf = off;
-  off = up256(off + E * 2 * I * H / v);
+  off = up256(off + E * 2 * I * row_bytes(c, H));
+  L->w13_sf = off;  // BF16: the adapters' A of gate and up, 64 rows per expert
+  off = up256(off + (bf16 ? E * 64 * 2 * H : E * 2 * I * H / v));
   L->w2_codes = off;
-  off = up256(off + E * H * moe::kb_padded(I, b));
-  L->w2_sf = off;
-  off = up256(off + E * H * I / v);
+  off = up256(off + E * H * row_bytes(c, I));
+  L->w2_sf = off;   // BF16: A of down and 32 zero rows
+  off = up256(off + (bf16 ? E * 64 * 2 * I : E * H * I / v));
   L->scales = off;
   off = up256(off + E * 3 * 4);
   L->total_bytes = off;
@@ -80,11 +92,14 @@ int64_t moe_max_rows(const moe_config* cfg, int64_t T) {
 
 int64_t moe_codes_bytes(const moe_config* cfg, int64_t rows, int64_t K) {
   if (check(cfg) != MOE_OK || rows < 0 || K <= 0 || rows % 128 != 0) return -1;
-  return rows * moe::kb_padded(K, bits_of(cfg));
+  if (cfg->fmt == MOE_BF16 && K % 64 != 0) return -1;
+  return rows * row_bytes(cfg, K);
 }
 
 int64_t moe_sf_bytes(const moe_config* cfg, int64_t rows, int64_t K) {
-  if (check(cfg) != MOE_OK || rows < 0 || K <= 0 || rows % 128 != 0 || K % (4 * sfvec_of(cfg)) != 0) return -1;
+  if (check(cfg) != MOE_OK || rows < 0 || K <= 0 || rows % 128 != 0) return -1;
+  if (cfg->fmt == MOE_BF16) return 0;  // no block scales
+  if (K % (4 * sfvec_of(cfg)) != 0) return -1;
   return rows * K / sfvec_of(cfg);
 }
 
@@ -95,11 +110,42 @@ int64_t moe_route_workspace_bytes(const moe_config* cfg, int64_t T) {
   return moe::route_workspace_bytes(cfg->num_experts, T);
 }
 
+moe_status moe_pack_weights_bf16(const moe_config* cfg, int32_t expert_begin, int32_t expert_count,
+                                 const void* w_gate, const void* w_up, const void* w_down, const void* lora_a_gate,
+                                 const void* lora_b_gate, const void* lora_a_up, const void* lora_b_up,
+                                 const void* lora_a_down, const void* lora_b_down, int32_t lora_rank,
+                                 float lora_scaling, void* packed, void* stream) {
+  moe_status s = check(cfg);
+  if (s != MOE_OK) return s;
+  if (cfg->fmt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (expert_begin < 0 || expert_count < 0 || expert_begin + expert_count > cfg->num_experts)
+    return MOE_ERR_INVALID_ARG;
+  if (expert_count == 0) return MOE_OK;
+  if (!w_gate || !w_up || !w_down || !packed) return MOE_ERR_INVALID_ARG;
+  const void* lora[6] = {lora_a_gate, lora_b_gate, lora_a_up, lora_b_up, lora_a_down, lora_b_down};
+  int given = 0;
+  for (const void* p : lora) given += p != nullptr;
+  if (given != 0 && given != 6) return MOE_ERR_INVALID_ARG;  // all six adapter matrices, or none
+  if (given == 6 && (lora_rank < 1 || lora_rank > 32)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(packed)) return MOE_ERR_INVALID_ARG;
+  if (given == 6 && (!aligned16(lora_a_gate) || !aligned16(lora_a_up) || !aligned16(lora_a_down)))
+    return MOE_ERR_INVALID_ARG;
+  moe_weights_layout L;
+  layout(cfg, &L);
+  uint8_t* base = static_cast<uint8_t*>(packed);
+  return from_cuda(moe::launch_pack_bf16(
+      cfg->d_model, cfg->d_ffn, expert_begin, expert_count, w_gate, w_up, w_down, lora_a_gate, lora_a_up,
+      lora_a_down, lora_b_gate, lora_b_up, lora_b_down, given == 6 ? lora_rank : 0, lora_scaling, base + L.w13_codes,
+      base + L.w13_sf, base + L.w2_codes, base + L.w2_sf, reinterpret_cast<float*>(base + L.scales),
+      static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_quantize_weights(const moe_config* cfg, int32_t expert_begin, int32_t expert_count,
                                 const float* w_gate, const float* w_up, const float* w_down, void* packed,
                                 void* stream) {
   moe_status s = check(cfg);
   if (s != MOE_OK) return s;
+  if (cfg->fmt == MOE_BF16) return MOE_ERR_UNSUPPORTED;  // moe_pack_weights_bf16
   if (expert_begin < 0 || expert_count < 0 || expert_begin + expert_count > cfg->num_experts)
     return MOE_ERR_INVALID_ARG;
   if (expert_count == 0) return MOE_OK;
@@ -162,9 +208,9 @@ moe_status moe_permute(const moe_config* cfg, int64_t T, const void* x_bf16, con
   if (s != MOE_OK) return s;
   if ((s = check_T(T)) != MOE_OK) return s;
   if (T == 0) return MOE_OK;
-  if (!x_bf16 || !slot_to_row || !a_codes || !a_sf) return MOE_ERR_INVALID_ARG;
+  if (!x_bf16 || !slot_to_row || !a_codes) return MOE_ERR_INVALID_ARG;
   if (cfg->fmt == MOE_NVFP4 && !act_scale) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x_bf16) || !aligned16(a_codes) || !aligned16(a_sf)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(a_codes) || !sf_ok(cfg, a_sf)) return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_permute(cfg->fmt, static_cast<int>(T), cfg->d_model, cfg->top_k, x_bf16, act_scale,
                                        slot_to_row, static_cast<uint8_t*>(a_codes), static_cast<uint8_t*>(a_sf),
                                        static_cast<cudaStream_t>(stream)));
@@ -180,6 +226,89 @@ static moe_status gemm_common(const moe_config* cfg, int64_t T, const void* pack
   return MOE_OK;
 }
 
+// Row groups of the expert GEMMs: experts (group_expert null) or segments
+// naming the expert whose weights they use.
+struct Groups {
+  int n;
+  const int32_t* offsets;
+  const int32_t* counts;
+  const int32_t* expert;
+  int64_t R_max;  // rows the buffers hold (bounds the adapter shrink's grid)
+};
+
+// gate/up GEMM + SwiGLU + h in the layer format.  BF16: the adapter shrink
+// of A first (into A's adapter K tile), the GEMM over d_model + 64, then the
+// shrink of h (into h's adapter K tile) for the down GEMM.
+static moe_status run_gateup(const moe_config* cfg, const Groups& G, const uint8_t* base, const void* a_codes,
+                             const void* a_sf, const float* act_scale, const float* inter_scale, void* h_codes,
+                             void* h_sf, float* dbg, uint32_t* status, cudaStream_t st) {
+  moe_weights_layout L;
+  layout(cfg, &L);
+  const bool bf16 = cfg->fmt == MOE_BF16;
+  const float* scales = reinterpret_cast<const float*>(base + L.scales);
+  if (bf16) {
+    const cudaError_t err = moe::launch_lora_shrink(
+        static_cast<uint8_t*>(const_cast<void*>(a_codes)), 2 * int64_t(cfg->d_model) + 128, cfg->d_model,
+        base + L.w13_sf, scales, G.offsets, G.counts, G.expert, cfg->num_experts, G.n, G.R_max, status, st);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  moe::GemmLaunch g{};
+  g.fmt = cfg->fmt;
+  g.gateup = true;
+  g.E = G.n;
+  g.K = cfg->d_model + (bf16 ? 64 : 0);
+  g.n_rows_b = 2 * cfg->d_ffn;
+  g.a_codes = static_cast<const uint8_t*>(a_codes);
+  g.a_sf = static_cast<const uint8_t*>(a_sf);
+  g.b_codes = base + L.w13_codes;
+  g.b_sf = base + L.w13_sf;
+  g.offsets = G.offsets;
+  g.counts = G.counts;
+  g.expert_map = G.expert;
+  g.n_weights = cfg->num_experts;
+  g.a_scale = act_scale;
+  g.w_scales = scales;
+  g.h_scale = inter_scale;
+  g.h_codes = static_cast<uint8_t*>(h_codes);
+  g.h_sf = static_cast<uint8_t*>(h_sf);
+  g.dbg = dbg;
+  g.status = status;
+  if (moe::launch_gemm(g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (bf16) {
+    return from_cuda(moe::launch_lora_shrink(static_cast<uint8_t*>(h_codes), 2 * int64_t(cfg->d_ffn) + 128,
+                                             cfg->d_ffn, base + L.w2_sf, scales, G.offsets, G.counts, G.expert,
+                                             cfg->num_experts, G.n, G.R_max, status, st));
+  }
+  return MOE_OK;
+}
+
+// down GEMM -> bf16 rows (BF16: over d_ffn + 64, the adapter tile of h).
+static moe_status run_down(const moe_config* cfg, const Groups& G, const uint8_t* base, const void* h_codes,
+                           const void* h_sf, const float* inter_scale, void* down_out, uint32_t* status,
+                           cudaStream_t st) {
+  moe_weights_layout L;
+  layout(cfg, &L);
+  moe::GemmLaunch g{};
+  g.fmt = cfg->fmt;
+  g.gateup = false;
+  g.E = G.n;
+  g.K = cfg->d_ffn + (cfg->fmt == MOE_BF16 ? 64 : 0);
+  g.n_rows_b = cfg->d_model;
+  g.a_codes = static_cast<const uint8_t*>(h_codes);
+  g.a_sf = static_cast<const uint8_t*>(h_sf);
+  g.b_codes = base + L.w2_codes;
+  g.b_sf = base + L.w2_sf;
+  g.offsets = G.offsets;
+  g.counts = G.counts;
+  g.expert_map = G.expert;
+  g.n_weights = cfg->num_experts;
+  g.a_scale = inter_scale;
+  g.w_scales = reinterpret_cast<const float*>(base + L.scales);
+  g.out = down_out;
+  g.status = status;
+  return from_cuda(moe::launch_gemm(g, st));
+}
+
 moe_status moe_forward_gateup(const moe_config* cfg, int64_t T, const void* packed, const void* a_codes,
                               const void* a_sf, const float* act_scale, const float* inter_scale,
                               const int32_t* expert_offsets, const int32_t* expert_counts, void* h_codes,
@@ -187,35 +316,13 @@ moe_status moe_forward_gateup(const moe_config* cfg, int64_t T, const void* pack
   moe_status s = gemm_common(cfg, T, packed, expert_offsets, expert_counts);
   if (s != MOE_OK) return s;
   if (T == 0) return MOE_OK;
-  if (!a_codes || !a_sf || !h_codes || !h_sf) return MOE_ERR_INVALID_ARG;
+  if (!a_codes || !h_codes || !aligned16(a_codes) || !aligned16(h_codes)) return MOE_ERR_INVALID_ARG;
+  if (!sf_ok(cfg, a_sf) || !sf_ok(cfg, h_sf)) return MOE_ERR_INVALID_ARG;
   if (cfg->fmt == MOE_NVFP4 && (!act_scale || !inter_scale)) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(h_codes) || !aligned16(h_sf)) return MOE_ERR_INVALID_ARG;
   if (gateup_debug && !aligned16(gateup_debug)) return MOE_ERR_INVALID_ARG;
-  moe_weights_layout L;
-  layout(cfg, &L);
-  const uint8_t* base = static_cast<const uint8_t*>(packed);
-  moe::GemmLaunch g{};
-  g.fmt = cfg->fmt;
-  g.gateup = true;
-  g.E = cfg->num_experts;
-  g.K = cfg->d_model;
-  g.n_rows_b = 2 * cfg->d_ffn;
-  g.R_max = max_rows(cfg, T);
-  g.a_codes = static_cast<const uint8_t*>(a_codes);
-  g.a_sf = static_cast<const uint8_t*>(a_sf);
-  g.b_codes = base + L.w13_codes;
-  g.b_sf = base + L.w13_sf;
-  g.offsets = expert_offsets;
-  g.counts = expert_counts;
-  g.a_scale = act_scale;
-  g.w_scales = reinterpret_cast<const float*>(base + L.scales);
-  g.h_scale = inter_scale;
-  g.h_codes = static_cast<uint8_t*>(h_codes);
-  g.h_sf = static_cast<uint8_t*>(h_sf);
-  g.dbg = gateup_debug;
-  g.out = nullptr;
-  g.status = status_word;
-  return from_cuda(moe::launch_gemm(g, static_cast<cudaStream_t>(stream)));
+  const Groups G{cfg->num_experts, expert_offsets, expert_counts, nullptr, max_rows(cfg, T)};
+  return run_gateup(cfg, G, static_cast<const uint8_t*>(packed), a_codes, a_sf, act_scale, inter_scale, h_codes,
+                    h_sf, gateup_debug, status_word, static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_forward_down(const moe_config* cfg, int64_t T, const void* packed, const void* h_codes,
@@ -224,31 +331,12 @@ moe_status moe_forward_down(const moe_config* cfg, int64_t T, const void* packed
   moe_status s = gemm_common(cfg, T, packed, expert_offsets, expert_counts);
   if (s != MOE_OK) return s;
   if (T == 0) return MOE_OK;
-  if (!h_codes || !h_sf || !down_out) return MOE_ERR_INVALID_ARG;
+  if (!h_codes || !down_out || !aligned16(h_codes) || !aligned16(down_out)) return MOE_ERR_INVALID_ARG;
+  if (!sf_ok(cfg, h_sf)) return MOE_ERR_INVALID_ARG;
   if (cfg->fmt == MOE_NVFP4 && !inter_scale) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(h_codes) || !aligned16(h_sf) || !aligned16(down_out)) return MOE_ERR_INVALID_ARG;
-  moe_weights_layout L;
-  layout(cfg, &L);
-  const uint8_t* base = static_cast<const uint8_t*>(packed);
-  moe::GemmLaunch g{};
-  g.fmt = cfg->fmt;
-  g.gateup = false;
-  g.E = cfg->num_experts;
-  g.K = cfg->d_ffn;
-  g.n_rows_b = cfg->d_model;
-  g.R_max = max_rows(cfg, T);
-  g.a_codes = static_cast<const uint8_t*>(h_codes);
-  g.a_sf = static_cast<const uint8_t*>(h_sf);
-  g.b_codes = base + L.w2_codes;
-  g.b_sf = base + L.w2_sf;
-  g.offsets = expert_offsets;
-  g.counts = expert_counts;
-  g.a_scale = inter_scale;
-  g.w_scales = reinterpret_cast<const float*>(base + L.scales);
-  g.h_scale = nullptr;
-  g.out = down_out;
-  g.status = status_word;
-  return from_cuda(moe::launch_gemm(g, static_cast<cudaStream_t>(stream)));
+  const Groups G{cfg->num_experts, expert_offsets, expert_counts, nullptr, max_rows(cfg, T)};
+  return run_down(cfg, G, static_cast<const uint8_t*>(packed), h_codes, h_sf, inter_scale, down_out, status_word,
+                  static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_forward(const moe_config* cfg, int64_t T, const void* packed, const void* a_codes,
@@ -262,65 +350,28 @@ moe_status moe_forward(const moe_config* cfg, int64_t T, const void* packed, con
                           status_word, stream);
 }
 
-moe_status moe_forward_grouped(const moe_config* cfg, int32_t num_groups, const void* packed, const void* a_codes,
-                               const void* a_sf, const float* act_scale, const float* inter_scale,
-                               const int32_t* group_offsets, const int32_t* group_counts,
+moe_status moe_forward_grouped(const moe_config* cfg, int32_t num_groups, int64_t max_rows_, const void* packed,
+                               const void* a_codes, const void* a_sf, const float* act_scale,
+                               const float* inter_scale, const int32_t* group_offsets, const int32_t* group_counts,
                                const int32_t* group_expert, void* h_codes, void* h_sf, void* down_out,
                                float* gateup_debug, uint32_t* status_word, void* stream) {
   moe_status s = check(cfg);
   if (s != MOE_OK) return s;
   if (num_groups < 0 || num_groups > 1024) return MOE_ERR_UNSUPPORTED;
-  if (num_groups == 0) return MOE_OK;
-  if (!packed || !a_codes || !a_sf || !group_offsets || !group_counts || !group_expert || !h_codes || !h_sf ||
-      !down_out)
+  if (max_rows_ < 0 || max_rows_ % 128 != 0) return MOE_ERR_INVALID_ARG;
+  if (num_groups == 0 || max_rows_ == 0) return MOE_OK;
+  if (!packed || !a_codes || !group_offsets || !group_counts || !group_expert || !h_codes || !down_out)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(a_codes) || !aligned16(h_codes) || !aligned16(down_out) ||
+      (gateup_debug && !aligned16(gateup_debug)) || !sf_ok(cfg, a_sf) || !sf_ok(cfg, h_sf))
     return MOE_ERR_INVALID_ARG;
   if (cfg->fmt == MOE_NVFP4 && (!act_scale || !inter_scale)) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(packed) || !aligned16(a_codes) || !aligned16(a_sf) || !aligned16(h_codes) || !aligned16(h_sf) ||
-      !aligned16(down_out) || (gateup_debug && !aligned16(gateup_debug)))
-    return MOE_ERR_INVALID_ARG;
-  moe_weights_layout L;
-  layout(cfg, &L);
   const uint8_t* base = static_cast<const uint8_t*>(packed);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  moe::GemmLaunch g{};
-  g.fmt = cfg->fmt;
-  g.E = num_groups;
-  g.offsets = group_offsets;
-  g.counts = group_counts;
-  g.expert_map = group_expert;
-  g.n_weights = cfg->num_experts;
-  g.w_scales = reinterpret_cast<const float*>(base + L.scales);
-  g.status = status_word;
-  // gate/up + SwiGLU + requantized h
-  g.gateup = true;
-  g.K = cfg->d_model;
-  g.n_rows_b = 2 * cfg->d_ffn;
-  g.a_codes = static_cast<const uint8_t*>(a_codes);
-  g.a_sf = static_cast<const uint8_t*>(a_sf);
-  g.b_codes = base + L.w13_codes;
-  g.b_sf = base + L.w13_sf;
-  g.a_scale = act_scale;
-  g.h_scale = inter_scale;
-  g.h_codes = static_cast<uint8_t*>(h_codes);
-  g.h_sf = static_cast<uint8_t*>(h_sf);
-  g.dbg = gateup_debug;
-  cudaError_t err = moe::launch_gemm(g, st);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
-  // down
-  g.gateup = false;
-  g.K = cfg->d_ffn;
-  g.n_rows_b = cfg->d_model;
-  g.a_codes = static_cast<const uint8_t*>(h_codes);
-  g.a_sf = static_cast<const uint8_t*>(h_sf);
-  g.b_codes = base + L.w2_codes;
-  g.b_sf = base + L.w2_sf;
-  g.a_scale = inter_scale;
-  g.h_scale = nullptr;
-  g.h_codes = nullptr;
-  g.h_sf = nullptr;
-  g.dbg = nullptr;
-  g.out = down_out;
-  return from_cuda(moe::launch_gemm(g, st));
+  const Groups G{num_groups, group_offsets, group_counts, group_expert, max_rows_};
+  s = run_gateup(cfg, G, base, a_codes, a_sf, act_scale, inter_scale, h_codes, h_sf, gateup_debug, status_word, st);
+  if (s != MOE_OK) return s;
+  return run_down(cfg, G, base, h_codes, h_sf, inter_scale, down_out, status_word, st);
 }
 
 moe_status moe_unpermute_combine(const moe_config* cfg, int64_t T, const void* down_out, const float* topk_w,

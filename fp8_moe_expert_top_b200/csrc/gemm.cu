@@ -178,17 +178,19 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
             break;
           }
           const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
-          const uint32_t sf_bytes = (FMT == MOE_NVFP4) ? 512u * kb_here : 512u;
+          const uint32_t sf_bytes = !Tr::kScaled ? 0u : ((FMT == MOE_NVFP4) ? 512u * kb_here : 512u);
           uint8_t* st = smem + stage * Tr::kStageBytes;
           mbar_arrive_expect_tx(&full_bar[stage], a_bytes + Tr::kBBytes + sf_bytes * (1 + kBN / 128));
           bulk_load(st, a_tiles + static_cast<int64_t>(kt) * Tr::kABytes, a_bytes, &full_bar[stage], pol_a);
           bulk_load(st + Tr::kABytes, b_tiles + static_cast<int64_t>(kt) * Tr::kBBytes, Tr::kBBytes, &full_bar[stage],
                     pol_w);
-          bulk_load(st + Tr::kSfaOff, a_sf + kt * Tr::kSfBytes128, sf_bytes, &full_bar[stage], pol_a);
+          if (Tr::kScaled) {
+            bulk_load(st + Tr::kSfaOff, a_sf + kt * Tr::kSfBytes128, sf_bytes, &full_bar[stage], pol_a);
 #pragma unroll
-          for (int h = 0; h < kBN / 128; ++h)
-            bulk_load(st + Tr::kSfbOff + h * Tr::kSfBytes128, b_sf + h * args.sf_rb_stride + kt * Tr::kSfBytes128,
-                      sf_bytes, &full_bar[stage], pol_w);
+            for (int h = 0; h < kBN / 128; ++h)
+              bulk_load(st + Tr::kSfbOff + h * Tr::kSfBytes128, b_sf + h * args.sf_rb_stride + kt * Tr::kSfBytes128,
+                        sf_bytes, &full_bar[stage], pol_w);
+          }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -214,7 +216,8 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
         for (int kt = 0; kt < k_tiles; ++kt) {
           // the scale copiers have seen the stage's operands land and their
           // copies have completed (the operand wait then returns at once)
-          if (!mbar_wait(&sf_bar[stage], phase, abort_flag) || !mbar_wait(&full_bar[stage], phase, abort_flag)) {
+          if ((Tr::kScaled && !mbar_wait(&sf_bar[stage], phase, abort_flag)) ||
+              !mbar_wait(&full_bar[stage], phase, abort_flag)) {
             fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
             ok = false;
             break;
@@ -226,7 +229,10 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
           const uint64_t bdesc = make_desc_sw128(st + Tr::kABytes);
           const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kSfColsPerStage<FMT>;
           const uint32_t sfb = sfa + Tr::kSfaCols;
-          if (FMT == MOE_NVFP4) {
+          if (FMT == MOE_BF16) {
+            for (int kb = 0; kb < kb_here; ++kb)
+              tc_mma_bf16(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_bf16(kBN), (kt | kb) != 0 ? 1u : 0u);
+          } else if (FMT == MOE_NVFP4) {
             for (int kb = 0; kb < kb_here; ++kb) {
               tc_mma_nvfp4(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_nvfp4(kBN), sfa + 4 * kb,
                            sfb + (kBN / 32) * kb, (kt | kb) != 0 ? 1u : 0u);
@@ -252,7 +258,7 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
   } else if (warp >= kThreads / 32) {
     // ------------------------------------------------------------ scale copiers
     const int part = warp - kThreads / 32;  // copies the scales of k blocks part, part + kCopierWarps, ...
-    if (lane == 0) {
+    if (lane == 0 && Tr::kScaled) {
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
@@ -391,19 +397,21 @@ static cudaError_t launch_one(const GemmArgs& a, cudaStream_t stream) {
 
 size_t gemm_smem_bytes(int fmt, int E) {
   const int sb = (fmt == MOE_NVFP4) ? GemmTraits<MOE_NVFP4, kBN, kStages>::kStageBytes
-                                    : GemmTraits<MOE_MXFP8, kBN, kStages>::kStageBytes;
+                 : (fmt == MOE_MXFP8) ? GemmTraits<MOE_MXFP8, kBN, kStages>::kStageBytes
+                                      : GemmTraits<MOE_BF16, kBN, kStages>::kStageBytes;
   return 1024 + kStages * sb + (3 * kStages + 3) * 8 + 16 + (E + 1) * 4;
 }
 
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
-  const int bits = (g.fmt == MOE_NVFP4) ? 4 : 8;
-  const int sfvec = (g.fmt == MOE_NVFP4) ? 16 : 32;
+  const int bits = (g.fmt == MOE_NVFP4) ? 4 : (g.fmt == MOE_MXFP8 ? 8 : 16);
+  const int sfvec = (g.fmt == MOE_MXFP8) ? 32 : 16;
   GemmArgs a;
   a.a_codes = g.a_codes;
   a.b_codes = g.b_codes;
   a.kb = kb_padded(g.K, bits);
   a.b_expert_stride = static_cast<int64_t>(g.n_rows_b) * a.kb;
-  a.h_kb = g.gateup ? kb_padded(g.n_rows_b / 2, bits) : 0;
+  // BF16: h carries the adapter K tile after its d_ffn channels
+  a.h_kb = g.gateup ? kb_padded(g.n_rows_b / 2 + (g.fmt == MOE_BF16 ? 64 : 0), bits) : 0;
   a.a_sf = g.a_sf;
   a.b_sf = g.b_sf;
   a.offsets = g.offsets;
@@ -425,6 +433,8 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
   a.b_sf_expert_stride = static_cast<int64_t>(g.n_rows_b) * (g.K / sfvec);
   if (g.fmt == MOE_NVFP4)
     return g.gateup ? launch_one<MOE_NVFP4, true>(a, stream) : launch_one<MOE_NVFP4, false>(a, stream);
+  if (g.fmt == MOE_BF16)
+    return g.gateup ? launch_one<MOE_BF16, true>(a, stream) : launch_one<MOE_BF16, false>(a, stream);
   return g.gateup ? launch_one<MOE_MXFP8, true>(a, stream) : launch_one<MOE_MXFP8, false>(a, stream);
 }
 

@@ -21,13 +21,14 @@ constexpr uint32_t kTmemCols = 512;
 // B_ROWS: weight rows a CTA loads per stage.
 template <int FMT, int B_ROWS, int STAGES>
 struct GemmTraits {
+  static constexpr bool kScaled = FMT != MOE_BF16;  // block-scaled formats carry scale atoms
   static constexpr int kStages = STAGES;
-  static constexpr int kElemsPerStage = (FMT == MOE_NVFP4) ? 256 : 128;
-  static constexpr int kMmaK = (FMT == MOE_NVFP4) ? 64 : 32;
+  static constexpr int kElemsPerStage = (FMT == MOE_NVFP4) ? 256 : (FMT == MOE_MXFP8 ? 128 : 64);
+  static constexpr int kMmaK = (FMT == MOE_NVFP4) ? 64 : (FMT == MOE_MXFP8 ? 32 : 16);
   static constexpr int kSfVec = (FMT == MOE_NVFP4) ? 16 : 32;
   // scale bytes of 128 rows for one stage: NVFP4 16 scales/row = 4 atoms,
-  // MXFP8 4 scales/row = 1 atom
-  static constexpr int kSfBytes128 = 128 * (kElemsPerStage / kSfVec);
+  // MXFP8 4 scales/row = 1 atom, BF16 none
+  static constexpr int kSfBytes128 = kScaled ? 128 * (kElemsPerStage / kSfVec) : 0;
   static constexpr int kABytes = kBM * kRowBytesPerStage;
   static constexpr int kBBytes = B_ROWS * kRowBytesPerStage;
   static constexpr int kSfaOff = kABytes + kBBytes;
@@ -88,7 +89,37 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, float* acc, 
                                               int half) {
   const int I = args.n_rows_b / 2;  // gate/up: channels
   const int H = args.n_rows_b;      // down: output channels
-  if (GATEUP) {
+  if (GATEUP && FMT == MOE_BF16) {
+    // columns of this half: [gate 32 | up 32] x 2, channels ch0 + [0, 64);
+    // h in bf16 fills one 128-byte row of h's K tile ch0 / 64
+    const int ch0 = nt * (kBN / 2) + half * (kBN / 4);
+    uint32_t p[32];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float* g = acc + 64 * j;
+      float* u = acc + 64 * j + 32;
+      if (args.dbg != nullptr) {
+        float4* dg = reinterpret_cast<float4*>(args.dbg + row * (2 * I) + ch0 + 32 * j);
+        float4* du = reinterpret_cast<float4*>(args.dbg + row * (2 * I) + I + ch0 + 32 * j);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          dg[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
+          du[i] = make_float4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float h0 = __fdividef(g[2 * i] * u[2 * i], 1.0f + __expf(-g[2 * i]));
+        const float h1 = __fdividef(g[2 * i + 1] * u[2 * i + 1], 1.0f + __expf(-g[2 * i + 1]));
+        const __nv_bfloat162 b = __floats2bfloat162_rn(h0, h1);
+        p[16 * j + i] = *reinterpret_cast<const uint32_t*>(&b);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      *reinterpret_cast<uint4*>(args.h_codes + tile_offset(row, 2 * ch0 + 16 * c, args.h_kb, kActTileRows)) =
+          make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
+  } else if (GATEUP) {
     // columns of this half: [gate 32 | up 32] x 2, channels ch0 + [0, 64)
     const int ch0 = nt * (kBN / 2) + half * (kBN / 4);
     const float sa = (FMT == MOE_NVFP4) ? __ldg(args.a_scale) : 1.0f;
@@ -150,6 +181,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, float* acc, 
     }
   } else {
     const float s = (FMT == MOE_NVFP4) ? __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scales + 3 * e + 2)) : 1.0f;
+    (void)I;
     uint4* dst = reinterpret_cast<uint4*>(args.out + row * H + nt * kBN + half * (kBN / 2));
 #pragma unroll
     for (int i = 0; i < kBN / 16; ++i) {

@@ -38,6 +38,19 @@ cudaError_t launch_quantize_weights(int fmt, int E, int H, int I, int expert_beg
                                     uint8_t* w13_sf, uint8_t* w2_codes, uint8_t* w2_sf, float* scales,
                                     cudaStream_t stream);
 
+// BF16 experts: bf16 weights and adapters into the tiled layout (see the
+// header's MOE_BF16 layout), and the adapter shrink z = s_e (a A_e^T) of the
+// rows of a tiled bf16 operand (kb bytes per row, K elements plus the adapter
+// tile), written into that tile.
+cudaError_t launch_pack_bf16(int H, int I, int expert_begin, int expert_count, const void* w_gate, const void* w_up,
+                             const void* w_down, const void* a_gate, const void* a_up, const void* a_down,
+                             const void* b_gate, const void* b_up, const void* b_down, int rank, float scaling,
+                             uint8_t* w13, uint8_t* s13, uint8_t* w2, uint8_t* s2, float* scales,
+                             cudaStream_t stream);
+cudaError_t launch_lora_shrink(uint8_t* a, int64_t kb, int K, const uint8_t* w, const float* scales,
+                               const int32_t* offsets, const int32_t* counts, const int32_t* expert_map,
+                               int n_weights, int E, int64_t R_max, uint32_t* status, cudaStream_t stream);
+
 struct GemmLaunch {
   int fmt;
   bool gateup;

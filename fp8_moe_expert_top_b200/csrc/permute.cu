@@ -96,9 +96,37 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
   }
 }
 
+// BF16 experts: no quantization; one thread per (token, 16 bytes of x) copies
+// them into each of the token's k rows (tiled, with the adapter K tile after
+// the d_model elements left to the adapter shrink).
+__global__ void __launch_bounds__(256) permute_bf16_kernel(int T, int H, int k, const uint4* __restrict__ x,
+                                                           const int32_t* __restrict__ slot_to_row,
+                                                           uint8_t* __restrict__ a_codes) {
+  const int chunks = H / 8;
+  const int64_t id = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  if (id >= static_cast<int64_t>(T) * chunks) return;
+  const int t = static_cast<int>(id / chunks);
+  const int c = static_cast<int>(id % chunks);
+  const uint4 v = __ldg(x + id);
+  const int64_t kb = 2 * static_cast<int64_t>(H) + 128;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j >= k) break;
+    const int64_t r = __ldg(slot_to_row + static_cast<int64_t>(t) * k + j);
+    *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 16 * static_cast<int64_t>(c), kb, kActTileRows)) = v;
+  }
+}
+
 cudaError_t launch_permute(int fmt, int T, int H, int k, const void* x, const float* act_scale,
                            const int32_t* slot_to_row, uint8_t* a_codes, uint8_t* a_sf, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
+  if (fmt == MOE_BF16) {
+    const int64_t n = static_cast<int64_t>(T) * (H / 8);
+    return launch_pdl(permute_bf16_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, stream, T, H,
+                      k, static_cast<const uint4*>(x), slot_to_row, a_codes);
+  }
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   const dim3 block(256);
   // small batches (fewer 32-element groups than 256 per SM): one 16-element

@@ -9,7 +9,9 @@
 // Four steps on the stream: zero the amax slots, reduce amax per matrix
 // (atomicMax on the float bits, exact and order-independent for values >= 0),
 // quantize every 64-element group, turn amax into the tensor scale.
+#include <algorithm>
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -173,6 +175,143 @@ cudaError_t launch_quantize_weights(int fmt, int E, int H, int I, int expert_beg
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   weight_scale_finalize_kernel<<<(3 * expert_count + 255) / 256, 256, 0, stream>>>(3 * expert_count, fmt, sc);
+  return cudaGetLastError();
+}
+
+
+
+// ---------------------------------------------------------------------------
+// BF16 experts with LoRA adapters (pages "thinkingmachines/Inkling-2-Small",
+// section Configurations, and "Thinking Machines releases Inkling 2 Small
+// weights under Apache 2.0", section "LoRA and reinforcement learning":
+// expert adapters need BF16 expert weights).  The bf16 weights are copied
+// into the tiled layout with one extra 64-element K tile per row holding the
+// adapter's B (gate rows: B_gate then zeros; up rows: zeros then B_up; down
+// rows: B_down then zeros); the A matrices (gate and up stacked, down and
+// zero rows) go to their own 64-row tiles.  Ranks below 32 are zero-padded.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct PackBf16Args {
+  const __nv_bfloat16 *wg, *wu, *wd;  // [n][I][H], [n][I][H], [n][H][I]
+  const __nv_bfloat16 *ag, *au, *ad;  // [n][r][H], [n][r][H], [n][r][I]; null: no adapters
+  const __nv_bfloat16 *bg, *bu, *bd;  // [n][I][r], [n][I][r], [n][H][r]
+  uint8_t *w13, *s13, *w2, *s2;       // outputs, already offset to the slice's first expert
+  int H, I, r;
+};
+
+// Eight bf16 of row `row` of a [rows][r] adapter B matrix, elements j0 .. j0+7
+// (zero past the rank).
+__device__ __forceinline__ uint4 load_b8(const __nv_bfloat16* b, int64_t row, int r, int j0) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int j = j0 + 2 * i;
+    const uint16_t lo = (j < r) ? __bfloat16_as_ushort(b[row * r + j]) : 0;
+    const uint16_t hi = (j + 1 < r) ? __bfloat16_as_ushort(b[row * r + j + 1]) : 0;
+    w[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// blockIdx.y: 0 = w13 rows, 1 = w2 rows, 2 = A of gate / up, 3 = A of down;
+// blockIdx.z = expert in the slice; one thread per 16-byte chunk of a row.
+__global__ void __launch_bounds__(256) pack_bf16_kernel(const PackBf16Args a) {
+  const int part = blockIdx.y, e = blockIdx.z;
+  const int H = a.H, I = a.I, r = a.r;
+  int rows, K, TR;
+  int64_t kb;
+  uint8_t* out;
+  if (part == 0) {
+    rows = 2 * I; K = H; kb = 2 * static_cast<int64_t>(H) + 128; TR = kWeightTileRows;
+    out = a.w13 + static_cast<int64_t>(e) * rows * kb;
+  } else if (part == 1) {
+    rows = H; K = I; kb = 2 * static_cast<int64_t>(I) + 128; TR = kWeightTileRows;
+    out = a.w2 + static_cast<int64_t>(e) * rows * kb;
+  } else if (part == 2) {
+    rows = 64; K = H; kb = 2 * static_cast<int64_t>(H); TR = 64;
+    out = a.s13 + static_cast<int64_t>(e) * rows * kb;
+  } else {
+    rows = 64; K = I; kb = 2 * static_cast<int64_t>(I); TR = 64;
+    out = a.s2 + static_cast<int64_t>(e) * rows * kb;
+  }
+  const int64_t chunks = kb / 16;
+  const int64_t id = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (id >= rows * chunks) return;
+  const int row = static_cast<int>(id / chunks);
+  const int j0 = static_cast<int>(id % chunks) * 8;  // first element of the chunk
+  const bool lora = a.ag != nullptr;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (part == 0) {
+    const bool up = (row & 63) >= 32;
+    const int64_t ch = 32 * (row / 64) + (row & 31);
+    const __nv_bfloat16* w = (up ? a.wu : a.wg) + static_cast<int64_t>(e) * I * H;
+    if (j0 < K) {
+      v = __ldg(reinterpret_cast<const uint4*>(w + ch * H + j0));
+    } else if (lora) {
+      const int jj = j0 - K;  // 0 .. 63: gate B in 0..31, up B in 32..63
+      if (!up && jj < 32) v = load_b8(a.bg + static_cast<int64_t>(e) * I * r, ch, r, jj);
+      if (up && jj >= 32) v = load_b8(a.bu + static_cast<int64_t>(e) * I * r, ch, r, jj - 32);
+    }
+  } else if (part == 1) {
+    const __nv_bfloat16* w = a.wd + static_cast<int64_t>(e) * H * I;
+    if (j0 < K) {
+      v = __ldg(reinterpret_cast<const uint4*>(w + static_cast<int64_t>(row) * I + j0));
+    } else if (lora && j0 - K < 32) {
+      v = load_b8(a.bd + static_cast<int64_t>(e) * H * r, row, r, j0 - K);
+    }
+  } else if (lora) {
+    const __nv_bfloat16* m = nullptr;
+    int ar = row;
+    if (part == 2) {
+      m = (row < 32) ? a.ag : a.au;
+      ar = row & 31;
+    } else if (row < 32) {
+      m = a.ad;
+    }
+    if (m != nullptr && ar < r)
+      v = __ldg(reinterpret_cast<const uint4*>(m + (static_cast<int64_t>(e) * r + ar) * K + j0));
+  }
+  *reinterpret_cast<uint4*>(out + tile_offset(row, 2 * static_cast<int64_t>(j0), kb, TR)) = v;
+}
+
+__global__ void bf16_scales_kernel(int n, float scaling, float* __restrict__ scales) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < 3 * n) scales[i] = (i % 3 == 0) ? scaling : 0.0f;
+}
+
+}  // namespace
+
+cudaError_t launch_pack_bf16(int H, int I, int expert_begin, int expert_count, const void* w_gate, const void* w_up,
+                             const void* w_down, const void* a_gate, const void* a_up, const void* a_down,
+                             const void* b_gate, const void* b_up, const void* b_down, int rank, float scaling,
+                             uint8_t* w13, uint8_t* s13, uint8_t* w2, uint8_t* s2, float* scales,
+                             cudaStream_t stream) {
+  if (expert_count == 0) return cudaSuccess;
+  PackBf16Args a;
+  a.wg = static_cast<const __nv_bfloat16*>(w_gate);
+  a.wu = static_cast<const __nv_bfloat16*>(w_up);
+  a.wd = static_cast<const __nv_bfloat16*>(w_down);
+  a.ag = static_cast<const __nv_bfloat16*>(a_gate);
+  a.au = static_cast<const __nv_bfloat16*>(a_up);
+  a.ad = static_cast<const __nv_bfloat16*>(a_down);
+  a.bg = static_cast<const __nv_bfloat16*>(b_gate);
+  a.bu = static_cast<const __nv_bfloat16*>(b_up);
+  a.bd = static_cast<const __nv_bfloat16*>(b_down);
+  const int64_t kb13 = 2 * static_cast<int64_t>(H) + 128, kb2 = 2 * static_cast<int64_t>(I) + 128;
+  a.w13 = w13 + static_cast<int64_t>(expert_begin) * 2 * I * kb13;
+  a.s13 = s13 + static_cast<int64_t>(expert_begin) * 64 * 2 * static_cast<int64_t>(H);
+  a.w2 = w2 + static_cast<int64_t>(expert_begin) * H * kb2;
+  a.s2 = s2 + static_cast<int64_t>(expert_begin) * 64 * 2 * static_cast<int64_t>(I);
+  a.H = H;
+  a.I = I;
+  a.r = rank;
+  const int64_t most = std::max(2 * static_cast<int64_t>(I) * kb13, static_cast<int64_t>(H) * kb2) / 16;
+  pack_bf16_kernel<<<dim3(static_cast<unsigned>((most + 255) / 256), 4, expert_count), 256, 0, stream>>>(a);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  bf16_scales_kernel<<<(3 * expert_count + 255) / 256, 256, 0, stream>>>(
+      expert_count, a.ag != nullptr ? scaling : 0.0f, scales + static_cast<int64_t>(expert_begin) * 3);
   return cudaGetLastError();
 }
 

@@ -232,7 +232,7 @@ class ExpertParallelLayer:
 
     def experts(self):
         """The grouped expert FFN over the received rows."""
-        B.moe_forward_grouped(self.cfg_loc, self.G * self.E_loc, self.packed, self.r_codes, self.r_sf,
+        B.moe_forward_grouped(self.cfg_loc, self.G * self.E_loc, self.R_recv, self.packed, self.r_codes, self.r_sf,
                               self.act_scale, self.inter_scale, self.group_offsets, self.group_counts,
                               self.group_expert, self.h_codes, self.h_sf, self.o_recv, None, self.status)
 

@@ -11,6 +11,9 @@ no shared expert, NVFP4 or MXFP8 experts; d_model 4096, expert ffn 2560):
   decode_mxfp8          T=256,   H=4096, I=2560, E=384, k=8, MXFP8
   prefill_nvfp4         T=8192,  H=4096, I=2560, E=384, k=8, NVFP4
   prefill_nvfp4_skewed  T=16384, H=4096, I=2560, E=384, k=8, NVFP4, Zipf bias
+  prefill_mxfp8         T=8192,  H=4096, I=2560, E=384, k=8, MXFP8
+  tiny_bf16_lora        T=64,    H=256,  I=128,  E=8,   k=2, BF16 + rank-32 adapters
+  decode_bf16_lora      T=64,    H=4096, I=2560, E=384, k=8, BF16 + rank-32 adapters
 
 Recipe
   x        bf16 ~ N(0, 1)            torch CPU generator, seed BASE + 2
@@ -20,6 +23,9 @@ Recipe
            (fan_in = H for gate/up, I for down), one generator per
            (expert, matrix) with seed BASE + 1000 + 3e + m, on the device
            the caller names.
+  BF16     the float32 weight draws rounded to bf16; adapters A ~ N(0,
+           1/fan_in), B ~ N(0, (0.15/sqrt(r))^2), rank 32, scaling 2, seed
+           BASE + 500000 + 6e + m (make_expert_lora).
   s_x, s_h static float32 activation tensor scales for NVFP4, the way a
            checkpoint carries them: s_x = 8/2688 (x ~ N(0,1) stays below 8),
            s_h = 24/2688.
@@ -35,6 +41,12 @@ BASE_SEED = 20261202
 
 NVFP4 = "nvfp4"
 MXFP8 = "mxfp8"
+BF16 = "bf16"
+
+# Adapters of the BF16 experts: rank 32 (the pages' validation run) and
+# scaling alpha / rank = 2.
+LORA_RANK = 32
+LORA_SCALING = 2.0
 
 S_X = np.float32(8.0 / 2688.0)
 S_H = np.float32(24.0 / 2688.0)
@@ -65,6 +77,9 @@ WORKLOADS = {
         Workload("prefill_nvfp4_skewed", 16384, 4096, 2560, 384, 8, NVFP4, skewed=True),
         # the MXFP8 layers (40-47) at the prefill batch of the NVFP4 layer
         Workload("prefill_mxfp8", 8192, 4096, 2560, 384, 8, MXFP8),
+        # BF16 experts with rank-32 adapters on gate, up and down
+        Workload("tiny_bf16_lora", 64, 256, 128, 8, 2, BF16),
+        Workload("decode_bf16_lora", 64, 4096, 2560, 384, 8, BF16),
     ]
 }
 
@@ -119,3 +134,25 @@ def make_logits_with_ties(T, E, seed):
     g = _gen(seed)
     v = torch.randint(-8, 9, (T, E), generator=g).to(torch.float32) * 0.25
     return v
+
+
+def make_expert_weights_bf16(wl: Workload, e, device="cpu"):
+    """bf16 (W_gate [I, H], W_up [I, H], W_down [H, I]) of expert e: the
+    float32 draws of make_expert_weights rounded to bf16."""
+    return tuple(w.to(torch.bfloat16) for w in make_expert_weights(wl, e, device))
+
+
+def make_expert_lora(wl: Workload, e, rank=LORA_RANK, device="cpu"):
+    """bf16 adapters (A_gate [r, H], B_gate [I, r], A_up [r, H], B_up [I, r],
+    A_down [r, I], B_down [H, r]) of expert e: A ~ N(0, 1/fan_in), B ~
+    N(0, (0.15 / sqrt(r))^2), so that with scaling 2 the adapter adds about a
+    third of the magnitude of the base projection.  One generator per
+    (expert, matrix), seed BASE + 500000 + 6e + m."""
+    H, I, r = wl.d_model, wl.d_ffn, int(rank)
+    shapes = (((r, H), 1 / math.sqrt(H)), ((I, r), 0.15 / math.sqrt(r)), ((r, H), 1 / math.sqrt(H)),
+              ((I, r), 0.15 / math.sqrt(r)), ((r, I), 1 / math.sqrt(I)), ((H, r), 0.15 / math.sqrt(r)))
+    out = []
+    for m, (shape, std) in enumerate(shapes):
+        g = _gen(BASE_SEED + 500000 + 6 * int(e) + m, device)
+        out.append((torch.randn(*shape, generator=g, dtype=torch.float32, device=device) * std).to(torch.bfloat16))
+    return tuple(out)

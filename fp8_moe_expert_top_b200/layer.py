@@ -45,15 +45,21 @@ class ExpertLayer:
         self.route_ws = torch.empty(B.moe_route_workspace_bytes(self.cfg, T), dtype=torch.uint8, device=dev)
         u8 = dict(dtype=torch.uint8, device=dev)
         self.a_codes = torch.empty(B.moe_codes_bytes(self.cfg, R, H), **u8)
-        self.a_sf = torch.empty(B.moe_sf_bytes(self.cfg, R, H), **u8)
         self.h_codes = torch.empty(B.moe_codes_bytes(self.cfg, R, I), **u8)
-        self.h_sf = torch.empty(B.moe_sf_bytes(self.cfg, R, I), **u8)
+        if self.cfg.fmt == B.MOE_BF16:   # no block scales
+            self.a_sf = self.h_sf = None
+        else:
+            self.a_sf = torch.empty(B.moe_sf_bytes(self.cfg, R, H), **u8)
+            self.h_sf = torch.empty(B.moe_sf_bytes(self.cfg, R, I), **u8)
         self.down_out = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
         self.y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
         self.status = torch.zeros(1, **i32)
         self.gateup_debug = torch.empty(R, 2 * I, dtype=torch.float32, device=dev) if debug else None
         f32 = dict(dtype=torch.float32, device=dev)
-        if self.fmt == B.MOE_NVFP4:
+        if self.fmt == B.MOE_BF16:
+            self.act_scale = None
+            self.inter_scale = None
+        elif self.fmt == B.MOE_NVFP4:
             if s_x is None or s_h is None:
                 raise ValueError("NVFP4 needs the static activation scales s_x and s_h")
             self.act_scale = torch.tensor([float(s_x)], **f32)
@@ -71,6 +77,26 @@ class ExpertLayer:
             if t.dtype != torch.float32 or tuple(t.shape) != shape:
                 raise ValueError(f"{name}: float32 {shape} expected, got {t.dtype} {tuple(t.shape)}")
         B.moe_quantize_weights(self.cfg, expert_begin, n, w_gate, w_up, w_down, self.packed)
+
+    def pack_experts_bf16(self, expert_begin, w_gate, w_up, w_down, lora=None, lora_rank=0, lora_scaling=0.0):
+        """BF16 layers: bf16 weights of experts [begin, begin + n) and their
+        adapters lora = (A_gate, B_gate, A_up, B_up, A_down, B_down) (bf16,
+        [n, r, H], [n, I, r], [n, r, H], [n, I, r], [n, r, I], [n, H, r]) or
+        None, into self.packed."""
+        if self.fmt != B.MOE_BF16:
+            raise ValueError("pack_experts_bf16 is for BF16 layers (quantize_experts for NVFP4 / MXFP8)")
+        n = w_gate.shape[0]
+        shapes = [(n, self.I, self.H), (n, self.I, self.H), (n, self.H, self.I)]
+        ts = [w_gate, w_up, w_down]
+        if lora is not None:
+            r = int(lora_rank)
+            shapes += [(n, r, self.H), (n, self.I, r), (n, r, self.H), (n, self.I, r), (n, r, self.I), (n, self.H, r)]
+            ts += list(lora)
+        for i, (t, shape) in enumerate(zip(ts, shapes)):
+            if t.dtype != torch.bfloat16 or tuple(t.shape) != shape:
+                raise ValueError(f"argument {i}: bfloat16 {shape} expected, got {t.dtype} {tuple(t.shape)}")
+        B.moe_pack_weights_bf16(self.cfg, expert_begin, n, w_gate, w_up, w_down, lora, lora_rank, lora_scaling,
+                                self.packed)
 
     # ------------------------------------------------------------- steps
     def _check_T(self, T):

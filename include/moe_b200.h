@@ -17,6 +17,12 @@
  *        MXFP8 experts": expert activations are quantized to match each
  *        layer's weight format, folded into the kernels that produce them.
  *
+ *   [P3] "thinkingmachines/Inkling-2-Small", section Configurations, and
+ *        "Thinking Machines releases Inkling 2 Small weights under Apache
+ *        2.0", section "LoRA and reinforcement learning": adapters on the
+ *        routed experts need BF16 expert weights (a rank-32 adapter in the
+ *        pages' validation run).
+ *
  * One layer on one stream is
  *     moe_route_topk -> moe_permute -> moe_forward -> moe_unpermute_combine
  * with moe_quantize_weights run once, offline.
@@ -77,7 +83,9 @@ typedef enum {
 
 typedef enum {
   MOE_NVFP4 = 0, /* E2M1 codes, 16-element E4M3 block scales, fp32 tensor scale [P1, P2] */
-  MOE_MXFP8 = 1  /* E4M3 codes, 32-element E8M0 block scales [P1] */
+  MOE_MXFP8 = 1, /* E4M3 codes, 32-element E8M0 block scales [P1] */
+  MOE_BF16 = 2   /* bf16 expert weights and activations, with LoRA adapters on the
+                    experts (rank <= 32) [P3] */
 } moe_format;
 
 typedef struct {
@@ -111,6 +119,19 @@ typedef struct {
  *   scales     [E][3] float32     tensor scales of (gate, up, down); 1.0 for
  *                                 MXFP8
  */
+/* MOE_BF16 (no quantization; one extra 64-element K tile per row carries
+ * the adapters, so kb(K) = 2K + 128):
+ *   w13_codes  [E][2I x kb(H)]    bf16 rows as above (gate / up interleaved);
+ *                                 the last K tile of a gate row holds
+ *                                 B_gate[c][0..32) then 32 zeros, of an up row
+ *                                 32 zeros then B_up[c][0..32)
+ *   w13_sf     [E][64 x 2H]       the adapters' A_gate (rows 0-31) and A_up
+ *                                 (rows 32-63), bf16, tiled with TR = 64
+ *   w2_codes   [E][H x kb(I)]     bf16 down rows; last K tile B_down[n][0..32)
+ *                                 then 32 zeros
+ *   w2_sf      [E][64 x 2I]       A_down (rows 0-31) and 32 zero rows, TR = 64
+ *   scales     [E][3] float32     (adapter scaling, 0, 0)
+ * An adapter of rank r < 32 is zero-padded; an expert without one has zeros. */
 typedef struct {
   int64_t w13_codes;
   int64_t w13_sf;
@@ -165,6 +186,25 @@ MOE_API int64_t moe_route_workspace_bytes(const moe_config* cfg, int64_t T);
 MOE_API moe_status moe_quantize_weights(const moe_config* cfg, int32_t expert_begin, int32_t expert_count,
                                 const float* w_gate, const float* w_up, const float* w_down, void* packed,
                                 void* stream);
+
+/* Offline packing of BF16 expert weights and their LoRA adapters [P3]
+ * (MOE_BF16 only; moe_quantize_weights returns MOE_ERR_UNSUPPORTED for it).
+ * Experts [expert_begin, expert_begin + expert_count) of `packed`:
+ *   w_gate, w_up    bf16 [n][I][H];  w_down  bf16 [n][H][I]
+ *   lora_a_gate, lora_a_up  bf16 [n][lora_rank][H]; lora_a_down bf16
+ *                   [n][lora_rank][I]; lora_b_gate, lora_b_up bf16
+ *                   [n][I][lora_rank]; lora_b_down bf16 [n][H][lora_rank]
+ *                   (all six, or all six NULL for experts without adapters)
+ *   lora_rank       1 .. 32 (MOE_ERR_UNSUPPORTED otherwise)
+ *   lora_scaling    the adapters' scaling (alpha / rank)
+ * Each projection then computes W a + lora_scaling * B (A a).  The adapters'
+ * products A a are rounded to bf16 (they feed the tensor cores as bf16 with
+ * the expert's own rows). */
+MOE_API moe_status moe_pack_weights_bf16(const moe_config* cfg, int32_t expert_begin, int32_t expert_count,
+                                         const void* w_gate, const void* w_up, const void* w_down,
+                                         const void* lora_a_gate, const void* lora_b_gate, const void* lora_a_up,
+                                         const void* lora_b_up, const void* lora_a_down, const void* lora_b_down,
+                                         int32_t lora_rank, float lora_scaling, void* packed, void* stream);
 
 /* Routing [P1 Overview; P2 "NVFP4 and MXFP8 experts": top-k of the routed
  * experts, no shared expert].  For T tokens of float32 logits [T][E]:
@@ -243,7 +283,13 @@ MOE_API moe_status moe_permute(const moe_config* cfg, int64_t T, const void* x_b
  *   gateup_debug      optional float32 [R_max][2I]: g in columns [0, I) and
  *                     u in [I, 2I) (NULL in normal use)
  *   status_word       optional uint32 device status word (MOE_DEVICE_*)
- * moe_forward runs moe_forward_gateup then moe_forward_down. */
+ * moe_forward runs moe_forward_gateup then moe_forward_down.
+ * MOE_BF16 [P3]: no quantization and no block scales (a_sf, h_sf may be
+ * NULL, the activation scales are ignored); h is bf16 (moe_codes_bytes(cfg,
+ * R_max, I)); moe_forward_gateup first writes each row's adapter product
+ * lora_scaling * (A_gate a, A_up a) into the last K tile of a_codes (left
+ * free by moe_permute), then the gate/up GEMM, then the down adapter's
+ * product of h into h's last K tile; moe_forward_down runs over it. */
 MOE_API moe_status moe_forward(const moe_config* cfg, int64_t T, const void* packed, const void* a_codes,
                        const void* a_sf, const float* act_scale, const float* inter_scale,
                        const int32_t* expert_offsets, const int32_t* expert_counts, void* h_codes, void* h_sf,
@@ -265,6 +311,8 @@ MOE_API moe_status moe_forward_down(const moe_config* cfg, int64_t T, const void
  * computes the rows of expert group_expert[g] of `packed`.
  *   cfg            num_experts = experts held in `packed` (this rank's slice)
  *   num_groups     row groups, 0 .. 1024
+ *   max_rows       rows the buffers hold (a multiple of 128, >= the last
+ *                  group offset)
  *   group_offsets  int32 [num_groups + 1], device: first row of each group,
  *                  multiples of 128, non-decreasing, group_offsets[0] = 0
  *   group_counts   int32 [num_groups], device: rows in use per group,
@@ -278,8 +326,8 @@ MOE_API moe_status moe_forward_down(const moe_config* cfg, int64_t T, const void
  *                  multiple of 128 rows at least that large)
  * The row layout and the results of each row are independent of the other
  * groups: a row gives the same bits as in moe_forward. */
-MOE_API moe_status moe_forward_grouped(const moe_config* cfg, int32_t num_groups, const void* packed,
-                                       const void* a_codes, const void* a_sf, const float* act_scale,
+MOE_API moe_status moe_forward_grouped(const moe_config* cfg, int32_t num_groups, int64_t max_rows,
+                                       const void* packed, const void* a_codes, const void* a_sf, const float* act_scale,
                                        const float* inter_scale, const int32_t* group_offsets,
                                        const int32_t* group_counts, const int32_t* group_expert, void* h_codes,
                                        void* h_sf, void* down_out, float* gateup_debug, uint32_t* status_word,

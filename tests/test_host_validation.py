@@ -27,7 +27,8 @@ CALLS = {
     "moe_forward": lambda h: B.moe_forward(CFG, 4, h, h, h, h, h, h, h, h, h, h),
     "moe_forward_gateup": lambda h: B.moe_forward_gateup(CFG, 4, h, h, h, h, h, h, h, h, h),
     "moe_forward_down": lambda h: B.moe_forward_down(CFG, 4, h, h, h, h, h, h, h),
-    "moe_forward_grouped": lambda h: B.moe_forward_grouped(CFG, 2, h, h, h, h, h, h, h, h, h, h, h),
+    "moe_forward_grouped": lambda h: B.moe_forward_grouped(CFG, 2, 128, h, h, h, h, h, h, h, h, h, h, h),
+    "moe_pack_weights_bf16": lambda h: B.moe_pack_weights_bf16(CFG, 0, 1, h, h, h, packed=h),
     "moe_unpermute_combine": lambda h: B.moe_unpermute_combine(CFG, 4, h, h, h, h),
     "moe_selftest_bounded_wait": lambda h: B.moe_selftest_bounded_wait(h, 1000),
 }
