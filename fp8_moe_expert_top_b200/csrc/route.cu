@@ -11,9 +11,9 @@
 //   1. route_topk_kernel  one warp per token, 8 tokens per CTA: top-k by k
 //      warp-wide arg-max rounds (ties to the lower index), the softmax, and
 //      bit t of the expert's token bitmap set (atomicOr, order-independent).
-//   2. route_scan_kernel  one CTA: for every expert the exclusive prefix of
-//      popc over its bitmap words (its slot count at the end), then the
-//      128-padded expert offsets.
+//   2. route_scan_kernel  one CTA per expert: the exclusive prefix of popc
+//      over its bitmap words (its slot count at the end); the last CTA to
+//      finish scans the 128-padded counts into the expert offsets.
 //   3. route_scatter_kernel  one thread per slot: row = offset[e] +
 //      prefix[e][t/32] + (tokens before t in word t/32 that chose e).
 // Nothing depends on thread timing, so the result is deterministic.
@@ -131,57 +131,76 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   return incl - v + (warp > 0 ? warp_sums[warp - 1] : 0);
 }
 
-// One CTA of 1024 threads.  Warp w scans the bitmaps of experts w, w + 32, ...:
-// prefix[e][i] = sum of popc over words 0..i-1 of expert e, 32 words (one per
-// lane, coalesced) per warp scan, with the loads of up to 8 such chunks
-// issued before their scans; then the padded offsets over experts.
-__global__ void __launch_bounds__(1024) route_scan_kernel(int E, int W, const uint32_t* __restrict__ bitmap,
-                                                           int32_t* __restrict__ prefix,
-                                                           int32_t* __restrict__ expert_counts,
-                                                           int32_t* __restrict__ expert_offsets) {
-  __shared__ int32_t s_count[1024];
+constexpr int kScanThreads = 256;
+constexpr int kScanWordsPerThread = 4;
+
+// One CTA per expert: prefix[e][i] = sum of popc over words 0..i-1 of expert
+// e's token bitmap (kScanWordsPerThread consecutive words per thread, one
+// block-wide scan per 1024 words), and expert_counts[e].  The CTA that
+// finishes last (a ticket counter, zeroed with the bitmaps) then scans the
+// 128-padded counts of all experts into expert_offsets.  Which CTA that is
+// depends on timing; what it computes does not.
+__global__ void __launch_bounds__(kScanThreads) route_scan_kernel(int E, int W, const uint32_t* __restrict__ bitmap,
+                                                                  int32_t* __restrict__ prefix,
+                                                                  int32_t* __restrict__ expert_counts,
+                                                                  int32_t* __restrict__ expert_offsets,
+                                                                  unsigned int* __restrict__ ticket) {
   __shared__ int32_t warp_sums[32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ int is_last;
+  const int e = blockIdx.x;
   pdl_wait();
   pdl_trigger();
-  for (int e = warp; e < E; e += 32) {
-    const uint32_t* bm = bitmap + static_cast<int64_t>(e) * W;
-    int32_t* pf = prefix + static_cast<int64_t>(e) * W;
-    int32_t base = 0;
-    for (int w0 = 0; w0 < W; w0 += 256) {
-      const int chunks = min(8, (W - w0 + 31) / 32);  // the same for the whole warp
-      int32_t c[8];
+  const uint32_t* bm = bitmap + static_cast<int64_t>(e) * W;
+  int32_t* pf = prefix + static_cast<int64_t>(e) * W;
+  int32_t base = 0;
+  for (int w0 = 0; w0 < W; w0 += kScanThreads * kScanWordsPerThread) {
+    const int i0 = w0 + kScanWordsPerThread * threadIdx.x;
+    int32_t c[kScanWordsPerThread];
+    int32_t mine = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = w0 + 32 * j + lane;
-        c[j] = (j < chunks && i < W) ? __popc(bm[i]) : 0;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j >= chunks) break;
-        int32_t incl = c[j];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-          if (lane >= off) incl += o;
-        }
-        const int i = w0 + 32 * j + lane;
-        if (i < W) pf[i] = base + incl - c[j];
-        base += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      }
+    for (int j = 0; j < kScanWordsPerThread; ++j) {
+      c[j] = (i0 + j < W) ? __popc(bm[i0 + j]) : 0;
+      mine += c[j];
     }
-    if (lane == 0) s_count[e] = base;
+    int32_t chunk_total = 0;
+    int32_t run = base + block_exclusive_scan(mine, warp_sums, &chunk_total);
+#pragma unroll
+    for (int j = 0; j < kScanWordsPerThread; ++j) {
+      if (i0 + j < W) pf[i0 + j] = run;
+      run += c[j];
+    }
+    base += chunk_total;
+    __syncthreads();  // warp_sums is reused by the next chunk's scan
+  }
+  if (threadIdx.x == 0) {
+    expert_counts[e] = base;
+    __threadfence();
+    is_last = atomicAdd(ticket, 1u) == static_cast<unsigned int>(E - 1);
   }
   __syncthreads();
-  const int e = threadIdx.x;
-  const int32_t cnt = (e < E) ? s_count[e] : 0;
-  int32_t total = 0;
-  const int32_t off = block_exclusive_scan(((cnt + 127) / 128) * 128, warp_sums, &total);
-  if (e < E) {
-    expert_counts[e] = cnt;
-    expert_offsets[e] = off;
+  if (!is_last) return;
+  __threadfence();
+  // padded exclusive offsets over the experts, kScanWordsPerThread experts per thread
+  const volatile int32_t* counts = expert_counts;
+  int32_t padded[kScanWordsPerThread];
+  int32_t mine = 0;
+  const int e0 = kScanWordsPerThread * threadIdx.x;
+#pragma unroll
+  for (int j = 0; j < kScanWordsPerThread; ++j) {
+    padded[j] = (e0 + j < E) ? (counts[e0 + j] + 127) / 128 * 128 : 0;
+    mine += padded[j];
   }
-  if (e == 0) expert_offsets[E] = total;
+  int32_t total = 0;
+  int32_t run = block_exclusive_scan(mine, warp_sums, &total);
+#pragma unroll
+  for (int j = 0; j < kScanWordsPerThread; ++j) {
+    if (e0 + j < E) expert_offsets[e0 + j] = run;
+    run += padded[j];
+  }
+  if (threadIdx.x == 0) {
+    expert_offsets[E] = total;
+    *ticket = 0u;
+  }
 }
 
 __global__ void route_scatter_kernel(int T, int E, int k, int W, const int32_t* __restrict__ topk_ids,
@@ -203,8 +222,19 @@ __global__ void route_scatter_kernel(int T, int E, int k, int W, const int32_t* 
 
 int64_t route_workspace_bytes(int E, int64_t T) {
   const int64_t W = (T + 31) / 32;
-  return static_cast<int64_t>(E) * W * 8 + 256;  // bitmap words + their prefix counts
+  return static_cast<int64_t>(E) * W * 8 + 256;  // bitmap words, ticket, their prefix counts
 }
+
+// Workspace: token bitmaps [E][W] words, a 16-byte ticket counter, prefix
+// counts [E][W]; the bitmaps and the ticket are zeroed by route_prepare.
+namespace {
+unsigned int* ws_ticket(void* ws, int E, int W) {
+  return reinterpret_cast<unsigned int*>(static_cast<uint32_t*>(ws) + static_cast<int64_t>(E) * W);
+}
+int32_t* ws_prefix(void* ws, int E, int W) {
+  return reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + static_cast<int64_t>(E) * W * 4 + 16);
+}
+}  // namespace
 
 cudaError_t route_prepare(int T, int E, int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
                           int64_t R_max, void* workspace, cudaStream_t stream) {
@@ -216,7 +246,7 @@ cudaError_t route_prepare(int T, int E, int32_t* expert_counts, int32_t* expert_
     return cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), stream);
   }
   const int W = (T + 31) / 32;
-  return cudaMemsetAsync(workspace, 0, static_cast<size_t>(E) * W * sizeof(uint32_t), stream);
+  return cudaMemsetAsync(workspace, 0, static_cast<size_t>(E) * W * sizeof(uint32_t) + 16, stream);
 }
 
 cudaError_t route_finish(int T, int E, int k, const int32_t* topk_ids, int32_t* expert_counts,
@@ -224,9 +254,9 @@ cudaError_t route_finish(int T, int E, int k, const int32_t* topk_ids, int32_t* 
                          cudaStream_t stream) {
   const int W = (T + 31) / 32;
   const uint32_t* bitmap = static_cast<const uint32_t*>(workspace);
-  int32_t* prefix = reinterpret_cast<int32_t*>(static_cast<uint32_t*>(workspace) + static_cast<int64_t>(E) * W);
-  cudaError_t err = launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, stream, E, W, bitmap, prefix,
-                               expert_counts, expert_offsets);
+  int32_t* prefix = ws_prefix(workspace, E, W);
+  cudaError_t err = launch_pdl(route_scan_kernel, dim3(E), dim3(kScanThreads), 0, stream, E, W, bitmap, prefix,
+                               expert_counts, expert_offsets, ws_ticket(workspace, E, W));
   if (err != cudaSuccess) return err;
   const int64_t slots = static_cast<int64_t>(T) * k;
   return launch_pdl(route_scatter_kernel, dim3(static_cast<unsigned>((slots + 255) / 256)), dim3(256), 0, stream, T,
