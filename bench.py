@@ -42,7 +42,8 @@ METRIC = "MoE layer tokens/s on 1 B200; % of HBM or NVFP4/FP8 tensor roofline"
 UNIT = "tokens/s"
 # the largest single-GPU layer, and the other full-size layers measured beside it
 HEADLINE = "prefill_nvfp4_skewed"
-FULL_SIZE = ("decode_nvfp4", "decode_mxfp8", "prefill_nvfp4", "prefill_nvfp4_skewed", "prefill_mxfp8")
+FULL_SIZE = ("decode_nvfp4", "decode_mxfp8", "prefill_nvfp4", "prefill_nvfp4_skewed", "prefill_mxfp8",
+             "decode_bf16_lora")
 
 
 # --------------------------------------------------------------------------- helpers
@@ -199,6 +200,15 @@ def build_layer(wl, device, T):
     chunk = 16
     for e0 in range(0, wl.num_experts, chunk):
         n = min(chunk, wl.num_experts - e0)
+        if wl.fmt == inputs.BF16:
+            # bf16 weights with rank-32 adapters on gate, up and down
+            ws = [inputs.make_expert_weights_bf16(wl, e, device=device) for e in range(e0, e0 + n)]
+            ls = [inputs.make_expert_lora(wl, e, device=device) for e in range(e0, e0 + n)]
+            lora = tuple(torch.stack([l_[m] for l_ in ls]).contiguous() for m in range(6))
+            layer.pack_experts_bf16(e0, *(torch.stack([w[m] for w in ws]).contiguous() for m in range(3)),
+                                    lora=lora, lora_rank=inputs.LORA_RANK, lora_scaling=inputs.LORA_SCALING)
+            del ws, ls, lora
+            continue
         ws = [inputs.make_expert_weights(wl, e, device=device) for e in range(e0, e0 + n)]
         wg = torch.stack([w[0] for w in ws]).contiguous()
         wu = torch.stack([w[1] for w in ws]).contiguous()
@@ -212,11 +222,18 @@ def build_layer(wl, device, T):
 def phase_bytes(wl, n_touched, slots):
     """Algorithmic HBM bytes of each phase (compulsory traffic, no re-reads)."""
     H, I, E, T = wl.d_model, wl.d_ffn, wl.num_experts, wl.T
-    bpe = 0.5 if wl.fmt == inputs.NVFP4 else 1.0
-    sf = 1.0 / (16 if wl.fmt == inputs.NVFP4 else 32)
-    q = bpe + sf                                  # bytes per quantized element (codes + block scales)
-    w13 = n_touched * 2 * I * H * q
-    w2 = n_touched * H * I * q
+    if wl.fmt == inputs.BF16:
+        # bf16 weights; each row carries its adapter's 64-element tile (B),
+        # plus the adapters' A (64 rows of H and of I per expert)
+        q = 2.0
+        w13 = n_touched * (2 * I * (H + 64) + 64 * H) * 2
+        w2 = n_touched * (H * (I + 64) + 64 * I) * 2
+    else:
+        bpe = 0.5 if wl.fmt == inputs.NVFP4 else 1.0
+        sf = 1.0 / (16 if wl.fmt == inputs.NVFP4 else 32)
+        q = bpe + sf                              # bytes per quantized element (codes + block scales)
+        w13 = n_touched * 2 * I * H * q
+        w2 = n_touched * H * I * q
     return {
         "route": T * E * 4 + T * wl.top_k * 8,
         "permute": T * H * 2 + slots * H * q,
@@ -342,7 +359,8 @@ def run_ours(args, wl, ws, rank, local):
     dom_flops = slots * flops_slot * (2.0 / 3.0 if dom == "gateup" else 1.0 / 3.0)
     t_dom = mean_ms[dom] * 1e-3
     bf16 = peaks.get("bf16_tflops", 1590.0)
-    tensor_peak = bf16 * (4.0 if wl.fmt == inputs.NVFP4 else 2.0)     # nominal fp4 / fp8 : bf16 ratios
+    ratio = {inputs.NVFP4: 4.0, inputs.MXFP8: 2.0, inputs.BF16: 1.0}[wl.fmt]   # nominal fp4 / fp8 : bf16
+    tensor_peak = bf16 * ratio
     t_hbm = bytes_[dom] / (peaks["hbm_gbs"] * 1e9)
     t_tc = dom_flops / (tensor_peak * 1e12)
     if t_hbm >= t_tc:
@@ -351,16 +369,15 @@ def run_ours(args, wl, ws, rank, local):
         roof = {"bound": "tensor", "achieved": dom_flops / t_dom / 1e12, "peak": tensor_peak, "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     # against the nominal B200 peaks (8 TB/s HBM; 9 / 4.5 PFLOP/s dense NVFP4 / FP8)
-    roof["frac_nominal"] = roof["achieved"] / (8000.0 if roof["bound"] == "hbm" else
-                                               (9000.0 if wl.fmt == inputs.NVFP4 else 4500.0))
+    nominal_tensor = {inputs.NVFP4: 9000.0, inputs.MXFP8: 4500.0, inputs.BF16: 2250.0}[wl.fmt]
+    roof["frac_nominal"] = roof["achieved"] / (8000.0 if roof["bound"] == "hbm" else nominal_tensor)
     roof["kernel"] = f"moe_gemm_kernel ({dom})"
     roof["peak_source"] = peak_kind + (" hbm_gbs" if roof["bound"] == "hbm" else
-                                       f" bf16_tflops x {4 if wl.fmt == inputs.NVFP4 else 2} (nominal ratio)")
+                                       f" bf16_tflops x {ratio:g} (nominal ratio)")
     roof["traffic"] = measured_traffic(wl.name, dom)
     # whole-layer roofline (slower of bytes at HBM peak and FLOPs at tensor peak)
     layer_t = max(bytes_["layer"] / (peaks["hbm_gbs"] * 1e9), slots * flops_slot / (tensor_peak * 1e12))
-    # nominal B200 peaks for context: 8 TB/s HBM, 9 / 4.5 PFLOP/s dense NVFP4 / FP8
-    nominal_tensor = 9000.0 if wl.fmt == inputs.NVFP4 else 4500.0
+    # nominal B200 peaks for context: 8 TB/s HBM, 9 / 4.5 / 2.25 PFLOP/s dense NVFP4 / FP8 / BF16
     layer_t_nominal = max(bytes_["layer"] / 8.0e12, slots * flops_slot / (nominal_tensor * 1e12))
     value = ws * T * args.steps / (total_ms * 1e-3)
     out = {
@@ -394,10 +411,69 @@ def run_ours(args, wl, ws, rank, local):
                            "(two graphs, upload and download streams); no L2 flush, each step streams "
                            "GBs of weights"},
         # per step: route top-k, scan, scatter; permute; gate/up; down; combine
-        "gpu_launches": 7 * args.steps,
+        # (BF16: and the two adapter shrinks)
+        "gpu_launches": (9 if wl.fmt == inputs.BF16 else 7) * args.steps,
         "clocks": clk,
     }
     return out, layer
+
+
+def time_fused_router(args, device):
+    """Routing from the layer input (router scores fused with the top-k,
+    moe_router_topk) against routing from given logits (moe_route_topk), at
+    the decode, prefill and skewed batch sizes.  Each is one CUDA graph,
+    replayed args.steps times with an L2 flush between replays; per-replay
+    device time from CUDA events."""
+    from fp8_moe_expert_top_b200 import binding as B
+    torch.cuda.set_device(device)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    out = {}
+    for name in ("decode_nvfp4", "prefill_nvfp4", "prefill_nvfp4_skewed"):
+        wl = inputs.WORKLOADS[name]
+        T, E, H, k = wl.T, wl.num_experts, wl.d_model, wl.top_k
+        cfg = B.make_config(E, k, H, wl.d_ffn, wl.fmt)
+        R = B.moe_max_rows(cfg, T)
+        i32 = dict(dtype=torch.int32, device=device)
+        bufs = (torch.empty(T, k, **i32), torch.empty(T, k, dtype=torch.float32, device=device),
+                torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R, **i32), torch.empty(T * k, **i32))
+        ws = torch.empty(B.moe_route_workspace_bytes(cfg, T), dtype=torch.uint8, device=device)
+        x = inputs.make_x(wl).to(device)
+        lg = inputs.make_logits(wl).to(device)
+        g = torch.Generator(device=device)
+        g.manual_seed(inputs.BASE_SEED + 3)
+        w_r = (torch.randn(E, H, generator=g, device=device) / H ** 0.5).to(torch.bfloat16)
+        status = torch.zeros(1, **i32)
+        calls = {"from_logits": lambda: B.moe_route_topk(cfg, T, lg, *bufs, ws),
+                 "fused_router": lambda: B.moe_router_topk(cfg, T, x, w_r, None, *bufs, ws, status)}
+        res = {}
+        for key, fn in calls.items():
+            for _ in range(args.warmup):
+                fn()
+            graph = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(device=device)
+            side.wait_stream(stream)
+            with torch.cuda.graph(graph, stream=side):
+                fn()
+            stream.wait_stream(side)
+            times = []
+            for _ in range(args.steps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+            res[key + "_ms"] = statistics.mean(times)
+            del graph
+        if int(status.item()) != 0:
+            raise RuntimeError(f"device status word {int(status.item()):#x} from the fused router")
+        flops = 2.0 * T * E * H
+        res["router_tflops"] = flops / (res["fused_router_ms"] * 1e-3) / 1e12
+        res["T"] = T
+        out[name] = res
+    return out
 
 
 def measured_traffic(workload, phase):
@@ -643,6 +719,7 @@ def main(argv=None):
                 out["workloads"][name] = {key: o[key] for key in (
                     "value", "unit", "ms_per_step", "dtype", "config", "roofline", "layer_roofline_frac",
                     "layer_roofline_frac_nominal", "step_ms_pct", "phase_ms", "e2e", "gpu_launches", "clocks")}
+            out["fused_router"] = time_fused_router(args, torch.device("cuda", local))
         if rank == 0:
             if ws == 1 and not args.no_cpu_baseline:
                 out["cpu_baseline"] = cpu_baseline(wl)
