@@ -1,16 +1,17 @@
-"""Expert-parallel plumbing on CPU (gloo, two ranks).
+"""Expert-parallel plumbing on CPU (gloo, two and four ranks).
 
 The exchanges of fp8_moe_expert_top_b200.ep (counts, dispatch of the
 quantized rows as whole 128-row blocks of tiled codes and scale atoms,
 return of the output rows) and its plan (split sizes, row groups) are the
-host side of the expert-parallel layer.  Here two gloo ranks run them on CPU
+host side of the expert-parallel layer.  Here gloo ranks (two, and four with
+uneven token counts) run them on CPU
 tensors laid out exactly as the kernels lay them out, with the oracle
 standing in for the kernels on each rank (routing, quantized rows, each
 received group's expert FFN, the combine).  Checked:
   * every received row group (s, e) holds, bit for bit, the codes and block
     scales of rank s's tokens routed to local expert e, in token order;
   * each rank's output equals the oracle's single-process forward over the
-    tokens of both ranks, on that rank's tokens;
+    tokens of all ranks, on that rank's tokens;
   * the plan alone, on random and edge-case counts (empty experts, a rank
     that sends nothing).
 """
@@ -31,7 +32,7 @@ from helpers import ACT_TR, kb_padded, pack_nvfp4, pad_row_bytes, sfvec, swizzle
     unswizzle_sf
 
 WL = inputs.WORKLOADS["tiny_nvfp4"]
-TOKENS = (40, 57)
+TOKENS = (40, 57, 3, 13)   # tokens of ranks 0..3 (the first `world` are used)
 
 
 def _free_port():
@@ -119,9 +120,8 @@ def _rank_main(rank, world, port, fmt, out_dir):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp8"])
-def test_ep_two_ranks_match_single_process(tmp_path, fmt):
-    world = 2
+@pytest.mark.parametrize("fmt,world", [("nvfp4", 2), ("mxfp8", 2), ("nvfp4", 4)])
+def test_ep_ranks_match_single_process(tmp_path, fmt, world):
     for _ in range(3):            # the probed port can be taken before gloo binds it
         try:
             mp.start_processes(_rank_main, args=(world, _free_port(), fmt, str(tmp_path)), nprocs=world,
