@@ -166,7 +166,8 @@ moe_status moe_route_topk(const moe_config* cfg, int64_t T, const float* logits,
   moe_status s = check(cfg);
   if (s != MOE_OK) return s;
   if ((s = check_T(T)) != MOE_OK) return s;
-  if (!expert_counts || !expert_offsets || !sorted_slots) return MOE_ERR_INVALID_ARG;
+  // sorted_slots has max_rows(T) rows: none for an empty batch
+  if (!expert_counts || !expert_offsets || (T > 0 && !sorted_slots)) return MOE_ERR_INVALID_ARG;
   if (T > 0 && (!logits || !topk_ids || !topk_w || !slot_to_row || !workspace)) return MOE_ERR_INVALID_ARG;
   if (workspace_bytes < moe::route_workspace_bytes(cfg->num_experts, T)) return MOE_ERR_WORKSPACE;
   if (workspace && !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
@@ -183,7 +184,7 @@ moe_status moe_router_topk(const moe_config* cfg, int64_t T, const void* x_bf16,
   if (s != MOE_OK) return s;
   if ((s = check_T(T)) != MOE_OK) return s;
   if (cfg->num_experts > 512) return MOE_ERR_UNSUPPORTED;  // all scores of a token in one TMEM accumulator
-  if (!expert_counts || !expert_offsets || !sorted_slots) return MOE_ERR_INVALID_ARG;
+  if (!expert_counts || !expert_offsets || (T > 0 && !sorted_slots)) return MOE_ERR_INVALID_ARG;
   if (T > 0 && (!x_bf16 || !w_router_bf16 || !topk_ids || !topk_w || !slot_to_row || !workspace))
     return MOE_ERR_INVALID_ARG;
   if (workspace_bytes < moe::route_workspace_bytes(cfg->num_experts, T)) return MOE_ERR_WORKSPACE;

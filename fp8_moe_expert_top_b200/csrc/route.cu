@@ -238,8 +238,11 @@ int32_t* ws_prefix(void* ws, int E, int W) {
 
 cudaError_t route_prepare(int T, int E, int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
                           int64_t R_max, void* workspace, cudaStream_t stream) {
-  cudaError_t err = cudaMemsetAsync(sorted_slots, 0xFF, static_cast<size_t>(R_max) * sizeof(int32_t), stream);
-  if (err != cudaSuccess) return err;
+  cudaError_t err = cudaSuccess;
+  if (R_max > 0) {
+    err = cudaMemsetAsync(sorted_slots, 0xFF, static_cast<size_t>(R_max) * sizeof(int32_t), stream);
+    if (err != cudaSuccess) return err;
+  }
   if (T == 0) {
     err = cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * E, stream);
     if (err != cudaSuccess) return err;

@@ -223,6 +223,7 @@ MOE_API moe_status moe_pack_weights_bf16(const moe_config* cfg, int32_t expert_b
  *   sorted_slots   int32 [R_max]  slot t*k+j held by each row, rows of one
  *                                 expert in ascending token order; -1 for
  *                                 padding rows and rows >= expert_offsets[E]
+ *                                 (R_max = 0 when T = 0: may then be NULL)
  *   slot_to_row    int32 [T*k]    row of each slot
  *   workspace      moe_route_workspace_bytes(cfg, T) bytes of scratch
  * Logits must not be NaN.  The result does not depend on thread timing. */

@@ -119,7 +119,7 @@ def test_ep_emulated_ranks_match_single_gpu(cuda_device, name, G, tokens):
 def test_ep_single_rank_forward(cuda_device):
     dev = cuda_device
     wl = inputs.WORKLOADS["tiny_nvfp4"]
-    ref = build_layer(wl, dev, debug=False)
+    ref = build_layer(wl, dev, debug=False, weight_device=dev)   # the ranks draw their weights on the device too
     x, lg = inputs.make_x(wl).to(dev), inputs.make_logits(wl).to(dev)
     y_ref = ref.forward(x, lg).clone()
     (r,) = _ranks(wl, 1, (wl.T,), dev)

@@ -17,7 +17,9 @@ float64 and rounds once (oracle.route.router_logits).
     (H additions, each off by at most one float32 ulp even if the hardware
     truncates, and the final rounding),
     and on every token whose k+1 largest exact scores are separated by more
-    than twice that bound the selection and its order are unique: ids must
+    than twice the largest distance of its scores from the exact sums (the
+    kernel's, bounded as above, plus the oracle's half-ulp rounding) the
+    selection and its order are unique on both sides: ids must
     equal the oracle's, and each weight is within the first-order effect of
     its token's score differences (twice the largest, plus float32 roundings).  For every
     token the routing must be consistent: counts, padded offsets and the slot
@@ -132,11 +134,15 @@ def test_router_random_inputs_within_bound(cuda_device, T):
     bound = H * 2.0 ** -23 * mag + np.abs(exact) * 2.0 ** -24
     assert np.all(np.abs(got - exact) <= bound), float(np.max(np.abs(got - exact) / bound))
     ref = ort.router_route(x, w, k, E)
-    # tokens whose top k+1 exact scores are separated by more than twice the bound
+    # Tokens whose top k+1 exact scores are separated by more than twice the
+    # largest distance of any of the token's scores from the exact sum, on
+    # either side (the kernel's, now bounded above, and the oracle's float32
+    # rounding, at most half an ulp): there both orders equal the exact one.
+    dev_t = (np.max(np.abs(got - exact), axis=1, keepdims=True)
+             + np.max(np.abs(exact), axis=1, keepdims=True) * 2.0 ** -24)
     srt = -np.sort(-exact, axis=1)[:, :k + 1]
-    tb = 2.0 * bound.max(axis=1, keepdims=True)
-    unique = np.all(srt[:, :-1] - srt[:, 1:] > tb, axis=1)
-    assert unique.sum() >= T // 20, unique.mean()
+    unique = np.all(srt[:, :-1] - srt[:, 1:] > 2.0 * dev_t, axis=1)
+    assert unique.mean() >= 0.5, unique.mean()
     ids = b["ids"].cpu().numpy()
     np.testing.assert_array_equal(ids[unique], ref["topk_ids"][unique])
     # softmax weights: d(log w_j) = dl_j - sum_i w_i dl_i, so a weight moves
