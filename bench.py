@@ -668,6 +668,8 @@ def main(argv=None):
     ap.add_argument("--only", action="store_true", help="measure only --workload, not the other full-size layers")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--router-only", action="store_true",
+                    help="time only routing: the fused router against routing from given logits")
     ap.add_argument("--experts", type=int, default=None,
                     help="profiling only: override the number of experts (smaller device footprint for ncu)")
     ap.add_argument("--tokens", type=int, default=None,
@@ -705,6 +707,10 @@ def main(argv=None):
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
+        if args.router_only:
+            if rank == 0:
+                print(json.dumps({"fused_router": time_fused_router(args, torch.device("cuda", local))}))
+            return 0
         out, layer = run_ours(args, wl, ws, rank, local)
         del layer
         torch.cuda.empty_cache()

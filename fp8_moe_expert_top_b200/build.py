@@ -19,9 +19,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
-SOURCES = ["api.cu", "route.cu", "router.cu", "permute.cu", "weights.cu", "gemm.cu", "lora.cu", "noalloc.cu",
-           "selftest.cu"]
-HEADERS = ["common.cuh", "quant.cuh", "kernels.cuh", "gemm_common.cuh", "route_common.cuh"]
+SOURCES = ["api.cu", "route.cu", "router.cu", "permute.cu", "weights.cu", "gemm.cu", "gemm_pair.cu", "lora.cu",
+           "noalloc.cu", "selftest.cu"]
+HEADERS = ["common.cuh", "quant.cuh", "kernels.cuh", "gemm_common.cuh", "route_common.cuh", "pair.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
 

@@ -234,7 +234,8 @@ struct Groups {
   const int32_t* offsets;
   const int32_t* counts;
   const int32_t* expert;
-  int64_t R_max;  // rows the buffers hold (bounds the adapter shrink's grid)
+  int64_t R_max;  // rows the buffers hold (bounds the adapter shrink's grid and the tensor maps)
+  int64_t slots;  // T * k when known (selects the GEMM kernel), else 0
 };
 
 // gate/up GEMM + SwiGLU + h in the layer format.  BF16: the adapter shrink
@@ -257,6 +258,8 @@ static moe_status run_gateup(const moe_config* cfg, const Groups& G, const uint8
   g.fmt = cfg->fmt;
   g.gateup = true;
   g.E = G.n;
+  g.R_max = G.R_max;
+  g.slots = G.slots;
   g.K = cfg->d_model + (bf16 ? 64 : 0);
   g.n_rows_b = 2 * cfg->d_ffn;
   g.a_codes = static_cast<const uint8_t*>(a_codes);
@@ -293,6 +296,8 @@ static moe_status run_down(const moe_config* cfg, const Groups& G, const uint8_t
   g.fmt = cfg->fmt;
   g.gateup = false;
   g.E = G.n;
+  g.R_max = G.R_max;
+  g.slots = G.slots;
   g.K = cfg->d_ffn + (cfg->fmt == MOE_BF16 ? 64 : 0);
   g.n_rows_b = cfg->d_model;
   g.a_codes = static_cast<const uint8_t*>(h_codes);
@@ -321,7 +326,7 @@ moe_status moe_forward_gateup(const moe_config* cfg, int64_t T, const void* pack
   if (!sf_ok(cfg, a_sf) || !sf_ok(cfg, h_sf)) return MOE_ERR_INVALID_ARG;
   if (cfg->fmt == MOE_NVFP4 && (!act_scale || !inter_scale)) return MOE_ERR_INVALID_ARG;
   if (gateup_debug && !aligned16(gateup_debug)) return MOE_ERR_INVALID_ARG;
-  const Groups G{cfg->num_experts, expert_offsets, expert_counts, nullptr, max_rows(cfg, T)};
+  const Groups G{cfg->num_experts, expert_offsets, expert_counts, nullptr, max_rows(cfg, T), T * cfg->top_k};
   return run_gateup(cfg, G, static_cast<const uint8_t*>(packed), a_codes, a_sf, act_scale, inter_scale, h_codes,
                     h_sf, gateup_debug, status_word, static_cast<cudaStream_t>(stream));
 }
@@ -335,7 +340,7 @@ moe_status moe_forward_down(const moe_config* cfg, int64_t T, const void* packed
   if (!h_codes || !down_out || !aligned16(h_codes) || !aligned16(down_out)) return MOE_ERR_INVALID_ARG;
   if (!sf_ok(cfg, h_sf)) return MOE_ERR_INVALID_ARG;
   if (cfg->fmt == MOE_NVFP4 && !inter_scale) return MOE_ERR_INVALID_ARG;
-  const Groups G{cfg->num_experts, expert_offsets, expert_counts, nullptr, max_rows(cfg, T)};
+  const Groups G{cfg->num_experts, expert_offsets, expert_counts, nullptr, max_rows(cfg, T), T * cfg->top_k};
   return run_down(cfg, G, static_cast<const uint8_t*>(packed), h_codes, h_sf, inter_scale, down_out, status_word,
                   static_cast<cudaStream_t>(stream));
 }
@@ -369,7 +374,7 @@ moe_status moe_forward_grouped(const moe_config* cfg, int32_t num_groups, int64_
   if (cfg->fmt == MOE_NVFP4 && (!act_scale || !inter_scale)) return MOE_ERR_INVALID_ARG;
   const uint8_t* base = static_cast<const uint8_t*>(packed);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Groups G{num_groups, group_offsets, group_counts, group_expert, max_rows_};
+  const Groups G{num_groups, group_offsets, group_counts, group_expert, max_rows_, 0};
   s = run_gateup(cfg, G, base, a_codes, a_sf, act_scale, inter_scale, h_codes, h_sf, gateup_debug, status_word, st);
   if (s != MOE_OK) return s;
   return run_down(cfg, G, base, h_codes, h_sf, inter_scale, down_out, status_word, st);

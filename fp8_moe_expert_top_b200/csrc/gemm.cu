@@ -30,11 +30,14 @@
 //               SwiGLU + requantization (gate/up) or bf16 store (down)
 //   warps 10-11 scale copiers: the stage's scale atoms SMEM -> TMEM
 //               (tcgen05.cp), alternate k blocks each, into per-stage TMEM
-//               columns.
-// A tcgen05.cp holds its issuing thread for about 50 cycles, copies from
-// different threads overlap, and copies issued by the MMA thread queue behind
-// its MMAs; so the MMA thread issues none and each stage's 12 (NVFP4) copies
-// are spread over two threads of their own.
+//               columns; they signal the MMA thread once the copies are
+//               issued (the copy -> MMA order is kept by the tensor pipe).
+// A tcgen05.cp holds its issuing thread for about 50 cycles and the copies
+// share the tensor pipe with the MMAs; issued by the MMA thread they delay
+// its MMAs (measured: the prefill gate/up GEMM 1.5x slower), so each stage's
+// 12 (NVFP4) copies are spread over threads of their own.  A tcgen05.cp is
+// issued once per warp instruction, not once per active lane: the issuing
+// threads must be lanes of different warps.
 // Every mbarrier wait is bounded; a wait that runs out raises a CTA-wide
 // abort flag and every role stops issuing.  Work already in flight (bulk
 // copies into stages nobody consumed, MMAs, scale copies) is then waited for,
@@ -43,6 +46,8 @@
 // operation.  A status bit reports the abort.
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
   uint64_t* empty_bar = full_bar + kStages;
   uint64_t* tfull_bar = empty_bar + kStages;
   uint64_t* tempty_bar = tfull_bar + 1;
-  uint64_t* sf_bar = tempty_bar + 1;  // a stage's scales are in TMEM
+  uint64_t* sf_bar = tempty_bar + 1;  // a stage's scale copies are issued
   uint64_t* drain_bar = sf_bar + kStages;  // after an abort: in-flight tcgen05 work has finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -214,8 +219,8 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
         tc_fence_after();
         bool ok = true;
         for (int kt = 0; kt < k_tiles; ++kt) {
-          // the scale copiers have seen the stage's operands land and their
-          // copies have completed (the operand wait then returns at once)
+          // the scale copiers have seen the stage's operands land and issued
+          // their copies (the operand wait then returns at once)
           if ((Tr::kScaled && !mbar_wait(&sf_bar[stage], phase, abort_flag)) ||
               !mbar_wait(&full_bar[stage], phase, abort_flag)) {
             fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
@@ -283,7 +288,7 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
 #pragma unroll
               for (int h = 0; h < kBN / 128; ++h)
                 tc_cp_sf_atom(sfb + (kBN / 32) * kb + 4 * h,
-                      make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
+                              make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
             }
           } else if (part == 0) {
             tc_cp_sf_atom(sfa, make_desc_sf(st + Tr::kSfaOff));
@@ -293,7 +298,12 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
             for (int h = 1; h < kBN / 128; ++h)
               tc_cp_sf_atom(sfb + 4 * h, make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128));
           }
-          tc_commit(&sf_bar[stage]);
+          // Signal that the copies are issued, not that they are complete:
+          // tcgen05.cp -> tcgen05.mma is a pipelined pair, so the MMA
+          // thread's fence::after_thread_sync after this barrier orders its
+          // MMAs behind these copies in the tensor pipe.
+          tc_fence_before();
+          mbar_arrive(&sf_bar[stage]);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
@@ -402,6 +412,22 @@ size_t gemm_smem_bytes(int fmt, int E) {
   return 1024 + kStages * sb + (3 * kStages + 3) * 8 + 16 + (E + 1) * 4;
 }
 
+cudaError_t launch_gemm_pair(const GemmLaunch& g, const GemmArgs& a, cudaStream_t stream);  // gemm_pair.cu
+
+namespace {
+// Which kernel serves block-scaled GEMMs: one SM per tile unless
+// MOE_B200_GEMM = "pair" asks for the SM-pair kernel (kept as an option: it
+// is exact but measured slower than one SM per tile at prefill).
+int gemm_mode() {
+  static const int mode = [] {
+    const char* v = std::getenv("MOE_B200_GEMM");
+    if (v == nullptr) return 0;
+    return std::strcmp(v, "pair") == 0 ? 2 : 1;
+  }();
+  return mode;
+}
+}  // namespace
+
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
   const int bits = (g.fmt == MOE_NVFP4) ? 4 : (g.fmt == MOE_MXFP8 ? 8 : 16);
   const int sfvec = (g.fmt == MOE_MXFP8) ? 32 : 16;
@@ -431,6 +457,9 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
   a.n_rows_b = g.n_rows_b;
   a.sf_rb_stride = static_cast<int64_t>(g.K / sfvec) * 128;
   a.b_sf_expert_stride = static_cast<int64_t>(g.n_rows_b) * (g.K / sfvec);
+  if (g.fmt != MOE_BF16 && g.R_max > 0) {
+    if (gemm_mode() == 2) return launch_gemm_pair(g, a, stream);
+  }
   if (g.fmt == MOE_NVFP4)
     return g.gateup ? launch_one<MOE_NVFP4, true>(a, stream) : launch_one<MOE_NVFP4, false>(a, stream);
   if (g.fmt == MOE_BF16)

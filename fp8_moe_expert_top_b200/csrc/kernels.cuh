@@ -72,6 +72,7 @@ struct GemmLaunch {
   uint32_t* status;
   const int32_t* expert_map;  // optional [E]: row group -> expert of the packed weights
   int n_weights;              // experts in the packed weights (with expert_map)
+  int64_t slots;              // token slots routed (T * k), 0 when unknown; selects the SM-pair kernel
 };
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream);
 

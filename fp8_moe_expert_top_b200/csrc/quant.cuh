@@ -147,7 +147,9 @@ __device__ __forceinline__ float nvfp4_candidate(const float* ax, float a, float
       d2[i + 1] = __fmul_rn(d1, d1);
     }
   } else {  // tiny scales: exact division throughout
-#pragma unroll 1
+    // unrolled like the paths above: a runtime index into ax / d2 would put
+    // both arrays in local memory for every call, not only for this path
+#pragma unroll
     for (int i = 0; i < 16; ++i) {
       const uint32_t m = e2m1_code_exact(ax[i], S);
       mags |= static_cast<uint64_t>(m) << (4 * i);

@@ -31,6 +31,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "pair.cuh"
 #include "route_common.cuh"
 
 namespace moe {
@@ -269,6 +270,277 @@ __global__ void __launch_bounds__(kRThreads, 1)
   }
 }
 
+// Small batches: the same scores with K split over a cluster of KS CTAs per
+// 128 tokens, so that a decode batch spreads its router weights over KS SMs
+// instead of one.  CTA r of the cluster accumulates k tiles
+// [r KT/KS, (r+1) KT/KS) of all NB expert blocks in TMEM; after every CTA's
+// MMAs are complete (first cluster barrier) each token row's partial scores
+// are pushed (st.shared::cluster) into the ring of the CTA that owns the row
+// (owner r holds rows [r RPO, (r+1) RPO), RPO = 128 / KS), slot r of it;
+// after the second cluster barrier each owner sums the KS partials of its
+// rows in rank order (so the scores do not depend on timing) and a warp per
+// row selects the top-k: each lane keeps a sorted top-8 of the experts
+// e = lane (mod 32), scanned in ascending order, and k rounds of a warp
+// argmax over the lanes' heads (higher score, then lower index) give the
+// ranked selection.  The softmax and the bitmap update are those of
+// route_topk_kernel.  Every thread passes both cluster barriers exactly once,
+// whatever happened before, so a CTA that timed out cannot stall the others.
+template <int NB, int ST, int KS>
+__global__ void __launch_bounds__(kRThreads, 1)
+    router_split_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                        const RouterArgs args) {
+  constexpr int kStageBytes = kRTileBytes * (1 + NB);
+  constexpr uint32_t kTmemCols = NB == 1 ? 128u : (NB == 2 ? 256u : 512u);
+  constexpr int EP = NB * 128;     // scores per row in the receive slots
+  constexpr int RPO = kRM / KS;    // rows owned by each CTA
+  static_assert(KS * RPO * EP * 4 <= ST * kStageBytes, "receive slots must fit in the ring");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* recv = reinterpret_cast<float*>(smem);  // [KS][RPO][EP], 16-byte units XOR-swizzled by row
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + ST * kStageBytes);
+  uint64_t* empty_bar = full_bar + ST;
+  uint64_t* acc_bar = empty_bar + ST;
+  uint64_t* drain_bar = acc_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* drain_failed = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int m0 = static_cast<int>(blockIdx.x / KS) * kRM;
+  const int kt_per = (args.H / kRKElems) / KS;
+  const int kt0 = static_cast<int>(rank) * kt_per;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(acc_bar, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *drain_failed = 0;
+    fence_mbar_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  pdl_wait();
+  pdl_trigger();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  uint32_t fail_bits = 0;
+  uint32_t armed = 0u, armed_par = 0u;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kt = kt0; kt < kt0 + kt_per; ++kt) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+          fail_bits |= MOE_DEVICE_TIMEOUT_PRODUCER;
+          break;
+        }
+        uint8_t* st = smem + stage * kStageBytes;
+        mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
+        tma_load_2d(st, &tmap_x, kt * kRKElems, m0, &full_bar[stage]);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+          tma_load_2d(st + kRTileBytes * (1 + b), &tmap_w, kt * kRKElems, b * 128, &full_bar[stage]);
+        armed |= 1u << stage;
+        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == ST) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = 0; i < kt_per; ++i) {
+        if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+          fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + stage * kStageBytes);
+        const uint64_t adesc = make_desc_sw128(st);
+#pragma unroll
+        for (int kk = 0; kk < kRKElems / 16; ++kk) {
+          const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
+#pragma unroll
+          for (int b = 0; b < NB; b += 2) {
+            const uint64_t bdesc = make_desc_sw128(st + kRTileBytes * (1 + b));
+            if (b + 1 < NB)
+              tc_mma_bf16(tmem_base + 128 * b, adesc + 2 * kk, bdesc + 2 * kk, idesc_bf16(256), acc);
+            else
+              tc_mma_bf16(tmem_base + 128 * b, adesc + 2 * kk, bdesc + 2 * kk, idesc_bf16(128), acc);
+          }
+        }
+        tc_commit(&empty_bar[stage]);
+        if (++stage == ST) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) tc_commit(acc_bar);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue: accumulator complete
+    if (!mbar_wait(acc_bar, 0, abort_flag)) fail_bits |= MOE_DEVICE_TIMEOUT_EPILOGUE;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (*abort_flag) {
+    // drain what is in flight before the ring is overwritten and TMEM freed
+    bool drained = true;
+    if (warp == 0 && lane == 0) {
+      for (int st = 0; st < ST; ++st)
+        if ((armed >> st) & 1u) drained = mbar_wait_drain(&full_bar[st], (armed_par >> st) & 1u) && drained;
+    } else if (warp == 1 && lane == 0) {
+      tc_commit(drain_bar);
+      drained = mbar_wait_drain(drain_bar, 0);
+    }
+    if (!drained) *drain_failed = 1;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  const bool acc_ok = !*abort_flag;
+  cluster_sync();  // every CTA's MMAs are complete: all rings may be written
+
+  if (warp >= 2 && acc_ok) {
+    // push this CTA's partial scores of each row into the row's owner
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t owner = static_cast<uint32_t>(row / RPO);
+    const int r_loc = row % RPO;
+    const uint32_t dst = mapa_shared(smem_u32(recv), owner) +
+                         static_cast<uint32_t>(((static_cast<int>(rank) * RPO + r_loc) * EP) * 4);
+    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+    for (int c = 0; c < NB * 4; ++c) {
+      float v[32];
+      tmem_ld32(t_row + 32 * c, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t unit = static_cast<uint32_t>(8 * c + u) ^ static_cast<uint32_t>(r_loc & 7);
+        st_cluster_v4(dst + 16u * unit, v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // every partial has arrived at its owner
+  tc_fence_after();
+
+  if (warp >= 2) {
+    // reduce the owned rows over the KS partials, then top-k (a warp per row)
+    for (int r_loc = warp - 2; r_loc < RPO; r_loc += kREpiWarps) {
+      const int t = m0 + static_cast<int>(rank) * RPO + r_loc;
+      if (t >= args.T) break;
+      float tv[8];
+      int ti[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        tv[j] = -INFINITY;
+        ti[j] = 0x7FFFFFFF;
+      }
+#pragma unroll
+      for (int i = 0; i < EP / 32; ++i) {
+        const int e = 32 * i + lane;
+        const int off = 4 * ((e >> 2) ^ (r_loc & 7)) + (e & 3);
+        float v = recv[(0 * RPO + r_loc) * EP + off];
+#pragma unroll
+        for (int s = 1; s < KS; ++s) v = __fadd_rn(v, recv[(s * RPO + r_loc) * EP + off]);
+        if (e < args.E) {
+          if (args.logits_out != nullptr) args.logits_out[static_cast<int64_t>(t) * args.E + e] = v;
+          if (v > tv[7] || ti[7] == 0x7FFFFFFF) {
+            tv[7] = v;
+            ti[7] = e;
+#pragma unroll
+            for (int j = 7; j > 0; --j) {
+              if (tv[j] > tv[j - 1] || ti[j - 1] == 0x7FFFFFFF) {
+                const float fv = tv[j];
+                tv[j] = tv[j - 1];
+                tv[j - 1] = fv;
+                const int fi = ti[j];
+                ti[j] = ti[j - 1];
+                ti[j - 1] = fi;
+              }
+            }
+          }
+        }
+      }
+      // k rounds of a warp argmax over the lanes' heads
+      const int k = args.k;
+      float sv[8];
+      int si[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float bv = tv[0];
+        int bi = ti[0];
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1) {
+          const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, d);
+          const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, d);
+          if (oi != 0x7FFFFFFF && (bi == 0x7FFFFFFF || ov > bv || (ov == bv && oi < bi))) {
+            bv = ov;
+            bi = oi;
+          }
+        }
+        sv[j] = bv;
+        si[j] = bi;
+        if (bi != 0x7FFFFFFF && (bi & 31) == lane) {  // the winner's lane drops its head
+#pragma unroll
+          for (int i = 0; i < 7; ++i) {
+            tv[i] = tv[i + 1];
+            ti[i] = ti[i + 1];
+          }
+          tv[7] = -INFINITY;
+          ti[7] = 0x7FFFFFFF;
+        }
+      }
+      // softmax over the k selected scores, as route_topk_kernel computes it
+      float ex[8];
+      float s = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        ex[j] = (j < k) ? exp_own(__fsub_rn(sv[j], sv[0])) : 0.0f;
+        if (j == 0) s = ex[0];
+        else if (j < k) s = __fadd_rn(s, ex[j]);
+      }
+      const int64_t o = static_cast<int64_t>(t) * k;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < k && lane == j) {
+          args.topk_ids[o + j] = si[j];
+          args.topk_w[o + j] = __fdiv_rn(ex[j], s);
+          atomicOr(&args.bitmap[static_cast<int64_t>(si[j]) * args.W + (t >> 5)], 1u << (t & 31));
+        }
+      }
+    }
+  }
+
+  if (fail_bits != 0u && args.status != nullptr) atomicOr(args.status, fail_bits);
+  if (warp == 1 && !*drain_failed) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
 template <int NB>
 constexpr int router_stages() {
   return (kRTileBytes * (1 + NB) * 4 <= 200 * 1024) ? 4 : ((kRTileBytes * (1 + NB) * 3 <= 200 * 1024) ? 3 : 2);
@@ -327,6 +599,57 @@ cudaError_t launch_nb(const CUtensorMap& mx, const CUtensorMap& mw, const Router
   return launch_pdl(router_topk_kernel<NB, ST>, grid, dim3(kRThreads), smem, stream, mx, mw, a);
 }
 
+template <int NB, int KS>
+cudaError_t launch_split(const CUtensorMap& mx, const CUtensorMap& mw, const RouterArgs& a, cudaStream_t stream) {
+  constexpr int ST = router_stages<NB>();
+  constexpr size_t smem = router_smem<NB>();
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(router_split_kernel<NB, ST, KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem));
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((a.T + kRM - 1) / kRM * KS));
+  cfg.blockDim = dim3(kRThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = KS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, router_split_kernel<NB, ST, KS>, mx, mw, a);
+}
+
+template <int NB>
+cudaError_t launch_any(const CUtensorMap& mx, const CUtensorMap& mw, const RouterArgs& a, int ks,
+                       cudaStream_t stream) {
+  switch (ks) {
+    case 2: return launch_split<NB, 2>(mx, mw, a, stream);
+    case 4: return launch_split<NB, 4>(mx, mw, a, stream);
+    case 8: return launch_split<NB, 8>(mx, mw, a, stream);
+    default: return launch_nb<NB>(mx, mw, a, stream);
+  }
+}
+
+// K split of the scores: the largest of 8, 4, 2 that divides the k tiles and
+// keeps the clusters within one wave of CTAs (148 SMs, one CTA each); 1 (no
+// split) for large batches and for 512 experts, whose receive slots would not
+// fit in the ring.
+int router_split(int T, int H, int nb) {
+  if (nb > 3) return 1;
+  const int m = (T + kRM - 1) / kRM, kt = H / kRKElems;
+  for (int ks = 8; ks >= 2; ks >>= 1)
+    if (kt % ks == 0 && m * ks <= 148) return ks;
+  return 1;
+}
+
 }  // namespace
 
 cudaError_t launch_router_topk(const void* x, const void* w_router, float* logits_out, int T, int E, int H, int k,
@@ -346,10 +669,11 @@ cudaError_t launch_router_topk(const void* x, const void* w_router, float* logit
   a.k = k;
   a.W = (T + 31) / 32;
   const int nb = (E + 127) / 128;
+  const int ks = router_split(T, H, nb);
   switch (nb) {
-    case 1: return launch_nb<1>(mx, mw, a, stream);
-    case 2: return launch_nb<2>(mx, mw, a, stream);
-    case 3: return launch_nb<3>(mx, mw, a, stream);
+    case 1: return launch_any<1>(mx, mw, a, ks, stream);
+    case 2: return launch_any<2>(mx, mw, a, ks, stream);
+    case 3: return launch_any<3>(mx, mw, a, ks, stream);
     case 4: return launch_nb<4>(mx, mw, a, stream);
     default: return cudaErrorInvalidValue;
   }

@@ -35,8 +35,11 @@ from oracle import route as ort
 
 # (T, E, H, k): tiny, one token, a ragged batch at the model's size, experts
 # not a multiple of 128, the 512-expert limit (two-stage ring), several tiles.
+# Batches of up to 74 row tiles split K over clusters of 2-8 CTAs; the
+# 512-expert case and the 9600-token case (75 row tiles) take the unsplit
+# kernel.
 GRID_CASES = [(64, 8, 256, 2), (1, 384, 4096, 8), (777, 384, 4096, 8), (300, 200, 512, 6), (256, 512, 1024, 8),
-              (129, 128, 256, 1)]
+              (129, 128, 256, 1), (9600, 384, 512, 8)]
 
 
 def _bufs(cfg, T, E, k, dev):
@@ -114,7 +117,7 @@ def _check_consistent(b, T, E, k):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("T", [2048, 8192])
+@pytest.mark.parametrize("T", [64, 2048, 8192, 16384])
 def test_router_random_inputs_within_bound(cuda_device, T):
     dev = cuda_device
     E, H, k = 384, 4096, 8
