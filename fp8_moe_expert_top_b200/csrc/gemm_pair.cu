@@ -1,23 +1,25 @@
-// The grouped block-scaled GEMMs on SM pairs, for batches whose experts hold
-// several 128-row blocks (prefill).
+// The grouped block-scaled GEMMs on SM pairs (selected with
+// MOE_B200_GEMM=pair; the one-SM kernel of gemm.cu is the default).
 //
-// Same computation and epilogue as the one-SM kernel (gemm.cu); the
-// difference is how a tile's operands reach the tensor cores.  A pair of CTAs
-// (a cluster of two, one per SM) owns a 256-row x 256-column output tile of
-// one expert: each CTA loads its own 128 activation rows and one half (128
-// rows) of the 256-row weight tile, plus the scales, and the leader CTA
-// issues tcgen05.mma.cta_group::2 (M = 256), which reads the weight halves
-// from both CTAs' shared memory.  A stage is 38 KB per SM instead of 54 KB for
-// the same 512 tensor-core clocks per SM: filling shared memory, which bounds
-// the one-SM kernel at prefill, needs a third fewer bytes per MMA.
+// Same computation and epilogue as the one-SM kernel; the difference is how a
+// tile's operands reach the tensor cores.  A pair of CTAs (a cluster of two,
+// one per SM) owns a 256-row x 256-column output tile of one expert: each CTA
+// loads its own 128 activation rows and one half (128 rows) of the 256-row
+// weight tile, plus the scales, and the leader CTA issues
+// tcgen05.mma.cta_group::2 (M = 256), which reads the weight halves from both
+// CTAs' shared memory.  A stage is 38 KB per SM instead of 54 KB for the same
+// tensor-core work.  Measured at prefill it is bit-exact but about 1.7x slower
+// per SM than the one-SM kernel: every MMA of the pair still needs its three
+// scale-atom copies (cta_group::2) in each CTA's TMEM, and the leader's MMA
+// thread spends most of its time waiting for them or blocked issuing.
 //
 // Synchronization: both CTAs' loads of a stage complete on the leader's
-// "full" barrier (cp.async.bulk.tensor .cta_group::2, no multicast); the
+// "full" barrier (cp.async.bulk.tensor .cta_group::2, no multicast), on which
+// each CTA's producer arrives once announcing its own bytes (the follower's
+// arrival is remote), so neither waits for the other before loading; the
 // MMA warp's commits arrive on the "empty" and "accumulator full" barriers of
 // both CTAs (tcgen05.commit multicast); both CTAs' epilogue threads release the
-// accumulator on the leader's "accumulator empty" barrier.  The follower loads
-// a stage only after the leader has armed its "full" barrier for that phase
-// (a remote arrive on the follower's "armed" barrier).  The leader's two
+// accumulator on the leader's "accumulator empty" barrier.  The leader's six
 // copier warps move each stage's scale atoms into both CTAs' TMEM
 // (tcgen05.cp.cta_group::2).  Every wait is bounded; a wait that runs out
 // raises the abort flags of both CTAs, work in flight is drained, and a
@@ -40,8 +42,17 @@ namespace moe {
 namespace {
 
 constexpr int kPairStages = 5;
-constexpr int kPairCopierWarps = 2;
-constexpr int kPairThreads = kThreads + 32 * kPairCopierWarps;
+// Warp roles as in the one-SM kernel: warp 0 producer (both CTAs), warp 1
+// MMA issuer (leader), warps 2-7 scale copiers (leader), warps 8-15 epilogue
+// (both CTAs); registers 72 for warps 0-7, 184 for the epilogue warpgroups.
+constexpr int kPairCopierWarps = 6;
+constexpr int kPairEpiWarp0 = 2 + kPairCopierWarps;
+constexpr int kPairThreads = 32 * (kPairEpiWarp0 + kEpiWarps);
+constexpr uint32_t kPairRegsLight = 72;
+constexpr uint32_t kPairRegsEpilogue = 184;
+static_assert(kPairThreads == 512 && kPairEpiWarp0 % 4 == 0, "warpgroup-aligned roles");
+static_assert(32 * kPairEpiWarp0 * kPairRegsLight + 32 * kEpiWarps * kPairRegsEpilogue <= 65536u,
+              "the register split must fit in the block's launch allocation (512 x 128)");
 template <int FMT>
 constexpr uint32_t kPairSfCols = (FMT == MOE_NVFP4) ? 48u : 12u;  // TMEM scale columns per stage
 static_assert(kBN + kPairStages * 48 <= kTmemCols, "scale buffers do not fit in TMEM");
@@ -78,8 +89,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint64_t* tfull_bar = empty_bar + kPairStages;
   uint64_t* tempty_bar = tfull_bar + 1;
   uint64_t* sf_bar = tempty_bar + 1;           // a stage's scale copies are issued
-  uint64_t* armed_bar = sf_bar + kPairStages;  // follower: the leader has armed the stage's full barrier
-  uint64_t* drain_bar = armed_bar + kPairStages;  // after an abort: the leader's tcgen05 work has finished
+  uint64_t* drain_bar = sf_bar + kPairStages;  // after an abort: the leader's tcgen05 work has finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* drain_failed = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -94,10 +104,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) {
-      mbar_init(&full_bar[s], 1);
+      mbar_init(&full_bar[s], 2);  // one arrival per CTA of the pair
       mbar_init(&empty_bar[s], 1);
       mbar_init(&sf_bar[s], kPairCopierWarps);
-      mbar_init(&armed_bar[s], 1);
     }
     mbar_init(tfull_bar, 1);
     mbar_init(tempty_bar, 2 * 32 * kEpiWarps);
@@ -176,193 +185,197 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     return c;
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
-      const uint64_t pol_stream = policy_evict_first();
-      const uint64_t pol_keep = policy_evict_normal();
-      const uint64_t pol_a = policy_evict_last();
-      const uint32_t full_leader0 = mapa_shared(smem_u32(&full_bar[0]), 0);
-      const uint32_t armed_peer0 = mapa_shared(smem_u32(&armed_bar[0]), 1);
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int tile = cid; tile < total && !*abort_flag; tile += ncl) {
-        const PairCoord c = coord(tile);
-        const int e = c.e, we = c.we;
-        const int rows_end = s_offsets[e] + __ldg(args.counts + e);
-        const int v0 = max(0, min(kBM, rows_end - c.mt0 * kBM));
-        const int v1 = max(0, min(kBM, rows_end - (c.mt0 + 1) * kBM));
-        const int my_rows = rows_loaded(rank ? v1 : v0);
-        const int my_mt = c.mt0 + static_cast<int>(rank);
-        const uint64_t pol_w = (s_offsets[e + 1] - s_offsets[e]) > 2 * kBM ? pol_keep : pol_stream;
-        // byte offsets of this CTA's k-tile 0 (tiles are 128 bytes wide, K tile fastest)
-        const int64_t a_off0 = static_cast<int64_t>(my_mt) * ktiles_row * (kBM * 128);
-        const int64_t b_off0 = (static_cast<int64_t>(we) * n_tiles + c.nt) * ktiles_row * (kBN * 128) +
-                               static_cast<int64_t>(kBM * 128) * rank;
-        // a CTA whose row block holds no valid row (past its group, possibly
-        // past the buffer) loads no codes, and the scales of the pair's first
-        // block (its output rows are never stored)
-        const int64_t asf0 = static_cast<int64_t>(my_rows > 0 ? my_mt : c.mt0) * args.sf_rb_stride;
-        const int64_t bsf0 = static_cast<int64_t>(we) * args.b_sf_expert_stride +
-                             static_cast<int64_t>(c.nt) * (kBN / 128) * args.sf_rb_stride;
-        for (int kt = 0; kt < k_tiles; ++kt) {
-          if (!mbar_wait_pair(&empty_bar[stage], phase ^ 1u, abort_flag, peer_abort)) {
-            fail_bits |= MOE_DEVICE_TIMEOUT_PRODUCER;
-            break;
-          }
-          const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
-          const int atoms = (FMT == MOE_NVFP4) ? kb_here : 1;
-          const uint32_t sf_bytes = 512u * atoms;
-          const uint32_t bar = full_leader0 + 8u * stage;
-          if (leader) {
-            const uint32_t a_bytes = static_cast<uint32_t>(rows_loaded(v0) + rows_loaded(v1)) * 128u;
-            mbar_arrive_expect_tx(&full_bar[stage], a_bytes + 2u * (16384u + 3u * sf_bytes));
-            armed |= 1u << stage;
-            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-            mbar_arrive_cluster(armed_peer0 + 8u * stage);  // the follower may load into this phase now
-          } else if (!mbar_wait_pair(&armed_bar[stage], phase, abort_flag, peer_abort)) {
-            // every copy of the pair lands in a phase the leader armed, so its
-            // drain after an abort covers the follower's copies too
-            fail_bits |= MOE_DEVICE_TIMEOUT_PRODUCER;
-            break;
-          }
-          uint8_t* st = smem + stage * Tr::kStageBytes;
-          const int64_t a_off = a_off0 + static_cast<int64_t>(kt) * (kBM * 128);
-          if (my_rows > 0)
-            tma_load_2d_pair(st, &maps.a[my_rows / 32 - 1], 0, static_cast<int32_t>(a_off / kLine), bar, pol_a);
-          tma_load_2d_pair(st + Tr::kABytes, &maps.b, 0,
-                           static_cast<int32_t>((b_off0 + static_cast<int64_t>(kt) * (kBN * 128)) / kLine), bar,
-                           pol_w);
-          const int64_t asf_off = asf0 + static_cast<int64_t>(kt) * Tr::kSfBytes128;
-          if (atoms == 4) {
-            tma_load_2d_pair(st + Tr::kSfaOff, &maps.asf4, 0, static_cast<int32_t>(asf_off / kLine), bar, pol_a);
-          } else {
-            for (int a = 0; a < atoms; ++a)
-              tma_load_2d_pair(st + Tr::kSfaOff + 512 * a, &maps.asf1, 0,
-                               static_cast<int32_t>((asf_off + 512 * a) / kLine), bar, pol_a);
-          }
-#pragma unroll
-          for (int h = 0; h < kBN / 128; ++h) {
-            const int64_t bsf_off = bsf0 + h * args.sf_rb_stride + static_cast<int64_t>(kt) * Tr::kSfBytes128;
-            uint8_t* dst = st + Tr::kSfbOff + h * Tr::kSfBytes128;
+  // Roles by warpgroup (every warp of a warpgroup executes the same setmaxnreg).
+  if (warp < kPairEpiWarp0) {
+    reg_dealloc<kPairRegsLight>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer (both CTAs)
+      if (lane == 0) {
+        const uint64_t pol_stream = policy_evict_first();
+        const uint64_t pol_keep = policy_evict_normal();
+        const uint64_t pol_a = policy_evict_last();
+        const uint32_t full_leader0 = mapa_shared(smem_u32(&full_bar[0]), 0);
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int tile = cid; tile < total && !*abort_flag; tile += ncl) {
+          const PairCoord c = coord(tile);
+          const int e = c.e, we = c.we;
+          const int rows_end = s_offsets[e] + __ldg(args.counts + e);
+          const int v0 = max(0, min(kBM, rows_end - c.mt0 * kBM));
+          const int v1 = max(0, min(kBM, rows_end - (c.mt0 + 1) * kBM));
+          const int my_rows = rows_loaded(rank ? v1 : v0);
+          const int my_mt = c.mt0 + static_cast<int>(rank);
+          const uint64_t pol_w = (s_offsets[e + 1] - s_offsets[e]) > 2 * kBM ? pol_keep : pol_stream;
+          // byte offsets of this CTA's k-tile 0 (tiles are 128 bytes wide, K tile fastest)
+          const int64_t a_off0 = static_cast<int64_t>(my_mt) * ktiles_row * (kBM * 128);
+          const int64_t b_off0 = (static_cast<int64_t>(we) * n_tiles + c.nt) * ktiles_row * (kBN * 128) +
+                                 static_cast<int64_t>(kBM * 128) * rank;
+          // a CTA whose row block holds no valid row (past its group, possibly
+          // past the buffer) loads no codes, and the scales of the pair's first
+          // block (its output rows are never stored)
+          const int64_t asf0 = static_cast<int64_t>(my_rows > 0 ? my_mt : c.mt0) * args.sf_rb_stride;
+          const int64_t bsf0 = static_cast<int64_t>(we) * args.b_sf_expert_stride +
+                               static_cast<int64_t>(c.nt) * (kBN / 128) * args.sf_rb_stride;
+          for (int kt = 0; kt < k_tiles; ++kt) {
+            if (!mbar_wait_pair(&empty_bar[stage], phase ^ 1u, abort_flag, peer_abort)) {
+              fail_bits |= MOE_DEVICE_TIMEOUT_PRODUCER;
+              break;
+            }
+            const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
+            const int atoms = (FMT == MOE_NVFP4) ? kb_here : 1;
+            const uint32_t sf_bytes = 512u * atoms;
+            const uint32_t bar = full_leader0 + 8u * stage;
+            // this CTA's bytes of the stage: its activation rows, its half of
+            // the weight tile, the activation scales and both weight halves' scales
+            const uint32_t my_bytes = static_cast<uint32_t>(my_rows) * 128u + 16384u + 3u * sf_bytes;
+            if (leader) {
+              mbar_arrive_expect_tx(&full_bar[stage], my_bytes);
+              armed |= 1u << stage;
+              armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+            } else {
+              // the previous phase of this stage completed before the MMAs that
+              // freed it ran, so this arrival belongs to the phase being filled
+              mbar_arrive_expect_tx_cluster(bar, my_bytes);
+            }
+            uint8_t* st = smem + stage * Tr::kStageBytes;
+            const int64_t a_off = a_off0 + static_cast<int64_t>(kt) * (kBM * 128);
+            if (my_rows > 0)
+              tma_load_2d_pair(st, &maps.a[my_rows / 32 - 1], 0, static_cast<int32_t>(a_off / kLine), bar, pol_a);
+            tma_load_2d_pair(st + Tr::kABytes, &maps.b, 0,
+                             static_cast<int32_t>((b_off0 + static_cast<int64_t>(kt) * (kBN * 128)) / kLine), bar,
+                             pol_w);
+            const int64_t asf_off = asf0 + static_cast<int64_t>(kt) * Tr::kSfBytes128;
             if (atoms == 4) {
-              tma_load_2d_pair(dst, &maps.bsf4, 0, static_cast<int32_t>(bsf_off / kLine), bar, pol_w);
+              tma_load_2d_pair(st + Tr::kSfaOff, &maps.asf4, 0, static_cast<int32_t>(asf_off / kLine), bar, pol_a);
             } else {
               for (int a = 0; a < atoms; ++a)
-                tma_load_2d_pair(dst + 512 * a, &maps.bsf1, 0, static_cast<int32_t>((bsf_off + 512 * a) / kLine),
-                                 bar, pol_w);
+                tma_load_2d_pair(st + Tr::kSfaOff + 512 * a, &maps.asf1, 0,
+                                 static_cast<int32_t>((asf_off + 512 * a) / kLine), bar, pol_a);
             }
-          }
-          if (++stage == kPairStages) {
-            stage = 0;
-            phase ^= 1u;
+  #pragma unroll
+            for (int h = 0; h < kBN / 128; ++h) {
+              const int64_t bsf_off = bsf0 + h * args.sf_rb_stride + static_cast<int64_t>(kt) * Tr::kSfBytes128;
+              uint8_t* dst = st + Tr::kSfbOff + h * Tr::kSfBytes128;
+              if (atoms == 4) {
+                tma_load_2d_pair(dst, &maps.bsf4, 0, static_cast<int32_t>(bsf_off / kLine), bar, pol_w);
+              } else {
+                for (int a = 0; a < atoms; ++a)
+                  tma_load_2d_pair(dst + 512 * a, &maps.bsf1, 0, static_cast<int32_t>((bsf_off + 512 * a) / kLine),
+                                   bar, pol_w);
+              }
+            }
+            if (++stage == kPairStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader)
-    if (lane == 0 && leader) {
-      int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      const uint32_t d_tmem = tmem_base;
-      for (int tile = cid; tile < total && !*abort_flag; tile += ncl) {
-        if (!mbar_wait_pair(tempty_bar, acc_phase ^ 1u, abort_flag, peer_abort)) {
-          fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
-          break;
-        }
-        tc_fence_after();
-        bool ok = true;
-        for (int kt = 0; kt < k_tiles; ++kt) {
-          if (!mbar_wait_pair(&sf_bar[stage], phase, abort_flag, peer_abort) ||
-              !mbar_wait_pair(&full_bar[stage], phase, abort_flag, peer_abort)) {
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer (leader)
+      if (lane == 0 && leader) {
+        int stage = 0;
+        uint32_t phase = 0, acc_phase = 0;
+        const uint32_t d_tmem = tmem_base;
+        for (int tile = cid; tile < total && !*abort_flag; tile += ncl) {
+          if (!mbar_wait_pair(tempty_bar, acc_phase ^ 1u, abort_flag, peer_abort)) {
             fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
-            ok = false;
             break;
           }
           tc_fence_after();
-          const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
-          const uint32_t st = smem_u32(smem + stage * Tr::kStageBytes);
-          const uint64_t adesc = make_desc_sw128(st);
-          const uint64_t bdesc = make_desc_sw128(st + Tr::kABytes);
-          const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kPairSfCols<FMT>;
-          const uint32_t sfb = sfa + Tr::kSfaCols;
-          if (FMT == MOE_NVFP4) {
-            for (int kb = 0; kb < kb_here; ++kb)
-              tc_mma_nvfp4_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_nvfp4(kBN, 2 * kBM), sfa + 4 * kb,
-                                sfb + (kBN / 32) * kb, (kt | kb) != 0 ? 1u : 0u);
-          } else {
-            for (int kb = 0; kb < kb_here; ++kb) {
-              const uint32_t sel = static_cast<uint32_t>(kb) << 30;
-              tc_mma_mxfp8_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_mxfp8(kBN, kb, 2 * kBM), sfa | sel,
-                                sfb | sel, (kt | kb) != 0 ? 1u : 0u);
+          bool ok = true;
+          for (int kt = 0; kt < k_tiles; ++kt) {
+            if (!mbar_wait_pair(&sf_bar[stage], phase, abort_flag, peer_abort) ||
+                !mbar_wait_pair(&full_bar[stage], phase, abort_flag, peer_abort)) {
+              fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
+            const uint32_t st = smem_u32(smem + stage * Tr::kStageBytes);
+            const uint64_t adesc = make_desc_sw128(st);
+            const uint64_t bdesc = make_desc_sw128(st + Tr::kABytes);
+            const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kPairSfCols<FMT>;
+            const uint32_t sfb = sfa + Tr::kSfaCols;
+            if (FMT == MOE_NVFP4) {
+              for (int kb = 0; kb < kb_here; ++kb)
+                tc_mma_nvfp4_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_nvfp4(kBN, 2 * kBM), sfa + 4 * kb,
+                                  sfb + (kBN / 32) * kb, (kt | kb) != 0 ? 1u : 0u);
+            } else {
+              for (int kb = 0; kb < kb_here; ++kb) {
+                const uint32_t sel = static_cast<uint32_t>(kb) << 30;
+                tc_mma_mxfp8_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_mxfp8(kBN, kb, 2 * kBM), sfa | sel,
+                                  sfb | sel, (kt | kb) != 0 ? 1u : 0u);
+              }
+            }
+            tc_commit_pair(&empty_bar[stage], 0x3);
+            if (++stage == kPairStages) {
+              stage = 0;
+              phase ^= 1u;
             }
           }
-          tc_commit_pair(&empty_bar[stage], 0x3);
-          if (++stage == kPairStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          if (!ok) break;
+          tc_commit_pair(tfull_bar, 0x3);
+          acc_phase ^= 1u;
         }
-        if (!ok) break;
-        tc_commit_pair(tfull_bar, 0x3);
-        acc_phase ^= 1u;
       }
-    }
-  } else if (warp >= kThreads / 32) {
-    // ------------------------------------------------------------ scale copiers (leader)
-    // Each CTA's scale atoms of every kPairCopierWarps-th k block go into its
-    // own TMEM (cta_group::2), into the stage's columns, last read by the MMAs
-    // of the same stage one ring turn ago (complete before the stage was freed
-    // and refilled, i.e. before the full barrier below completes).
-    const int part = warp - kThreads / 32;
-    if (lane == 0 && leader) {
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int tile = cid; tile < total && !*abort_flag; tile += ncl) {
-        bool ok = true;
-        for (int kt = 0; kt < k_tiles; ++kt) {
-          if (!mbar_wait_pair(&full_bar[stage], phase, abort_flag, peer_abort)) {
-            fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
-          const uint32_t st = smem_u32(smem + stage * Tr::kStageBytes);
-          const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kPairSfCols<FMT>;
-          const uint32_t sfb = sfa + Tr::kSfaCols;
-          if (FMT == MOE_NVFP4) {
-            for (int kb = part; kb < kb_here; kb += kPairCopierWarps) {
-              tc_cp_sf_atom_pair(sfa + 4 * kb, make_desc_sf(st + Tr::kSfaOff + 512 * kb));
-#pragma unroll
-              for (int h = 0; h < kBN / 128; ++h)
-                tc_cp_sf_atom_pair(sfb + (kBN / 32) * kb + 4 * h,
-                                   make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
+    } else if (warp < kPairEpiWarp0) {
+      // ------------------------------------------------------------ scale copiers (leader)
+      // Copier c moves atoms c and c + 6 of an NVFP4 stage (atom j: k block
+      // j / 3; the A atom or weight half j % 3 - 1), atom c of an MXFP8 stage,
+      // of each CTA into its own TMEM (cta_group::2), into the stage's columns,
+      // last read by the MMAs of the same stage one ring turn ago (complete
+      // before the stage was freed and refilled, i.e. before the full barrier
+      // below completes).
+      const int cp = warp - 2;
+      if (lane == 0 && leader) {
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int tile = cid; tile < total && !*abort_flag; tile += ncl) {
+          bool ok = true;
+          for (int kt = 0; kt < k_tiles; ++kt) {
+            if (!mbar_wait_pair(&full_bar[stage], phase, abort_flag, peer_abort)) {
+              fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
+              ok = false;
+              break;
             }
-          } else if (part == 0) {
-            tc_cp_sf_atom_pair(sfa, make_desc_sf(st + Tr::kSfaOff));
-            tc_cp_sf_atom_pair(sfb, make_desc_sf(st + Tr::kSfbOff));
-          } else {
-#pragma unroll
-            for (int h = 1; h < kBN / 128; ++h)
-              tc_cp_sf_atom_pair(sfb + 4 * h, make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128));
+            tc_fence_after();
+            const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
+            const uint32_t st = smem_u32(smem + stage * Tr::kStageBytes);
+            const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kPairSfCols<FMT>;
+            const uint32_t sfb = sfa + Tr::kSfaCols;
+            if (FMT == MOE_NVFP4) {
+              for (int j = cp; j < 3 * kb_here; j += kPairCopierWarps) {
+                const int kb = j / 3, m = j % 3;
+                if (m == 0)
+                  tc_cp_sf_atom_pair(sfa + 4 * kb, make_desc_sf(st + Tr::kSfaOff + 512 * kb));
+                else
+                  tc_cp_sf_atom_pair(sfb + (kBN / 32) * kb + 4 * (m - 1),
+                                     make_desc_sf(st + Tr::kSfbOff + (m - 1) * Tr::kSfBytes128 + 512 * kb));
+              }
+            } else if (cp == 0) {
+              tc_cp_sf_atom_pair(sfa, make_desc_sf(st + Tr::kSfaOff));
+            } else if (cp < 3) {
+              tc_cp_sf_atom_pair(sfb + 4 * (cp - 1), make_desc_sf(st + Tr::kSfbOff + (cp - 1) * Tr::kSfBytes128));
+            }
+            // issued, not completed: copy -> MMA is a pipelined pair (see gemm.cu)
+            tc_fence_before();
+            mbar_arrive(&sf_bar[stage]);
+            if (++stage == kPairStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          // issued, not completed: copy -> MMA is a pipelined pair (see gemm.cu)
-          tc_fence_before();
-          mbar_arrive(&sf_bar[stage]);
-          if (++stage == kPairStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          if (!ok) break;
         }
-        if (!ok) break;
       }
     }
   } else {
+    reg_alloc<kPairRegsEpilogue>();
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int half = (warp - kPairEpiWarp0) >> 2;
     const int row_l = q * 32 + lane;
     const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + half * (kBN / 2);
     const uint32_t tempty_leader = mapa_shared(smem_u32(tempty_bar), 0);
@@ -402,9 +415,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     if (leader && warp == 0 && lane == 0) {
       for (int st = 0; st < kPairStages; ++st)
         if ((armed >> st) & 1u) drained = mbar_wait_drain_cluster(&full_bar[st], (armed_par >> st) & 1u) && drained;
-    } else if (leader && (warp == 1 || warp >= kThreads / 32) && lane == 0) {
+    } else if (leader && warp >= 1 && warp < kPairEpiWarp0 && lane == 0) {
       tc_commit_pair(drain_bar, 0x1);
       drained = mbar_wait_drain_cluster(drain_bar, 0);
+    } else if (!leader && warp == 0 && lane == 0) {
+      // copies this CTA issued into a phase the leader never arrived on
+      // complete on no barrier anyone waits for: give them time to land (a
+      // bulk copy of one stage takes microseconds) before the CTA can exit
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 50000u) {
+      }
     }
     if (!drained) {
       *drain_failed = 1;
@@ -457,7 +477,7 @@ bool make_line_map(CUtensorMap* map, const void* base, int64_t bytes, int box_by
 template <int FMT, bool GATEUP>
 size_t pair_smem(int E) {
   using Tr = GemmTraits<FMT, 128, kPairStages>;
-  return 1024 + kPairStages * Tr::kStageBytes + (4 * kPairStages + 3) * 8 + 16 + 2 * (E + 1) * 4;
+  return 1024 + kPairStages * Tr::kStageBytes + (3 * kPairStages + 3) * 8 + 16 + 2 * (E + 1) * 4;
 }
 
 template <int FMT, bool GATEUP>
