@@ -200,7 +200,7 @@ moe_status moe_router_topk(const moe_config* cfg, int64_t T, const void* x_bf16,
                                 topk_w, workspace, status_word, st);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   return from_cuda(moe::route_finish(static_cast<int>(T), E, k, topk_ids, expert_counts, expert_offsets, sorted_slots,
-                                     slot_to_row, workspace, st));
+                                     slot_to_row, max_rows(cfg, T), workspace, st));
 }
 
 moe_status moe_permute(const moe_config* cfg, int64_t T, const void* x_bf16, const float* act_scale,

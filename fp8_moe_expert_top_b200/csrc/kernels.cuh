@@ -14,12 +14,16 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
 
 // The routing steps around the top-k: zero the token bitmaps and mark every
 // row of sorted_slots as padding (prepare), then per-expert counts, padded
-// offsets and the slot scatter from the bitmaps (finish).
+// offsets and the slot scatter from the bitmaps (finish).  Small batches
+// (route_small) need no prepare step and no bitmaps from the top-k: the
+// finish step builds them itself from topk_ids in one CTA.
+constexpr int kSmallWords = 8192;  // E * ceil(T / 32) bitmap words of a small batch
+bool route_small(int T, int E);
 cudaError_t route_prepare(int T, int E, int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
                           int64_t R_max, void* workspace, cudaStream_t stream);
 cudaError_t route_finish(int T, int E, int k, const int32_t* topk_ids, int32_t* expert_counts,
-                         int32_t* expert_offsets, int32_t* sorted_slots, int32_t* slot_to_row, void* workspace,
-                         cudaStream_t stream);
+                         int32_t* expert_offsets, int32_t* sorted_slots, int32_t* slot_to_row, int64_t R_max,
+                         void* workspace, cudaStream_t stream);
 
 // Router scores fused with the top-k (logits = x W_r^T on tcgen05, then the
 // same top-k, softmax and bitmaps as route_topk_kernel); E <= 512.

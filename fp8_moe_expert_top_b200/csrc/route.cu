@@ -6,8 +6,8 @@
 // section "NVFP4 and MXFP8 experts": each token is routed to 8 of 384
 // experts, with no shared expert.
 //
-// Three kernels after two small memsets (token bitmaps to zero, every row of
-// sorted_slots to -1):
+// Large batches: three kernels after two small memsets (token bitmaps to
+// zero, every row of sorted_slots to -1):
 //   1. route_topk_kernel  one warp per token, 8 tokens per CTA: top-k by k
 //      warp-wide arg-max rounds (ties to the lower index), the softmax, and
 //      bit t of the expert's token bitmap set (atomicOr, order-independent).
@@ -16,8 +16,13 @@
 //      finish scans the 128-padded counts into the expert offsets.
 //   3. route_scatter_kernel  one thread per slot: row = offset[e] +
 //      prefix[e][t/32] + (tokens before t in word t/32 that chose e).
+// Small batches (route_small: up to 512 tokens) take two kernels and no
+// memset: the top-k kernel without the bitmaps, then route_small_kernel, one
+// CTA that builds the token bitmaps in shared memory and writes the counts,
+// the padded offsets, the padding rows and the slot scatter; same results.
 // Nothing depends on thread timing, so the result is deterministic.
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -102,7 +107,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32) route_topk_kernel(const float
   if (lane < k) {
     topk_ids[static_cast<int64_t>(t) * k + lane] = my_e;
     topk_w[static_cast<int64_t>(t) * k + lane] = w;
-    atomicOr(&bitmap[static_cast<int64_t>(my_e) * W + (t >> 5)], 1u << (t & 31));
+    if (bitmap != nullptr) atomicOr(&bitmap[static_cast<int64_t>(my_e) * W + (t >> 5)], 1u << (t & 31));
   }
 }
 
@@ -220,6 +225,66 @@ __global__ void route_scatter_kernel(int T, int E, int k, int W, const int32_t* 
   slot_to_row[s] = row;
 }
 
+constexpr int kSmallThreads = 1024;
+
+// Routing steps after the top-k for a small batch, in one CTA (E <= 1024,
+// E * ceil(T / 32) <= kSmallWords): token bitmaps of every expert in shared
+// memory, per-word prefix counts, the counts, the 128-padded offsets (one
+// expert per thread, block scan), every row of sorted_slots set to -1, then
+// the scatter.  Identical results to the scan / scatter kernels.
+__global__ void __launch_bounds__(kSmallThreads) route_small_kernel(int T, int E, int k, int64_t R_max,
+                                                                    const int32_t* __restrict__ topk_ids,
+                                                                    int32_t* __restrict__ expert_counts,
+                                                                    int32_t* __restrict__ expert_offsets,
+                                                                    int32_t* __restrict__ sorted_slots,
+                                                                    int32_t* __restrict__ slot_to_row) {
+  extern __shared__ uint32_t sm_small[];
+  __shared__ int32_t warp_sums[32];
+  const int W = (T + 31) >> 5;
+  uint32_t* bm = sm_small;                                    // [E][W] token bitmaps
+  int32_t* pf = reinterpret_cast<int32_t*>(sm_small + E * W);  // [E][W] prefix counts
+  int32_t* off = pf + E * W;                                  // [E] padded offsets
+  const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  for (int i = tid; i < E * W; i += blockDim.x) bm[i] = 0u;
+  __syncthreads();
+  const int S = T * k;
+  for (int s = tid; s < S; s += blockDim.x) {
+    const int t = s / k;
+    atomicOr(&bm[topk_ids[s] * W + (t >> 5)], 1u << (t & 31));
+  }
+  __syncthreads();
+  int32_t cnt = 0;
+  if (tid < E) {
+    for (int w = 0; w < W; ++w) {
+      pf[tid * W + w] = cnt;
+      cnt += __popc(bm[tid * W + w]);
+    }
+    expert_counts[tid] = cnt;
+  }
+  int32_t total = 0;
+  const int32_t run = block_exclusive_scan(tid < E ? (cnt + 127) / 128 * 128 : 0, warp_sums, &total);
+  if (tid < E) {
+    expert_offsets[tid] = run;
+    off[tid] = run;
+  }
+  if (tid == 0) expert_offsets[E] = total;
+  for (int64_t r = tid; r < R_max; r += blockDim.x) sorted_slots[r] = -1;
+  __syncthreads();  // the padding marks land before the scatter overwrites the used rows
+  for (int s = tid; s < S; s += blockDim.x) {
+    const int t = s / k, e = topk_ids[s];
+    const int i = e * W + (t >> 5);
+    const int32_t row = off[e] + pf[i] + __popc(bm[i] & ((1u << (t & 31)) - 1u));
+    sorted_slots[row] = s;
+    slot_to_row[s] = row;
+  }
+}
+
+bool route_small(int T, int E) {
+  return T > 0 && T <= 512 && E <= kSmallThreads && static_cast<int64_t>(E) * ((T + 31) / 32) <= kSmallWords;
+}
+
 int64_t route_workspace_bytes(int E, int64_t T) {
   const int64_t W = (T + 31) / 32;
   return static_cast<int64_t>(E) * W * 8 + 256;  // bitmap words, ticket, their prefix counts
@@ -239,6 +304,7 @@ int32_t* ws_prefix(void* ws, int E, int W) {
 cudaError_t route_prepare(int T, int E, int32_t* expert_counts, int32_t* expert_offsets, int32_t* sorted_slots,
                           int64_t R_max, void* workspace, cudaStream_t stream) {
   cudaError_t err = cudaSuccess;
+  if (route_small(T, E)) return cudaSuccess;  // route_small_kernel writes everything itself
   if (R_max > 0) {
     err = cudaMemsetAsync(sorted_slots, 0xFF, static_cast<size_t>(R_max) * sizeof(int32_t), stream);
     if (err != cudaSuccess) return err;
@@ -253,9 +319,21 @@ cudaError_t route_prepare(int T, int E, int32_t* expert_counts, int32_t* expert_
 }
 
 cudaError_t route_finish(int T, int E, int k, const int32_t* topk_ids, int32_t* expert_counts,
-                         int32_t* expert_offsets, int32_t* sorted_slots, int32_t* slot_to_row, void* workspace,
-                         cudaStream_t stream) {
+                         int32_t* expert_offsets, int32_t* sorted_slots, int32_t* slot_to_row, int64_t R_max,
+                         void* workspace, cudaStream_t stream) {
   const int W = (T + 31) / 32;
+  if (route_small(T, E)) {
+    const size_t smem = static_cast<size_t>(E) * W * 8 + static_cast<size_t>(E) * 4;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+      attr_err = cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(kSmallWords * 8 + kSmallThreads * 4));
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    return launch_pdl(route_small_kernel, dim3(1), dim3(kSmallThreads), smem, stream, T, E, k, R_max, topk_ids,
+                      expert_counts, expert_offsets, sorted_slots, slot_to_row);
+  }
   const uint32_t* bitmap = static_cast<const uint32_t*>(workspace);
   int32_t* prefix = ws_prefix(workspace, E, W);
   cudaError_t err = launch_pdl(route_scan_kernel, dim3(E), dim3(kScanThreads), 0, stream, E, W, bitmap, prefix,
@@ -273,7 +351,7 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
   cudaError_t err = route_prepare(T, E, expert_counts, expert_offsets, sorted_slots, R_max, workspace, stream);
   if (err != cudaSuccess || T == 0) return err;
   const int W = (T + 31) / 32;
-  uint32_t* bitmap = static_cast<uint32_t*>(workspace);
+  uint32_t* bitmap = route_small(T, E) ? nullptr : static_cast<uint32_t*>(workspace);
   const int npl = (E + 31) / 32;
   const dim3 grid((T + kTopkWarps - 1) / kTopkWarps), block(kTopkWarps * 32);
   const float* lg = logits;
@@ -286,7 +364,8 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
   else
     err = launch_pdl(route_topk_kernel<32>, grid, block, 0, stream, lg, T, E, k, W, topk_ids, topk_w, bitmap);
   if (err != cudaSuccess) return err;
-  return route_finish(T, E, k, topk_ids, expert_counts, expert_offsets, sorted_slots, slot_to_row, workspace, stream);
+  return route_finish(T, E, k, topk_ids, expert_counts, expert_offsets, sorted_slots, slot_to_row, R_max, workspace,
+                      stream);
 }
 
 }  // namespace moe

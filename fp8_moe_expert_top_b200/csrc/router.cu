@@ -236,7 +236,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
           if (j < k) {
             args.topk_ids[o + j] = ti[j];
             args.topk_w[o + j] = __fdiv_rn(ex[j], s);
-            atomicOr(&args.bitmap[static_cast<int64_t>(ti[j]) * args.W + (t >> 5)], 1u << (t & 31));
+            if (args.bitmap != nullptr)
+              atomicOr(&args.bitmap[static_cast<int64_t>(ti[j]) * args.W + (t >> 5)], 1u << (t & 31));
           }
         }
       }
@@ -528,7 +529,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
         if (j < k && lane == j) {
           args.topk_ids[o + j] = si[j];
           args.topk_w[o + j] = __fdiv_rn(ex[j], s);
-          atomicOr(&args.bitmap[static_cast<int64_t>(si[j]) * args.W + (t >> 5)], 1u << (t & 31));
+          if (args.bitmap != nullptr)
+            atomicOr(&args.bitmap[static_cast<int64_t>(si[j]) * args.W + (t >> 5)], 1u << (t & 31));
         }
       }
     }
@@ -661,7 +663,7 @@ cudaError_t launch_router_topk(const void* x, const void* w_router, float* logit
   a.logits_out = logits_out;
   a.topk_ids = topk_ids;
   a.topk_w = topk_w;
-  a.bitmap = static_cast<uint32_t*>(workspace);
+  a.bitmap = route_small(T, E) ? nullptr : static_cast<uint32_t*>(workspace);  // small batches: no bitmaps here
   a.status = status;
   a.T = T;
   a.E = E;

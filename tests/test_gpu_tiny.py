@@ -137,11 +137,16 @@ def test_layer_edge_cases(cuda_device, wl, case):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("wl", [TINY_PREFILL, TINY_PREFILL_MX], ids=lambda w: w.name)
-@pytest.mark.parametrize("case", ["hot_experts", "empty_experts", "ragged"])
+@pytest.mark.parametrize("case", ["hot_experts", "empty_experts", "ragged", "small_route_limit", "large_route_min"])
 def test_prefill_layer_edge_cases(cuda_device, wl, case):
-    """Prefill-shaped layer with skewed routing, empty experts and a ragged batch."""
+    """Prefill-shaped layer with skewed routing, empty experts and a ragged batch;
+    512 tokens is the largest batch routed by the one-CTA small-batch path, 513
+    the smallest routed by the bitmap scan / scatter kernels."""
     layer = get_layer(wl, cuda_device)
-    if case == "hot_experts":
+    if case in ("small_route_limit", "large_route_min"):
+        T = 512 if case == "small_route_limit" else 513
+        x, lg = inputs.make_x(wl, T=T, seed=29), inputs.make_logits(wl, T=T, seed=30)
+    elif case == "hot_experts":
         x, lg = inputs.make_x(wl, seed=23), inputs.make_logits(wl, seed=24)
         lg[:, 3] += 50.0
     elif case == "empty_experts":
