@@ -182,16 +182,30 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, float* acc, 
   } else {
     const float s = (FMT == MOE_NVFP4) ? __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scales + 3 * e + 2)) : 1.0f;
     (void)I;
-    uint4* dst = reinterpret_cast<uint4*>(args.out + row * H + nt * kBN + half * (kBN / 2));
+    __nv_bfloat16* dst = args.out + row * H + nt * kBN + half * (kBN / 2);
+    if ((reinterpret_cast<uintptr_t>(args.out) & 31u) == 0u) {
+      // the row's 256 bytes as eight whole 32-byte sectors
 #pragma unroll
-    for (int i = 0; i < kBN / 16; ++i) {
-      uint32_t p[4];
+      for (int i = 0; i < kBN / 32; ++i) {
+        uint32_t p[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const __nv_bfloat162 b = __floats2bfloat162_rn(acc[8 * i + 2 * c] * s, acc[8 * i + 2 * c + 1] * s);
-        p[c] = *reinterpret_cast<const uint32_t*>(&b);
+        for (int c = 0; c < 8; ++c) {
+          const __nv_bfloat162 b = __floats2bfloat162_rn(acc[16 * i + 2 * c] * s, acc[16 * i + 2 * c + 1] * s);
+          p[c] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+        st_global_v8(dst + 16 * i, p);
       }
-      dst[i] = make_uint4(p[0], p[1], p[2], p[3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kBN / 16; ++i) {
+        uint32_t p[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const __nv_bfloat162 b = __floats2bfloat162_rn(acc[8 * i + 2 * c] * s, acc[8 * i + 2 * c + 1] * s);
+          p[c] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+        reinterpret_cast<uint4*>(dst)[i] = make_uint4(p[0], p[1], p[2], p[3]);
+      }
     }
   }
 }
