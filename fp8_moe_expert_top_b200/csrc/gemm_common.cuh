@@ -79,6 +79,20 @@ __device__ __forceinline__ int find_expert(const int32_t* offs, int E, int row) 
   return lo;
 }
 
+// Two 16-byte chunks c0, c1 of a row at logical bytes [byte, byte + 32) of the
+// tiled layout (byte a multiple of 32) in one 32-byte store: the 128-byte
+// swizzle keeps the pair in one aligned 32-byte slot, in order when the row's
+// swizzle key (row % 8) is even and swapped when it is odd.  base must be
+// 32-byte aligned.
+__device__ __forceinline__ void store_tiled32(uint8_t* base, int64_t row, int64_t byte, int64_t kb, int64_t TR,
+                                              uint4 c0, uint4 c1) {
+  const int64_t o0 = tile_offset(row, byte, kb, TR);
+  const bool swap = ((row % TR) & 1) != 0;
+  const uint4 lo = swap ? c1 : c0, hi = swap ? c0 : c1;
+  const uint32_t v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  st_global_v8(base + (swap ? o0 - 16 : o0), v);
+}
+
 // Epilogue of one accumulator row slice: acc holds columns
 // [half * kBN/2, (half + 1) * kBN/2) of row `row` (weight tile nt, expert e).
 //   gate/up: tensor scales, SwiGLU, requantization of h (NVFP4 4-vs-6 or
@@ -150,7 +164,12 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, float* acc, 
       for (int i = 0; i < 32; ++i) g[i] = __fdividef(g[i] * u[i], 1.0f + __expf(-g[i]));
     }
     // h of this thread: acc[0..32) channels ch0 + [0, 32), acc[64..96) ch0 + [32, 64)
+    // the thread's 64 channels: NVFP4 4 blocks = 32 code bytes + 4 adjacent
+    // scale bytes, MXFP8 2 blocks = 2 x 32 code bytes + 2 adjacent scale bytes
+    const bool wide = (reinterpret_cast<uintptr_t>(args.h_codes) & 31u) == 0u;
     if (FMT == MOE_NVFP4) {
+      uint32_t cw[8];
+      uint32_t sfw = 0;
 #pragma unroll 1
       for (int b = 0; b < 4; ++b) {
         float blk[16];
@@ -158,12 +177,28 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, float* acc, 
         for (int i = 0; i < 16; ++i)
           blk[i] = (b == 0) ? acc[i] : (b == 1) ? acc[16 + i] : (b == 2) ? acc[64 + i] : acc[80 + i];
         const Nvfp4Block qb = nvfp4_quantize16_h(blk, sh);
-        const int ch = ch0 + 16 * b;
-        *reinterpret_cast<uint2*>(args.h_codes + tile_offset(row, ch / 2, args.h_kb, kActTileRows)) =
-            make_uint2(static_cast<uint32_t>(qb.codes), static_cast<uint32_t>(qb.codes >> 32));
-        args.h_sf[sf_offset(row, ch / 16, I / 16)] = static_cast<uint8_t>(qb.sf);
+        const uint32_t lo = static_cast<uint32_t>(qb.codes), hi = static_cast<uint32_t>(qb.codes >> 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (j == b) {
+            cw[2 * j] = lo;
+            cw[2 * j + 1] = hi;
+          }
+        }
+        sfw |= (qb.sf & 0xFFu) << (8 * b);
+        if (!wide) {
+          const int ch = ch0 + 16 * b;
+          *reinterpret_cast<uint2*>(args.h_codes + tile_offset(row, ch / 2, args.h_kb, kActTileRows)) =
+              make_uint2(lo, hi);
+        }
       }
+      if (wide)
+        store_tiled32(args.h_codes, row, ch0 / 2, args.h_kb, kActTileRows, make_uint4(cw[0], cw[1], cw[2], cw[3]),
+                      make_uint4(cw[4], cw[5], cw[6], cw[7]));
+      // blocks ch0 / 16 .. + 3: four adjacent bytes of one scale atom row
+      *reinterpret_cast<uint32_t*>(args.h_sf + sf_offset(row, ch0 / 16, I / 16)) = sfw;
     } else {
+      uint32_t sfw = 0;
 #pragma unroll 1
       for (int b = 0; b < 2; ++b) {
         float blk[32];
@@ -172,12 +207,19 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, float* acc, 
         uint32_t w[8];
         const uint32_t ex = mxfp8_quantize32(blk, w);
         const int ch = ch0 + 32 * b;
-        *reinterpret_cast<uint4*>(args.h_codes + tile_offset(row, ch, args.h_kb, kActTileRows)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(args.h_codes + tile_offset(row, ch + 16, args.h_kb, kActTileRows)) =
-            make_uint4(w[4], w[5], w[6], w[7]);
-        args.h_sf[sf_offset(row, ch / 32, I / 32)] = static_cast<uint8_t>(ex);
+        if (wide) {
+          store_tiled32(args.h_codes, row, ch, args.h_kb, kActTileRows, make_uint4(w[0], w[1], w[2], w[3]),
+                        make_uint4(w[4], w[5], w[6], w[7]));
+        } else {
+          *reinterpret_cast<uint4*>(args.h_codes + tile_offset(row, ch, args.h_kb, kActTileRows)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(args.h_codes + tile_offset(row, ch + 16, args.h_kb, kActTileRows)) =
+              make_uint4(w[4], w[5], w[6], w[7]);
+        }
+        sfw |= (ex & 0xFFu) << (8 * b);
       }
+      // blocks ch0 / 32, + 1: two adjacent bytes of one scale atom row
+      *reinterpret_cast<uint16_t*>(args.h_sf + sf_offset(row, ch0 / 32, I / 32)) = static_cast<uint16_t>(sfw);
     }
   } else {
     const float s = (FMT == MOE_NVFP4) ? __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scales + 3 * e + 2)) : 1.0f;

@@ -84,13 +84,24 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
   } else {
     uint32_t w[8];
     const uint32_t e = mxfp8_quantize32(f, w);
+    const bool wide = (reinterpret_cast<uintptr_t>(a_codes) & 31u) == 0u;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (j >= k) break;
       const int64_t r = __ldg(slot_to_row + static_cast<int64_t>(t) * k + j);
-      *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 32 * g, kb, kActTileRows)) = make_uint4(w[0], w[1], w[2], w[3]);
-      *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 32 * g + 16, kb, kActTileRows)) =
-          make_uint4(w[4], w[5], w[6], w[7]);
+      if (wide) {
+        // the block's 32 code bytes as one store (one aligned slot under the swizzle)
+        const int64_t o0 = tile_offset(r, 32 * g, kb, kActTileRows);
+        const bool swap = ((r % kActTileRows) & 1) != 0;
+        const uint32_t v[8] = {swap ? w[4] : w[0], swap ? w[5] : w[1], swap ? w[6] : w[2], swap ? w[7] : w[3],
+                               swap ? w[0] : w[4], swap ? w[1] : w[5], swap ? w[2] : w[6], swap ? w[3] : w[7]};
+        st_global_v8(a_codes + (swap ? o0 - 16 : o0), v);
+      } else {
+        *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 32 * g, kb, kActTileRows)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(a_codes + tile_offset(r, 32 * g + 16, kb, kActTileRows)) =
+            make_uint4(w[4], w[5], w[6], w[7]);
+      }
       a_sf[sf_offset(r, g, nsf)] = static_cast<uint8_t>(e);
     }
   }
