@@ -102,10 +102,12 @@ def make_config(num_experts, top_k, d_model, d_ffn, fmt):
 def _marshal(name, stream, *tensors):
     """Device pointers of `tensors` (None stays NULL) and the stream handle.
 
-    Every tensor must be a contiguous CUDA tensor on the stream's device (the
-    current stream of the current device when `stream` is None): the library
-    takes raw device pointers, so a host tensor, a strided view or another
-    GPU's memory is refused here, before anything is enqueued.
+    Every tensor must be a contiguous CUDA tensor on the stream's device, and
+    the stream must belong to the current device (the current stream of the
+    current device when `stream` is None): the library takes raw device
+    pointers and launches on the current device, so a host tensor, a strided
+    view, another GPU's memory or another GPU's stream is refused here,
+    before anything is enqueued.
     """
     for i, t in enumerate(tensors):
         if t is None:
@@ -115,6 +117,9 @@ def _marshal(name, stream, *tensors):
         if not t.is_contiguous():
             raise ValueError(f"{name}: argument {i} is not contiguous")
     s = torch.cuda.current_stream() if stream is None else stream
+    if s.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name}: the stream is on {s.device} but the current device is "
+                         f"cuda:{torch.cuda.current_device()} (the library launches on the current device)")
     for i, t in enumerate(tensors):
         if t is not None and t.device != s.device:
             raise ValueError(f"{name}: argument {i} is on {t.device}, the stream on {s.device}")

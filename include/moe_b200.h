@@ -32,7 +32,11 @@
  *     (for example a PyTorch tensor's data_ptr()), unless stated otherwise.
  *     The library never allocates, frees or keeps device memory and keeps no
  *     pointer after a call returns.  Pointers must be 16-byte aligned.
- *   - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).
+ *   - Streams: `stream` is a cudaStream_t (NULL = legacy default stream)
+ *     of the current device, where the work is launched; a stream of
+ *     another device is not supported (moe_route_topk_noalloc refuses it
+ *     with MOE_ERR_INVALID_ARG, the Python binding refuses it for every
+ *     call).
  *     Every call only enqueues work: nothing blocks the host and nothing is
  *     copied back to the host, so the whole layer can be captured in a CUDA
  *     graph.  Device-side scalars (activation scales) are read on the device.
