@@ -192,38 +192,41 @@ __device__ __forceinline__ Nvfp4Block nvfp4_quantize16(const float* x, float s_g
 
 
 // One candidate of the 4-vs-6 search for the requantization of h in the
-// gate/up epilogue.  Same block-scale code (exact), same error terms and
-// pairwise tree as nvfp4_candidate; the element quotient is taken as
-// RN(|x| * RN(1/S)) instead of RN(|x| / S), converted two elements at a time.
-// The two quotients differ by at most 2^-23 relative, so an element code can
-// differ from the definition only where |x| / S lies that close to a
-// rounding midpoint of E2M1; the intermediate's parity bar (at most 1e-3 of
-// its codes may differ, since h itself is computed in float32 with a fast
-// exponential) absorbs that.  Zero and tiny scales take the exact path.
+// gate/up epilogue.  Same block-scale code (exact) as nvfp4_candidate; two
+// departures from the definition, both for speed in the GEMM epilogue:
+//   - the element quotient is RN(|x| * RN(1/S)) instead of RN(|x| / S),
+//     converted two elements at a time.  The two differ by at most 2^-23
+//     relative, so an element code can differ only where |x| / S lies that
+//     close to a rounding midpoint of E2M1;
+//   - the squared error is accumulated with fused multiply-adds, |x| - v S
+//     and then its square added in, even and odd elements in two running
+//     sums, instead of separately rounded products and a pairwise tree.
+//     The sum differs from the definition's in its last bits, which can
+//     change the pick only where the two candidates' errors nearly tie.
+// The intermediate's parity bar (at most 1e-3 of its codes may differ, since
+// h itself is computed in float32 with a fast exponential) absorbs both.
+// Zero and tiny scales take the exact path.
 __device__ __forceinline__ float nvfp4_candidate_h(const float* ax, float a, float s_g, float c, uint64_t& mags,
                                                    uint32_t& sf) {
   sf = e4m3_code_of_quotient(a, __fmul_rn(c, s_g));
   const float S = __fmul_rn(e4m3_decode(sf), s_g);
   if (!(S >= 0x1p-100f)) return nvfp4_candidate(ax, a, s_g, c, mags, sf);
   const float rS = __frcp_rn(S);
-  float d2[16];
-  mags = 0;
+  uint32_t mlo = 0, mhi = 0;
+  float e0 = 0.0f, e1 = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; i += 2) {
     const uint32_t p = cvt_e2m1x2(__fmul_rn(ax[i], rS), __fmul_rn(ax[i + 1], rS)) & 0x77u;
-    mags |= static_cast<uint64_t>(p) << (4 * i);
+    if (i < 8) mlo |= p << (4 * i);
+    else mhi |= p << (4 * (i - 8));
     const float2 v = e2m1x2_decode(p);
-    const float d0 = __fsub_rn(ax[i], __fmul_rn(v.x, S));
-    const float d1 = __fsub_rn(ax[i + 1], __fmul_rn(v.y, S));
-    d2[i] = __fmul_rn(d0, d0);
-    d2[i + 1] = __fmul_rn(d1, d1);
+    const float d0 = __fmaf_rn(-v.x, S, ax[i]);
+    const float d1 = __fmaf_rn(-v.y, S, ax[i + 1]);
+    e0 = __fmaf_rn(d0, d0, e0);
+    e1 = __fmaf_rn(d1, d1, e1);
   }
-#pragma unroll
-  for (int w = 8; w >= 1; w >>= 1) {
-#pragma unroll
-    for (int i = 0; i < w; ++i) d2[i] = __fadd_rn(d2[2 * i], d2[2 * i + 1]);
-  }
-  return d2[0];
+  mags = static_cast<uint64_t>(mlo) | (static_cast<uint64_t>(mhi) << 32);
+  return __fadd_rn(e0, e1);
 }
 
 // NVFP4 4-vs-6 quantization of 16 values of h (see nvfp4_candidate_h).
