@@ -420,7 +420,9 @@ def run_ours(args, wl, ws, rank, local):
 
 def time_fused_router(args, device):
     """Routing from the layer input (router scores fused with the top-k,
-    moe_router_topk) against routing from given logits (moe_route_topk), at
+    moe_router_topk) against the unfused pair (the router product by a
+    library bf16 GEMM into float32 logits, then moe_route_topk) and against
+    routing from given logits alone (moe_route_topk, no router product), at
     the decode, prefill and skewed batch sizes.  Each is one CUDA graph,
     replayed args.steps times with an L2 flush between replays; per-replay
     device time from CUDA events."""
@@ -444,7 +446,16 @@ def time_fused_router(args, device):
         g.manual_seed(inputs.BASE_SEED + 3)
         w_r = (torch.randn(E, H, generator=g, device=device) / H ** 0.5).to(torch.bfloat16)
         status = torch.zeros(1, **i32)
+        lg_mm = torch.empty(T, E, dtype=torch.float32, device=device)
+
+        def gemm_then_route():
+            # timing baseline only: a library bf16 GEMM (bf16 result, widened
+            # to float32 logits), then routing from those logits
+            lg_mm.copy_(torch.mm(x, w_r.t()))
+            B.moe_route_topk(cfg, T, lg_mm, *bufs, ws)
+
         calls = {"from_logits": lambda: B.moe_route_topk(cfg, T, lg, *bufs, ws),
+                 "gemm_then_route": gemm_then_route,
                  "fused_router": lambda: B.moe_router_topk(cfg, T, x, w_r, None, *bufs, ws, status)}
         res = {}
         for key, fn in calls.items():
@@ -471,6 +482,7 @@ def time_fused_router(args, device):
             raise RuntimeError(f"device status word {int(status.item()):#x} from the fused router")
         flops = 2.0 * T * E * H
         res["router_tflops"] = flops / (res["fused_router_ms"] * 1e-3) / 1e12
+        res["fused_vs_gemm_then_route"] = res["gemm_then_route_ms"] / res["fused_router_ms"]
         res["T"] = T
         out[name] = res
     return out

@@ -447,9 +447,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
   cluster_sync();  // every partial has arrived at its owner
   tc_fence_after();
 
-  if (warp >= 2) {
-    // reduce the owned rows over the KS partials, then top-k (a warp per row)
-    for (int r_loc = warp - 2; r_loc < RPO; r_loc += kREpiWarps) {
+  {
+    // reduce the owned rows over the KS partials, then top-k (a warp per row,
+    // every warp of the CTA)
+    for (int r_loc = warp; r_loc < RPO; r_loc += kRThreads / 32) {
       const int t = m0 + static_cast<int>(rank) * RPO + r_loc;
       if (t >= args.T) break;
       float tv[8];
@@ -633,21 +634,23 @@ template <int NB>
 cudaError_t launch_any(const CUtensorMap& mx, const CUtensorMap& mw, const RouterArgs& a, int ks,
                        cudaStream_t stream) {
   switch (ks) {
-    case 2: return launch_split<NB, 2>(mx, mw, a, stream);
     case 4: return launch_split<NB, 4>(mx, mw, a, stream);
     case 8: return launch_split<NB, 8>(mx, mw, a, stream);
     default: return launch_nb<NB>(mx, mw, a, stream);
   }
 }
 
-// K split of the scores: the largest of 8, 4, 2 that divides the k tiles and
-// keeps the clusters within one wave of CTAs (148 SMs, one CTA each); 1 (no
-// split) for large batches and for 512 experts, whose receive slots would not
-// fit in the ring.
+// K split of the scores: 8 or 4 (each owner CTA ranking at most 32 rows) when
+// it divides the k tiles and keeps the clusters within one wave of CTAs (148
+// SMs, one CTA each); 1 (no split) for larger batches, where the unsplit
+// kernel already fills the GPU and a 2-way split's per-row ranking costs more
+// than it saves (measured: 101 us for 8192 tokens split in two against 73 us
+// unsplit for 16384), and for 512 experts, whose receive slots would not fit
+// in the ring.
 int router_split(int T, int H, int nb) {
   if (nb > 3) return 1;
   const int m = (T + kRM - 1) / kRM, kt = H / kRKElems;
-  for (int ks = 8; ks >= 2; ks >>= 1)
+  for (int ks = 8; ks >= 4; ks >>= 1)
     if (kt % ks == 0 && m * ks <= 148) return ks;
   return 1;
 }

@@ -253,9 +253,9 @@ MOE_API moe_status moe_route_topk(const moe_config* cfg, int64_t T, const float*
  * Supported: num_experts <= 512 (MOE_ERR_UNSUPPORTED otherwise).  The
  * float32 sums are taken in the tensor core's order, so a score can differ
  * from the exactly rounded sum in its last bits; results do not depend on
- * thread timing.  Batches of up to 74 tiles of 128 tokens (with at most 384
- * experts) split d_model over a cluster of 2, 4 or 8 CTAs per tile and add
- * the partial sums, on chip, in cluster-rank order. */
+ * thread timing.  Batches of up to 37 tiles of 128 tokens (with at most 384
+ * experts) split d_model over a cluster of 4 or 8 CTAs per tile and add the
+ * partial sums, on chip, in cluster-rank order. */
 MOE_API moe_status moe_router_topk(const moe_config* cfg, int64_t T, const void* x_bf16, const void* w_router_bf16,
                                    float* logits_out, int32_t* topk_ids, float* topk_w, int32_t* expert_counts,
                                    int32_t* expert_offsets, int32_t* sorted_slots, int32_t* slot_to_row,

@@ -35,9 +35,9 @@ from oracle import route as ort
 
 # (T, E, H, k): tiny, one token, a ragged batch at the model's size, experts
 # not a multiple of 128, the 512-expert limit (two-stage ring), several tiles.
-# Batches of up to 74 row tiles split K over clusters of 2-8 CTAs; the
-# 512-expert case and the 9600-token case (75 row tiles) take the unsplit
-# kernel.
+# Batches of up to 37 row tiles split K over clusters of 4 or 8 CTAs (the
+# first four cases and 777 tokens: 8; 64 and 129 tokens at d_model 256: 4);
+# the 512-expert case and the 9600-token case take the unsplit kernel.
 GRID_CASES = [(64, 8, 256, 2), (1, 384, 4096, 8), (777, 384, 4096, 8), (300, 200, 512, 6), (256, 512, 1024, 8),
               (129, 128, 256, 1), (9600, 384, 512, 8)]
 
