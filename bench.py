@@ -247,6 +247,18 @@ def phase_bytes(wl, n_touched, slots):
 PHASES = ("route", "permute", "gateup", "down", "combine")
 
 
+def kernels_per_step(wl, T):
+    """The library's kernel launches in one layer step: routing (top-k, then
+    scan and scatter, or for batches of up to 512 tokens with at most 8192
+    bitmap words one small-batch kernel), permute, gate/up (BF16: with the
+    two adapter shrinks before and after it), down, combine."""
+    W = (T + 31) // 32
+    small = 0 < T <= 512 and wl.num_experts <= 1024 and wl.num_experts * W <= 8192
+    route = 2 if small else 3
+    gateup = 3 if wl.fmt == inputs.BF16 else 1
+    return route + 1 + gateup + 1 + 1
+
+
 def run_ours(args, wl, ws, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
@@ -410,9 +422,7 @@ def run_ours(args, wl, ws, rank, local):
                 "overlap": "HostPipeline: step i+1's upload and step i-1's download overlap step i "
                            "(two graphs, upload and download streams); no L2 flush, each step streams "
                            "GBs of weights"},
-        # per step: route top-k, scan, scatter; permute; gate/up; down; combine
-        # (BF16: and the two adapter shrinks)
-        "gpu_launches": (9 if wl.fmt == inputs.BF16 else 7) * args.steps,
+        "gpu_launches": kernels_per_step(wl, T) * args.steps,
         "clocks": clk,
     }
     return out, layer
@@ -577,7 +587,7 @@ def run_depth(args, local, n_nv, n_mx):
         "stack_roofline_frac": (layer_bytes / (peaks["hbm_gbs"] * 1e9)) / (ms * 1e-3),
         "ms_per_layer": ms / (n_nv + n_mx),
         "step_ms_pct": {"p10": pct(step_ms, 10), "p50": pct(step_ms, 50), "p90": pct(step_ms, 90)},
-        "gpu_launches": 7 * (n_nv + n_mx) * args.steps,
+        "gpu_launches": (n_nv * kernels_per_step(wl_n, T) + n_mx * kernels_per_step(wl_m, T)) * args.steps,
         "clocks": clk,
     }
 
