@@ -69,8 +69,19 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
     }
   } else if (FMT == MOE_NVFP4) {
     const float s_x = __ldg(act_scale);
-    const Nvfp4Block q0 = nvfp4_quantize16(f, s_x);
-    const Nvfp4Block q1 = nvfp4_quantize16(f + 16, s_x);
+    // both blocks through one copy of the quantizer's code: the kernel is
+    // bound by its instruction stream, and two inlined copies measured 6-10%
+    // slower (instruction-cache misses)
+    Nvfp4Block q0, q1;
+#pragma unroll 1
+    for (int b = 0; b < 2; ++b) {
+      float blk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) blk[i] = b ? f[16 + i] : f[i];
+      const Nvfp4Block q = nvfp4_quantize16(blk, s_x);
+      if (b == 0) q0 = q;
+      else q1 = q;
+    }
     const uint4 c = make_uint4(static_cast<uint32_t>(q0.codes), static_cast<uint32_t>(q0.codes >> 32),
                                static_cast<uint32_t>(q1.codes), static_cast<uint32_t>(q1.codes >> 32));
     const uint16_t sf = static_cast<uint16_t>(q0.sf | (q1.sf << 8));
