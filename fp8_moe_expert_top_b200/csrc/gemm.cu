@@ -211,6 +211,12 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       const uint32_t d_tmem = tmem_base;
+      // Descriptors of stage 0; a stage adds kStageDesc 16-byte units (the
+      // 14-bit start field never carries: shared memory is below 256 KB).
+      const uint64_t adesc0 = make_desc_sw128(smem_u32(smem));
+      const uint64_t bdesc0 = make_desc_sw128(smem_u32(smem) + Tr::kABytes);
+      constexpr uint32_t kStageDesc = Tr::kStageBytes >> 4;
+      const int full_stages = args.K / Tr::kElemsPerStage;  // stages with all 4 k blocks
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
         if (!mbar_wait(tempty_bar, acc_phase ^ 1u, abort_flag)) {
           fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
@@ -228,25 +234,43 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
             break;
           }
           tc_fence_after();
-          const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
-          const uint32_t st = smem_u32(smem + stage * Tr::kStageBytes);
-          const uint64_t adesc = make_desc_sw128(st);
-          const uint64_t bdesc = make_desc_sw128(st + Tr::kABytes);
+          // The issuing thread's own instruction latency is on the tensor
+          // pipe's critical path: whole stages issue their four MMAs
+          // unrolled, with operands computed independently of each other.
+          const uint64_t adesc = adesc0 + static_cast<uint64_t>(stage) * kStageDesc;
+          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(stage) * kStageDesc;
           const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kSfColsPerStage<FMT>;
           const uint32_t sfb = sfa + Tr::kSfaCols;
-          if (FMT == MOE_BF16) {
-            for (int kb = 0; kb < kb_here; ++kb)
-              tc_mma_bf16(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_bf16(kBN), (kt | kb) != 0 ? 1u : 0u);
-          } else if (FMT == MOE_NVFP4) {
-            for (int kb = 0; kb < kb_here; ++kb) {
-              tc_mma_nvfp4(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_nvfp4(kBN), sfa + 4 * kb,
-                           sfb + (kBN / 32) * kb, (kt | kb) != 0 ? 1u : 0u);
+          const uint32_t acc0 = kt != 0 ? 1u : 0u;
+          if (kt < full_stages) {
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+              const uint32_t accum = kb != 0 ? 1u : acc0;
+              if (FMT == MOE_BF16) {
+                tc_mma_bf16(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_bf16(kBN), accum);
+              } else if (FMT == MOE_NVFP4) {
+                tc_mma_nvfp4(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_nvfp4(kBN), sfa + 4 * kb,
+                             sfb + (kBN / 32) * kb, accum);
+              } else {
+                const uint32_t sel = static_cast<uint32_t>(kb) << 30;
+                tc_mma_mxfp8(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_mxfp8(kBN, kb), sfa | sel, sfb | sel,
+                             accum);
+              }
             }
           } else {
+            const int kb_here = (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK;
             for (int kb = 0; kb < kb_here; ++kb) {
-              const uint32_t sel = static_cast<uint32_t>(kb) << 30;
-              tc_mma_mxfp8(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_mxfp8(kBN, kb), sfa | sel, sfb | sel,
-                           (kt | kb) != 0 ? 1u : 0u);
+              const uint32_t accum = kb != 0 ? 1u : acc0;
+              if (FMT == MOE_BF16) {
+                tc_mma_bf16(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_bf16(kBN), accum);
+              } else if (FMT == MOE_NVFP4) {
+                tc_mma_nvfp4(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_nvfp4(kBN), sfa + 4 * kb,
+                             sfb + (kBN / 32) * kb, accum);
+              } else {
+                const uint32_t sel = static_cast<uint32_t>(kb) << 30;
+                tc_mma_mxfp8(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc_mxfp8(kBN, kb), sfa | sel, sfb | sel,
+                             accum);
+              }
             }
           }
           tc_commit(&empty_bar[stage]);
@@ -266,6 +290,11 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
     if (lane == 0 && Tr::kScaled) {
       int stage = 0;
       uint32_t phase = 0;
+      // scale-atom descriptor of stage 0's A scales; every other atom is a
+      // constant number of 16-byte units away
+      const uint64_t sdesc0 = make_desc_sf(smem_u32(smem) + Tr::kSfaOff);
+      constexpr uint32_t kStageDesc = Tr::kStageBytes >> 4;
+      const int full_stages = args.K / Tr::kElemsPerStage;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
         bool ok = true;
         for (int kt = 0; kt < k_tiles; ++kt) {
@@ -278,25 +307,27 @@ __global__ void __launch_bounds__(kThreadsOne, 1)
             break;
           }
           tc_fence_after();
-          const int kb_here = min(4, (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK);
-          const uint32_t st = smem_u32(smem + stage * Tr::kStageBytes);
+          const uint64_t sdesc = sdesc0 + static_cast<uint64_t>(stage) * kStageDesc;  // this stage's A atom 0
+          constexpr uint32_t kSfbDesc = (Tr::kSfbOff - Tr::kSfaOff) >> 4;
+          constexpr uint32_t kAtomDesc = 512 >> 4;
           const uint32_t sfa = tmem_base + Tr::kTmemSfa + stage * kSfColsPerStage<FMT>;
           const uint32_t sfb = sfa + Tr::kSfaCols;
           if (FMT == MOE_NVFP4) {
+            // this warp's k blocks part, part + kCopierWarps, ...
+            const int kb_here = kt < full_stages ? 4 : (args.K - kt * Tr::kElemsPerStage) / Tr::kMmaK;
             for (int kb = part; kb < kb_here; kb += kCopierWarps) {
-              tc_cp_sf_atom(sfa + 4 * kb, make_desc_sf(st + Tr::kSfaOff + 512 * kb));
+              tc_cp_sf_atom(sfa + 4 * kb, sdesc + kAtomDesc * kb);
 #pragma unroll
               for (int h = 0; h < kBN / 128; ++h)
                 tc_cp_sf_atom(sfb + (kBN / 32) * kb + 4 * h,
-                              make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128 + 512 * kb));
+                              sdesc + kSfbDesc + h * (Tr::kSfBytes128 >> 4) + kAtomDesc * kb);
             }
           } else if (part == 0) {
-            tc_cp_sf_atom(sfa, make_desc_sf(st + Tr::kSfaOff));
-            tc_cp_sf_atom(sfb, make_desc_sf(st + Tr::kSfbOff));
+            tc_cp_sf_atom(sfa, sdesc);
+            tc_cp_sf_atom(sfb, sdesc + kSfbDesc);
           } else {
 #pragma unroll
-            for (int h = 1; h < kBN / 128; ++h)
-              tc_cp_sf_atom(sfb + 4 * h, make_desc_sf(st + Tr::kSfbOff + h * Tr::kSfBytes128));
+            for (int h = 1; h < kBN / 128; ++h) tc_cp_sf_atom(sfb + 4 * h, sdesc + kSfbDesc + h * (Tr::kSfBytes128 >> 4));
           }
           // Signal that the copies are issued, not that they are complete:
           // tcgen05.cp -> tcgen05.mma is a pipelined pair, so the MMA
