@@ -140,6 +140,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, float* acc, 
     const float sg = (FMT == MOE_NVFP4) ? __fmul_rn(sa, __ldg(args.w_scales + 3 * e + 0)) : 1.0f;
     const float su = (FMT == MOE_NVFP4) ? __fmul_rn(sa, __ldg(args.w_scales + 3 * e + 1)) : 1.0f;
     const float sh = (FMT == MOE_NVFP4) ? __ldg(args.h_scale) : 1.0f;
+    const HScale hs = make_hscale(sh);
 #pragma unroll
     for (int j = 0; j < kBN / 128; ++j) {
       float* g = acc + 64 * j;
@@ -171,25 +172,28 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, float* acc, 
       uint32_t cw[8];
       uint32_t sfw = 0;
 #pragma unroll 1
-      for (int b = 0; b < 4; ++b) {
-        float blk[16];
+      for (int b2 = 0; b2 < 2; ++b2) {
+        float blk[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          blk[i] = (b == 0) ? acc[i] : (b == 1) ? acc[16 + i] : (b == 2) ? acc[64 + i] : acc[80 + i];
-        const Nvfp4Block qb = nvfp4_quantize16_h(blk, sh);
-        const uint32_t lo = static_cast<uint32_t>(qb.codes), hi = static_cast<uint32_t>(qb.codes >> 32);
+        for (int i = 0; i < 32; ++i) blk[i] = (b2 == 0) ? acc[i] : acc[64 + i];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (j == b) {
-            cw[2 * j] = lo;
-            cw[2 * j + 1] = hi;
+        for (int jb = 0; jb < 2; ++jb) {
+          const int b = 2 * b2 + jb;
+          const Nvfp4Block qb = nvfp4_quantize16_h(blk + 16 * jb, hs);
+          const uint32_t lo = static_cast<uint32_t>(qb.codes), hi = static_cast<uint32_t>(qb.codes >> 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j == b) {
+              cw[2 * j] = lo;
+              cw[2 * j + 1] = hi;
+            }
           }
-        }
-        sfw |= (qb.sf & 0xFFu) << (8 * b);
-        if (!wide) {
-          const int ch = ch0 + 16 * b;
-          *reinterpret_cast<uint2*>(args.h_codes + tile_offset(row, ch / 2, args.h_kb, kActTileRows)) =
-              make_uint2(lo, hi);
+          sfw |= (qb.sf & 0xFFu) << (8 * b);
+          if (!wide) {
+            const int ch = ch0 + 16 * b;
+            *reinterpret_cast<uint2*>(args.h_codes + tile_offset(row, ch / 2, args.h_kb, kActTileRows)) =
+                make_uint2(lo, hi);
+          }
         }
       }
       if (wide)

@@ -92,14 +92,18 @@ static __device__ __noinline__ uint32_t e4m3_code_exact(float num, float den) {
   return e4m3_encode(__fdiv_rn(num, den));
 }
 
-// E4M3 code of RN(num / den), num >= 0, den > 0.
-__device__ __forceinline__ uint32_t e4m3_code_of_quotient(float num, float den) {
+// E4M3 code of RN(num / den), num >= 0, den > 0, given rden = RN(1 / den).
+__device__ __forceinline__ uint32_t e4m3_code_of_quotient_r(float num, float den, float rden) {
   if (num == 0.0f) return 0u;
-  const float q = __fmul_rn(num, __frcp_rn(den));
+  const float q = __fmul_rn(num, rden);
   const uint32_t pair = cvt_e4m3x2(__fmul_rn(q, kBracketLo), __fmul_rn(q, kBracketHi));
   const uint32_t lo = pair & 0xFFu, hi = pair >> 8;
   if (lo == hi) return lo;
   return e4m3_code_exact(num, den);
+}
+// E4M3 code of RN(num / den), num >= 0, den > 0.
+__device__ __forceinline__ uint32_t e4m3_code_of_quotient(float num, float den) {
+  return e4m3_code_of_quotient_r(num, den, __frcp_rn(den));
 }
 
 // Two E2M1 codes (element 2j in the low nibble) decoded to float (exact).
@@ -191,9 +195,9 @@ __device__ __forceinline__ Nvfp4Block nvfp4_quantize16(const float* x, float s_g
 }
 
 
-// One candidate of the 4-vs-6 search for the requantization of h in the
-// gate/up epilogue.  Same block-scale code (exact) as nvfp4_candidate; two
-// departures from the definition, both for speed in the GEMM epilogue:
+// The 4-vs-6 search for the requantization of h in the gate/up epilogue.
+// Same block-scale codes (exact) as nvfp4_candidate; two departures from the
+// definition, both for speed in the GEMM epilogue:
 //   - the element quotient is RN(|x| * RN(1/S)) instead of RN(|x| / S),
 //     converted two elements at a time.  The two differ by at most 2^-23
 //     relative, so an element code can differ only where |x| / S lies that
@@ -206,49 +210,83 @@ __device__ __forceinline__ Nvfp4Block nvfp4_quantize16(const float* x, float s_g
 // The intermediate's parity bar (at most 1e-3 of its codes may differ, since
 // h itself is computed in float32 with a fast exponential) absorbs both.
 // Zero and tiny scales take the exact path.
-__device__ __forceinline__ float nvfp4_candidate_h(const float* ax, float a, float s_g, float c, uint64_t& mags,
-                                                   uint32_t& sf) {
-  sf = e4m3_code_of_quotient(a, __fmul_rn(c, s_g));
-  const float S = __fmul_rn(e4m3_decode(sf), s_g);
-  if (!(S >= 0x1p-100f)) return nvfp4_candidate(ax, a, s_g, c, mags, sf);
+//
+// The signed values go through the conversion as they are: rounding is
+// symmetric in sign, so the magnitude code, x - v S and its square are those
+// of |x| and the conversion supplies the sign bit (cleared afterwards where
+// the magnitude is zero).
+
+// Per-thread constants of the h tensor scale s_g: the reciprocals of both
+// candidates' scale denominators RN(c s_g), c = 6 and 4.
+struct HScale {
+  float s_g, rd6, rd4;
+};
+__device__ __forceinline__ HScale make_hscale(float s_g) {
+  HScale h;
+  h.s_g = s_g;
+  h.rd6 = __frcp_rn(__fmul_rn(6.0f, s_g));
+  h.rd4 = __frcp_rn(__fmul_rn(4.0f, s_g));
+  return h;
+}
+
+// One candidate with a normal scale S: signed codes (element i in bits
+// [4i, 4i+4)) and the squared error.
+__device__ __forceinline__ float nvfp4_candidate_hs(const float* x, float S, uint64_t& codes) {
   const float rS = __frcp_rn(S);
-  uint32_t mlo = 0, mhi = 0;
+  uint32_t clo = 0, chi = 0;
   float e0 = 0.0f, e1 = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; i += 2) {
-    const uint32_t p = cvt_e2m1x2(__fmul_rn(ax[i], rS), __fmul_rn(ax[i + 1], rS)) & 0x77u;
-    if (i < 8) mlo |= p << (4 * i);
-    else mhi |= p << (4 * (i - 8));
+    const uint32_t p = cvt_e2m1x2(__fmul_rn(x[i], rS), __fmul_rn(x[i + 1], rS));
+    if (i < 8) clo |= p << (4 * i);
+    else chi |= p << (4 * (i - 8));
     const float2 v = e2m1x2_decode(p);
-    const float d0 = __fmaf_rn(-v.x, S, ax[i]);
-    const float d1 = __fmaf_rn(-v.y, S, ax[i + 1]);
+    const float d0 = __fmaf_rn(-v.x, S, x[i]);
+    const float d1 = __fmaf_rn(-v.y, S, x[i + 1]);
     e0 = __fmaf_rn(d0, d0, e0);
     e1 = __fmaf_rn(d1, d1, e1);
   }
-  mags = static_cast<uint64_t>(mlo) | (static_cast<uint64_t>(mhi) << 32);
+  codes = static_cast<uint64_t>(clo) | (static_cast<uint64_t>(chi) << 32);
   return __fadd_rn(e0, e1);
 }
 
-// NVFP4 4-vs-6 quantization of 16 values of h (see nvfp4_candidate_h).
-__device__ __forceinline__ Nvfp4Block nvfp4_quantize16_h(const float* x, float s_g) {
+// One candidate with a zero or tiny scale: the exact path on |x|, with the
+// sign bits of the negative elements added.
+__device__ __forceinline__ float nvfp4_candidate_h_exact(const float* x, float a, float s_g, float c,
+                                                         uint64_t& codes) {
   float ax[16];
-  float a = 0.0f;
   uint64_t neg = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     ax[i] = fabsf(x[i]);
-    a = fmaxf(a, ax[i]);
     neg |= static_cast<uint64_t>(x[i] < 0.0f) << (4 * i + 3);
   }
-  uint64_t m6, m4;
-  uint32_t e6, e4;
-  const float err6 = nvfp4_candidate_h(ax, a, s_g, 6.0f, m6, e6);
-  const float err4 = nvfp4_candidate_h(ax, a, s_g, 4.0f, m4, e4);
+  uint64_t mags;
+  uint32_t sf;
+  const float err = nvfp4_candidate(ax, a, s_g, c, mags, sf);
+  codes = mags | neg;
+  return err;
+}
+
+// NVFP4 4-vs-6 quantization of 16 values of h.
+__device__ __forceinline__ Nvfp4Block nvfp4_quantize16_h(const float* x, const HScale& hs) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
+  const uint32_t e6 = e4m3_code_of_quotient_r(a, __fmul_rn(6.0f, hs.s_g), hs.rd6);
+  const uint32_t e4 = e4m3_code_of_quotient_r(a, __fmul_rn(4.0f, hs.s_g), hs.rd4);
+  const float S6 = __fmul_rn(e4m3_decode(e6), hs.s_g);
+  const float S4 = __fmul_rn(e4m3_decode(e4), hs.s_g);
+  uint64_t c6, c4;
+  const float err6 = (S6 >= 0x1p-100f) ? nvfp4_candidate_hs(x, S6, c6) : nvfp4_candidate_h_exact(x, a, hs.s_g, 6.0f, c6);
+  const float err4 = (S4 >= 0x1p-100f) ? nvfp4_candidate_hs(x, S4, c4) : nvfp4_candidate_h_exact(x, a, hs.s_g, 4.0f, c4);
   const bool four = err4 < err6;
-  const uint64_t mags = four ? m4 : m6;
+  const uint64_t codes = four ? c4 : c6;
+  // sign bit only where the magnitude code is non-zero (canonical +0)
+  const uint64_t mags = codes & 0x7777777777777777ull;
   const uint64_t nz = (mags | (mags >> 1) | (mags >> 2)) & 0x1111111111111111ull;
   Nvfp4Block b;
-  b.codes = mags | (neg & (nz << 3));
+  b.codes = mags | (codes & (nz << 3));
   b.sf = four ? e4 : e6;
   return b;
 }
