@@ -140,7 +140,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, float* acc, 
     const float sg = (FMT == MOE_NVFP4) ? __fmul_rn(sa, __ldg(args.w_scales + 3 * e + 0)) : 1.0f;
     const float su = (FMT == MOE_NVFP4) ? __fmul_rn(sa, __ldg(args.w_scales + 3 * e + 1)) : 1.0f;
     const float sh = (FMT == MOE_NVFP4) ? __ldg(args.h_scale) : 1.0f;
-    const HScale hs = make_hscale(sh);
+    const Nvfp4Scale hs = make_nvfp4_scale(sh);
 #pragma unroll
     for (int j = 0; j < kBN / 128; ++j) {
       float* g = acc + 64 * j;

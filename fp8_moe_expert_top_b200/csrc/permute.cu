@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
   for (int i = 0; i < G / 16; ++i) load16_bf16(x + static_cast<int64_t>(t) * H + G * g + 16 * i, f + 16 * i);
   const int64_t kb = kb_padded(H, FMT == MOE_NVFP4 ? 4 : 8);
   if (FMT == MOE_NVFP4 && G == 16) {
-    const Nvfp4Block q = nvfp4_quantize16(f, __ldg(act_scale));
+    const Nvfp4Block q = nvfp4_quantize16(f, make_nvfp4_scale(__ldg(act_scale)));
     const uint2 c = make_uint2(static_cast<uint32_t>(q.codes), static_cast<uint32_t>(q.codes >> 32));
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(256) permute_kernel(int T, int H, int k, const
       a_sf[sf_offset(r, g, nsf)] = static_cast<uint8_t>(q.sf);
     }
   } else if (FMT == MOE_NVFP4) {
-    const float s_x = __ldg(act_scale);
+    const Nvfp4Scale s_x = make_nvfp4_scale(__ldg(act_scale));
     // both blocks through one copy of the quantizer's code: the kernel is
     // bound by its instruction stream, and two inlined copies measured 6-10%
     // slower (instruction-cache misses)

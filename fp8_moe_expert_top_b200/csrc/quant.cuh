@@ -115,6 +115,19 @@ __device__ __forceinline__ float2 e2m1x2_decode(uint32_t pair) {
   return __half22float2(*reinterpret_cast<const __half2*>(&h2));
 }
 
+// Per-thread constants of a tensor scale s_g: the reciprocals of both
+// candidates' scale denominators RN(c s_g), c = 6 and 4.
+struct Nvfp4Scale {
+  float s_g, rd6, rd4;
+};
+__device__ __forceinline__ Nvfp4Scale make_nvfp4_scale(float s_g) {
+  Nvfp4Scale t;
+  t.s_g = s_g;
+  t.rd6 = __frcp_rn(__fmul_rn(6.0f, s_g));
+  t.rd4 = __frcp_rn(__fmul_rn(4.0f, s_g));
+  return t;
+}
+
 // One candidate of the 4-vs-6 search on magnitudes ax[16] (block maximum a
 // mapped to c).  Returns the squared error; mags receives the 3-bit
 // magnitude codes (element i in bits [4i, 4i+4)), sf the scale code.
@@ -169,31 +182,94 @@ __device__ __forceinline__ float nvfp4_candidate(const float* ax, float a, float
   return d2[0];
 }
 
-// NVFP4 4-vs-6 quantization of 16 float32 values with tensor scale s_g > 0.
-__device__ __forceinline__ Nvfp4Block nvfp4_quantize16(const float* x, float s_g) {
+// One candidate with a zero or tiny scale: nvfp4_candidate on |x|, with the
+// sign bits of the negative elements added.
+__device__ __forceinline__ float nvfp4_candidate_tiny(const float* x, float a, float s_g, float c, uint64_t& codes) {
   float ax[16];
-  float a = 0.0f;
   uint64_t neg = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     ax[i] = fabsf(x[i]);
-    a = fmaxf(a, ax[i]);
     neg |= static_cast<uint64_t>(x[i] < 0.0f) << (4 * i + 3);
   }
-  uint64_t m6, m4;
-  uint32_t e6, e4;
-  const float err6 = nvfp4_candidate(ax, a, s_g, 6.0f, m6, e6);
-  const float err4 = nvfp4_candidate(ax, a, s_g, 4.0f, m4, e4);
+  uint64_t mags;
+  uint32_t sf;
+  const float err = nvfp4_candidate(ax, a, s_g, c, mags, sf);
+  codes = mags | neg;
+  return err;
+}
+
+// One candidate on the signed values x (the exact definition): rounding is
+// symmetric in sign, so the magnitude codes, x - v S and its square are those
+// of |x|, and the conversion supplies each element's sign bit (cleared by the
+// caller where the magnitude is zero).  Zero and tiny scales take
+// nvfp4_candidate on |x|.
+__device__ __forceinline__ float nvfp4_candidate_s(const float* x, float a, float s_g, float c, float rden,
+                                                   uint64_t& codes, uint32_t& sf) {
+  sf = e4m3_code_of_quotient_r(a, __fmul_rn(c, s_g), rden);
+  const float S = __fmul_rn(e4m3_decode(sf), s_g);
+  if (!(S >= 0x1p-100f)) return nvfp4_candidate_tiny(x, a, s_g, c, codes);
+  const float rS = __frcp_rn(S);
+  float d2[16];
+  uint32_t clo = 0, chi = 0;
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    // both ends of both elements' brackets, two elements per conversion
+    const float q0 = __fmul_rn(x[i], rS), q1 = __fmul_rn(x[i + 1], rS);
+    const uint32_t lo = cvt_e2m1x2(__fmul_rn(q0, kBracketLo), __fmul_rn(q1, kBracketLo));
+    const uint32_t hi = cvt_e2m1x2(__fmul_rn(q0, kBracketHi), __fmul_rn(q1, kBracketHi));
+    uint32_t p = lo;
+    if (lo != hi) {  // an end differs (never the sign): settle that element by the exact division
+      const uint32_t m0 = ((lo ^ hi) & 0x7u) ? (e2m1_code_exact(fabsf(x[i]), S) | (lo & 0x8u)) : (lo & 0xFu);
+      const uint32_t m1 =
+          ((lo ^ hi) & 0x70u) ? ((e2m1_code_exact(fabsf(x[i + 1]), S) << 4) | (lo & 0x80u)) : (lo & 0xF0u);
+      p = m0 | m1;
+    }
+    if (i < 8) clo |= p << (4 * i);
+    else chi |= p << (4 * (i - 8));
+    const float2 v = e2m1x2_decode(p);
+    const float d0 = __fsub_rn(x[i], __fmul_rn(v.x, S));
+    const float d1 = __fsub_rn(x[i + 1], __fmul_rn(v.y, S));
+    d2[i] = __fmul_rn(d0, d0);
+    d2[i + 1] = __fmul_rn(d1, d1);
+  }
+  codes = static_cast<uint64_t>(clo) | (static_cast<uint64_t>(chi) << 32);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) d2[i] = __fadd_rn(d2[2 * i], d2[2 * i + 1]);
+  }
+  return d2[0];
+}
+
+// Signed codes -> block: the lower-error candidate (ties to 6), with the sign
+// bit kept only where the magnitude code is non-zero (canonical +0).
+__device__ __forceinline__ Nvfp4Block nvfp4_pick(float err6, uint64_t c6, uint32_t e6, float err4, uint64_t c4,
+                                                 uint32_t e4) {
   const bool four = err4 < err6;
-  const uint64_t mags = four ? m4 : m6;
-  // sign bit only where the magnitude code is non-zero (canonical +0)
+  const uint64_t codes = four ? c4 : c6;
+  const uint64_t mags = codes & 0x7777777777777777ull;
   const uint64_t nz = (mags | (mags >> 1) | (mags >> 2)) & 0x1111111111111111ull;
   Nvfp4Block b;
-  b.codes = mags | (neg & (nz << 3));
+  b.codes = mags | (codes & (nz << 3));
   b.sf = four ? e4 : e6;
   return b;
 }
 
+// NVFP4 4-vs-6 quantization of 16 float32 values with tensor scale s_g > 0.
+__device__ __forceinline__ Nvfp4Block nvfp4_quantize16(const float* x, const Nvfp4Scale& ts) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
+  uint64_t c6, c4;
+  uint32_t e6, e4;
+  const float err6 = nvfp4_candidate_s(x, a, ts.s_g, 6.0f, ts.rd6, c6, e6);
+  const float err4 = nvfp4_candidate_s(x, a, ts.s_g, 4.0f, ts.rd4, c4, e4);
+  return nvfp4_pick(err6, c6, e6, err4, c4, e4);
+}
+__device__ __forceinline__ Nvfp4Block nvfp4_quantize16(const float* x, float s_g) {
+  return nvfp4_quantize16(x, make_nvfp4_scale(s_g));
+}
 
 // The 4-vs-6 search for the requantization of h in the gate/up epilogue.
 // Same block-scale codes (exact) as nvfp4_candidate; two departures from the
@@ -216,19 +292,6 @@ __device__ __forceinline__ Nvfp4Block nvfp4_quantize16(const float* x, float s_g
 // of |x| and the conversion supplies the sign bit (cleared afterwards where
 // the magnitude is zero).
 
-// Per-thread constants of the h tensor scale s_g: the reciprocals of both
-// candidates' scale denominators RN(c s_g), c = 6 and 4.
-struct HScale {
-  float s_g, rd6, rd4;
-};
-__device__ __forceinline__ HScale make_hscale(float s_g) {
-  HScale h;
-  h.s_g = s_g;
-  h.rd6 = __frcp_rn(__fmul_rn(6.0f, s_g));
-  h.rd4 = __frcp_rn(__fmul_rn(4.0f, s_g));
-  return h;
-}
-
 // One candidate with a normal scale S: signed codes (element i in bits
 // [4i, 4i+4)) and the squared error.
 __device__ __forceinline__ float nvfp4_candidate_hs(const float* x, float S, uint64_t& codes) {
@@ -250,26 +313,8 @@ __device__ __forceinline__ float nvfp4_candidate_hs(const float* x, float S, uin
   return __fadd_rn(e0, e1);
 }
 
-// One candidate with a zero or tiny scale: the exact path on |x|, with the
-// sign bits of the negative elements added.
-__device__ __forceinline__ float nvfp4_candidate_h_exact(const float* x, float a, float s_g, float c,
-                                                         uint64_t& codes) {
-  float ax[16];
-  uint64_t neg = 0;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    ax[i] = fabsf(x[i]);
-    neg |= static_cast<uint64_t>(x[i] < 0.0f) << (4 * i + 3);
-  }
-  uint64_t mags;
-  uint32_t sf;
-  const float err = nvfp4_candidate(ax, a, s_g, c, mags, sf);
-  codes = mags | neg;
-  return err;
-}
-
 // NVFP4 4-vs-6 quantization of 16 values of h.
-__device__ __forceinline__ Nvfp4Block nvfp4_quantize16_h(const float* x, const HScale& hs) {
+__device__ __forceinline__ Nvfp4Block nvfp4_quantize16_h(const float* x, const Nvfp4Scale& hs) {
   float a = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
@@ -278,17 +323,9 @@ __device__ __forceinline__ Nvfp4Block nvfp4_quantize16_h(const float* x, const H
   const float S6 = __fmul_rn(e4m3_decode(e6), hs.s_g);
   const float S4 = __fmul_rn(e4m3_decode(e4), hs.s_g);
   uint64_t c6, c4;
-  const float err6 = (S6 >= 0x1p-100f) ? nvfp4_candidate_hs(x, S6, c6) : nvfp4_candidate_h_exact(x, a, hs.s_g, 6.0f, c6);
-  const float err4 = (S4 >= 0x1p-100f) ? nvfp4_candidate_hs(x, S4, c4) : nvfp4_candidate_h_exact(x, a, hs.s_g, 4.0f, c4);
-  const bool four = err4 < err6;
-  const uint64_t codes = four ? c4 : c6;
-  // sign bit only where the magnitude code is non-zero (canonical +0)
-  const uint64_t mags = codes & 0x7777777777777777ull;
-  const uint64_t nz = (mags | (mags >> 1) | (mags >> 2)) & 0x1111111111111111ull;
-  Nvfp4Block b;
-  b.codes = mags | (codes & (nz << 3));
-  b.sf = four ? e4 : e6;
-  return b;
+  const float err6 = (S6 >= 0x1p-100f) ? nvfp4_candidate_hs(x, S6, c6) : nvfp4_candidate_tiny(x, a, hs.s_g, 6.0f, c6);
+  const float err4 = (S4 >= 0x1p-100f) ? nvfp4_candidate_hs(x, S4, c4) : nvfp4_candidate_tiny(x, a, hs.s_g, 4.0f, c4);
+  return nvfp4_pick(err6, c6, e6, err4, c4, e4);
 }
 
 // MXFP8 quantization of 32 float32 values: codes (4 bytes per uint32, element
