@@ -9,7 +9,7 @@
 // Large batches: three kernels after two small memsets (token bitmaps to
 // zero, every row of sorted_slots to -1):
 //   1. route_topk_kernel  one warp per token, 8 tokens per CTA: top-k by k
-//      warp-wide arg-max rounds (ties to the lower index), the softmax, and
+//      warp-wide max rounds (ties to the lower index), the softmax, and
 //      bit t of the expert's token bitmap set (atomicOr, order-independent).
 //   2. route_scan_kernel  one CTA per expert: the exclusive prefix of popc
 //      over its bitmap words (its slot count at the end); the last CTA to
@@ -33,49 +33,69 @@ namespace moe {
 
 constexpr int kTopkWarps = 8;  // tokens per CTA of the top-k kernel
 
-// Top-k of one token's logits by k warp-wide arg-max rounds, then the softmax
-// over the selected logits (lane j computes exp of rank j, lane 0 sums in rank
-// order).  Every lane ends with the same sel_i; lane j < k holds w of rank j.
+// A logit as an unsigned key with the same order (-0 taken as +0, so that the
+// two compare equal like the floats do); 0 is below every logit's key and
+// marks an expert that is not there.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  const uint32_t b = __float_as_uint(__fadd_rn(v, 0.0f));
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Top-k of one token's logits by k warp-wide rounds, then the softmax over
+// the selected logits (lane j computes exp of rank j, lane 0 sums in rank
+// order).  Lane l holds the logits of experts l, l + 32, ... and keeps its
+// best one not yet taken; a round takes the warp's largest key and, among
+// the lanes holding it, the lowest expert index, and only the winning lane
+// looks for its next best.  Every lane ends with the same sel_i; lane j < k
+// holds w of rank j.
 template <int NPL>
 __device__ __forceinline__ void topk_token(const float* __restrict__ row, int E, int k, int lane, int* sel_i,
                                            float& w_lane) {
-  float v[NPL];
+  uint32_t key[NPL];
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
     const int e = lane + 32 * i;
-    v[i] = (e < E) ? __ldg(row + e) : -INFINITY;
+    key[i] = (e < E) ? logit_key(__ldg(row + e)) : 0u;
   }
   uint32_t taken = 0u;
-  float my_v = 0.0f;  // lane j keeps the logit of rank j
+  // this lane's best: largest key, the lower expert among equal keys
+  uint32_t head = 0u;
+  int head_i = 0;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    if (key[i] > head) {
+      head = key[i];
+      head_i = i;
+    }
+  }
+  uint32_t my_key = 0u;  // lane j keeps the key of rank j
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     if (j >= k) break;
-    float bv = -INFINITY;
-    int bi = 0x7FFFFFFF;
+    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, head);
+    const uint32_t my_e = static_cast<uint32_t>(lane + 32 * head_i);
+    const uint32_t win = __reduce_min_sync(0xFFFFFFFFu, head == m ? my_e : 0xFFFFFFFFu);
+    if (lane == j) my_key = m;
+    sel_i[j] = static_cast<int>(win);
+    if (my_e == win) {
+      taken |= 1u << head_i;
+      head = 0u;
+      head_i = 0;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
-      // strict '>' keeps the lower index among equal values of this lane
-      if (e < E && !((taken >> i) & 1u) && (v[i] > bv || bi == 0x7FFFFFFF)) {
-        bv = v[i];
-        bi = e;
+      for (int i = 0; i < NPL; ++i) {
+        if (!((taken >> i) & 1u) && key[i] > head) {
+          head = key[i];
+          head_i = i;
+        }
       }
     }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-      const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
-      if (oi != 0x7FFFFFFF && (bi == 0x7FFFFFFF || ov > bv || (ov == bv && oi < bi))) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (lane == j) my_v = bv;
-    sel_i[j] = bi;
   }
-  const float m = __shfl_sync(0xFFFFFFFFu, my_v, 0);
-  const float ex = (lane < k) ? exp_own(__fsub_rn(my_v, m)) : 0.0f;
+  const float my_v = key_logit(my_key);
+  const float mx = __shfl_sync(0xFFFFFFFFu, my_v, 0);
+  const float ex = (lane < k) ? exp_own(__fsub_rn(my_v, mx)) : 0.0f;
   // s = ((e_0 + e_1) + e_2) + ... in rank order, on lane 0
   float s = __shfl_sync(0xFFFFFFFFu, ex, 0);
 #pragma unroll
