@@ -33,24 +33,9 @@ namespace moe {
 
 constexpr int kTopkWarps = 8;  // tokens per CTA of the top-k kernel
 
-// A logit as an unsigned key with the same order (-0 taken as +0, so that the
-// two compare equal like the floats do); 0 is below every logit's key and
-// marks an expert that is not there.
-__device__ __forceinline__ uint32_t logit_key(float v) {
-  const uint32_t b = __float_as_uint(__fadd_rn(v, 0.0f));
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-__device__ __forceinline__ float key_logit(uint32_t key) {
-  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
-}
-
-// Top-k of one token's logits by k warp-wide rounds, then the softmax over
-// the selected logits (lane j computes exp of rank j, lane 0 sums in rank
-// order).  Lane l holds the logits of experts l, l + 32, ... and keeps its
-// best one not yet taken; a round takes the warp's largest key and, among
-// the lanes holding it, the lowest expert index, and only the winning lane
-// looks for its next best.  Every lane ends with the same sel_i; lane j < k
-// holds w of rank j.
+// Top-k of one token's logits (warp_topk_keys), then the softmax over the
+// selected logits.  Every lane ends with the same sel_i; lane j < k holds w
+// of rank j.
 template <int NPL>
 __device__ __forceinline__ void topk_token(const float* __restrict__ row, int E, int k, int lane, int* sel_i,
                                            float& w_lane) {
@@ -60,50 +45,8 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ row, int E,
     const int e = lane + 32 * i;
     key[i] = (e < E) ? logit_key(__ldg(row + e)) : 0u;
   }
-  uint32_t taken = 0u;
-  // this lane's best: largest key, the lower expert among equal keys
-  uint32_t head = 0u;
-  int head_i = 0;
-#pragma unroll
-  for (int i = 0; i < NPL; ++i) {
-    if (key[i] > head) {
-      head = key[i];
-      head_i = i;
-    }
-  }
-  uint32_t my_key = 0u;  // lane j keeps the key of rank j
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (j >= k) break;
-    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, head);
-    const uint32_t my_e = static_cast<uint32_t>(lane + 32 * head_i);
-    const uint32_t win = __reduce_min_sync(0xFFFFFFFFu, head == m ? my_e : 0xFFFFFFFFu);
-    if (lane == j) my_key = m;
-    sel_i[j] = static_cast<int>(win);
-    if (my_e == win) {
-      taken |= 1u << head_i;
-      head = 0u;
-      head_i = 0;
-#pragma unroll
-      for (int i = 0; i < NPL; ++i) {
-        if (!((taken >> i) & 1u) && key[i] > head) {
-          head = key[i];
-          head_i = i;
-        }
-      }
-    }
-  }
-  const float my_v = key_logit(my_key);
-  const float mx = __shfl_sync(0xFFFFFFFFu, my_v, 0);
-  const float ex = (lane < k) ? exp_own(__fsub_rn(my_v, mx)) : 0.0f;
-  // s = ((e_0 + e_1) + e_2) + ... in rank order, on lane 0
-  float s = __shfl_sync(0xFFFFFFFFu, ex, 0);
-#pragma unroll
-  for (int j = 1; j < 8; ++j) {
-    const float ej = __shfl_sync(0xFFFFFFFFu, ex, j);
-    if (j < k) s = __fadd_rn(s, ej);
-  }
-  w_lane = __fdiv_rn(ex, s);
+  const uint32_t my_key = warp_topk_keys<NPL>(key, k, lane, sel_i);
+  w_lane = warp_topk_softmax(key_logit(my_key), k, lane);
 }
 
 // NPL = logits per lane (ceil(E / 32)); W = bitmap words per expert.

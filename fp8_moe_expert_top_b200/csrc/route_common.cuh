@@ -1,5 +1,6 @@
 // Routing pieces shared by the top-k kernel over given logits and the fused
-// router (GEMM + top-k): the softmax's exponential.
+// router (GEMM + top-k): the warp-wide top-k selection and the softmax's
+// exponential.
 #pragma once
 
 #include <cstdint>
@@ -30,6 +31,76 @@ __device__ __forceinline__ float exp_own(float x) {
   p = __fadd_rn(__fmul_rn(p, r), c0);
   const float two_n = __uint_as_float(static_cast<uint32_t>(static_cast<int>(n) + 127) << 23);
   return __fmul_rn(p, two_n);
+}
+
+// A logit as an unsigned key with the same order (-0 taken as +0, so that the
+// two compare equal like the floats do); 0 is below every logit's key and
+// marks an expert that is not there.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  const uint32_t b = __float_as_uint(__fadd_rn(v, 0.0f));
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Top-k (k <= 8) of one token whose logits are spread over a warp: lane l
+// holds the keys of experts l, l + 32, ... (NPL of them).  Each lane keeps
+// its best key not yet taken; a round takes the warp's largest key and, among
+// the lanes holding it, the lowest expert index (two warp reductions), and
+// only the winning lane looks for its next best.  Every lane ends with the
+// same sel_i[0..k); lane j < k returns the key of rank j.
+template <int NPL>
+__device__ __forceinline__ uint32_t warp_topk_keys(const uint32_t* key, int k, int lane, int* sel_i) {
+  uint32_t taken = 0u;
+  // this lane's best: largest key, the lower expert among equal keys
+  uint32_t head = 0u;
+  int head_i = 0;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    if (key[i] > head) {
+      head = key[i];
+      head_i = i;
+    }
+  }
+  uint32_t my_key = 0u;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j >= k) break;
+    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, head);
+    const uint32_t my_e = static_cast<uint32_t>(lane + 32 * head_i);
+    const uint32_t win = __reduce_min_sync(0xFFFFFFFFu, head == m ? my_e : 0xFFFFFFFFu);
+    if (lane == j) my_key = m;
+    sel_i[j] = static_cast<int>(win);
+    if (my_e == win) {
+      taken |= 1u << head_i;
+      head = 0u;
+      head_i = 0;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        if (!((taken >> i) & 1u) && key[i] > head) {
+          head = key[i];
+          head_i = i;
+        }
+      }
+    }
+  }
+  return my_key;
+}
+
+// Softmax over the k selected logits, lane j holding the logit of rank j:
+// e_j = exp(l_j - l_0), s = ((e_0 + e_1) + e_2) + ... in rank order, and lane
+// j < k returns e_j / s.
+__device__ __forceinline__ float warp_topk_softmax(float my_v, int k, int lane) {
+  const float mx = __shfl_sync(0xFFFFFFFFu, my_v, 0);
+  const float ex = (lane < k) ? exp_own(__fsub_rn(my_v, mx)) : 0.0f;
+  float s = __shfl_sync(0xFFFFFFFFu, ex, 0);
+#pragma unroll
+  for (int j = 1; j < 8; ++j) {
+    const float ej = __shfl_sync(0xFFFFFFFFu, ex, j);
+    if (j < k) s = __fadd_rn(s, ej);
+  }
+  return __fdiv_rn(ex, s);
 }
 
 }  // namespace moe

@@ -274,16 +274,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
 // Small batches: the same scores with K split over a cluster of KS CTAs per
 // 128 tokens, so that a decode batch spreads its router weights over KS SMs
 // instead of one.  CTA r of the cluster accumulates k tiles
-// [r KT/KS, (r+1) KT/KS) of all NB expert blocks in TMEM; after every CTA's
-// MMAs are complete (first cluster barrier) each token row's partial scores
-// are pushed (st.shared::cluster) into the ring of the CTA that owns the row
-// (owner r holds rows [r RPO, (r+1) RPO), RPO = 128 / KS), slot r of it;
-// after the second cluster barrier each owner sums the KS partials of its
-// rows in rank order (so the scores do not depend on timing) and a warp per
-// row selects the top-k: each lane keeps a sorted top-8 of the experts
-// e = lane (mod 32), scanned in ascending order, and k rounds of a warp
-// argmax over the lanes' heads (higher score, then lower index) give the
-// ranked selection.  The softmax and the bitmap update are those of
+// [r KT/KS, (r+1) KT/KS) of all NB expert blocks in TMEM.  After every CTA's
+// MMAs are complete (first cluster barrier) each valid token row's partial
+// scores are pushed (st.shared::cluster) into the ring of the CTA that owns
+// the row, slot r of it; the tile's t_tile valid rows are shared out evenly
+// (owner r holds rows [r rpo, (r+1) rpo), rpo = ceil(t_tile / KS) <= 128 /
+// KS).  After the second cluster barrier each owner sums the KS partials of
+// its rows in rank order (so the scores do not depend on timing) and a warp
+// per row selects the top-k with warp_topk_keys (the largest scores, ties to
+// the lower index).  The softmax and the bitmap update are those of
 // route_topk_kernel.  Every thread passes both cluster barriers exactly once,
 // whatever happened before, so a CTA that timed out cannot stall the others.
 template <int NB, int ST, int KS>
@@ -422,12 +421,20 @@ __global__ void __launch_bounds__(kRThreads, 1)
   const bool acc_ok = !*abort_flag;
   cluster_sync();  // every CTA's MMAs are complete: all rings may be written
 
-  if (warp >= 2 && acc_ok) {
+  // The tile's valid rows are shared out evenly: owner r holds rows
+  // [r rpo, (r + 1) rpo) of the t_tile valid ones (rpo <= RPO), so a batch
+  // smaller than 128 tokens spreads its rows, and its top-k work, over all
+  // KS CTAs, and rows past the batch are neither pushed nor reduced.
+  const int t_tile = min(kRM, args.T - m0);
+  const int rpo = (t_tile + KS - 1) / KS;
+  if (warp >= 2 && acc_ok && (warp & 3) * 32 < t_tile) {
     // push this CTA's partial scores of each row into the row's owner
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    const uint32_t owner = static_cast<uint32_t>(row / RPO);
-    const int r_loc = row % RPO;
+    // rows past the batch push nothing; their owner is set to this CTA only
+    // so that the address below is computed for a rank of the cluster
+    const uint32_t owner = row < t_tile ? static_cast<uint32_t>(row / rpo) : rank;
+    const int r_loc = row < t_tile ? row % rpo : 0;
     const uint32_t dst = mapa_shared(smem_u32(recv), owner) +
                          static_cast<uint32_t>(((static_cast<int>(rank) * RPO + r_loc) * EP) * 4);
     const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
@@ -436,10 +443,12 @@ __global__ void __launch_bounds__(kRThreads, 1)
       float v[32];
       tmem_ld32(t_row + 32 * c, v);
       tmem_ld_wait();
+      if (row < t_tile) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t unit = static_cast<uint32_t>(8 * c + u) ^ static_cast<uint32_t>(r_loc & 7);
-        st_cluster_v4(dst + 16u * unit, v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t unit = static_cast<uint32_t>(8 * c + u) ^ static_cast<uint32_t>(r_loc & 7);
+          st_cluster_v4(dst + 16u * unit, v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        }
       }
     }
   }
@@ -450,16 +459,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
   {
     // reduce the owned rows over the KS partials, then top-k (a warp per row,
     // every warp of the CTA)
-    for (int r_loc = warp; r_loc < RPO; r_loc += kRThreads / 32) {
-      const int t = m0 + static_cast<int>(rank) * RPO + r_loc;
-      if (t >= args.T) break;
-      float tv[8];
-      int ti[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        tv[j] = -INFINITY;
-        ti[j] = 0x7FFFFFFF;
-      }
+    const int own0 = static_cast<int>(rank) * rpo;
+    for (int r_loc = warp; r_loc < rpo && own0 + r_loc < t_tile; r_loc += kRThreads / 32) {
+      const int t = m0 + own0 + r_loc;
+      uint32_t key[EP / 32];
 #pragma unroll
       for (int i = 0; i < EP / 32; ++i) {
         const int e = 32 * i + lane;
@@ -467,69 +470,23 @@ __global__ void __launch_bounds__(kRThreads, 1)
         float v = recv[(0 * RPO + r_loc) * EP + off];
 #pragma unroll
         for (int s = 1; s < KS; ++s) v = __fadd_rn(v, recv[(s * RPO + r_loc) * EP + off]);
+        key[i] = 0u;
         if (e < args.E) {
           if (args.logits_out != nullptr) args.logits_out[static_cast<int64_t>(t) * args.E + e] = v;
-          if (v > tv[7] || ti[7] == 0x7FFFFFFF) {
-            tv[7] = v;
-            ti[7] = e;
-#pragma unroll
-            for (int j = 7; j > 0; --j) {
-              if (tv[j] > tv[j - 1] || ti[j - 1] == 0x7FFFFFFF) {
-                const float fv = tv[j];
-                tv[j] = tv[j - 1];
-                tv[j - 1] = fv;
-                const int fi = ti[j];
-                ti[j] = ti[j - 1];
-                ti[j - 1] = fi;
-              }
-            }
-          }
+          key[i] = logit_key(v);
         }
       }
-      // k rounds of a warp argmax over the lanes' heads
+      // top-k and softmax as route_topk_kernel computes them
       const int k = args.k;
-      float sv[8];
       int si[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float bv = tv[0];
-        int bi = ti[0];
-#pragma unroll
-        for (int d = 16; d >= 1; d >>= 1) {
-          const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, d);
-          const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, d);
-          if (oi != 0x7FFFFFFF && (bi == 0x7FFFFFFF || ov > bv || (ov == bv && oi < bi))) {
-            bv = ov;
-            bi = oi;
-          }
-        }
-        sv[j] = bv;
-        si[j] = bi;
-        if (bi != 0x7FFFFFFF && (bi & 31) == lane) {  // the winner's lane drops its head
-#pragma unroll
-          for (int i = 0; i < 7; ++i) {
-            tv[i] = tv[i + 1];
-            ti[i] = ti[i + 1];
-          }
-          tv[7] = -INFINITY;
-          ti[7] = 0x7FFFFFFF;
-        }
-      }
-      // softmax over the k selected scores, as route_topk_kernel computes it
-      float ex[8];
-      float s = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        ex[j] = (j < k) ? exp_own(__fsub_rn(sv[j], sv[0])) : 0.0f;
-        if (j == 0) s = ex[0];
-        else if (j < k) s = __fadd_rn(s, ex[j]);
-      }
+      const uint32_t my_key = warp_topk_keys<EP / 32>(key, k, lane, si);
+      const float w = warp_topk_softmax(key_logit(my_key), k, lane);
       const int64_t o = static_cast<int64_t>(t) * k;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j < k && lane == j) {
           args.topk_ids[o + j] = si[j];
-          args.topk_w[o + j] = __fdiv_rn(ex[j], s);
+          args.topk_w[o + j] = w;
           if (args.bitmap != nullptr)
             atomicOr(&args.bitmap[static_cast<int64_t>(si[j]) * args.W + (t >> 5)], 1u << (t & 31));
         }
