@@ -42,6 +42,10 @@ constexpr int kRM = 128;           // tokens per CTA (TMEM lanes)
 constexpr int kRKElems = 64;       // bf16 of K per stage (128 bytes per row)
 constexpr int kREpiWarps = 4;
 constexpr int kRThreads = 64 + 32 * kREpiWarps;
+// The large-batch kernel's epilogue has two warps per TMEM lane quarter, each
+// selecting over half of a row's scores (one warp per quarter scanning all of
+// them took as long as the MMAs).
+constexpr int kRThreadsTopk = 64 + 32 * 2 * kREpiWarps;
 constexpr int kRTileBytes = kRM * 128;  // one 128-row x 128-byte tile
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* tmap, int c0, int c1, uint64_t* bar) {
@@ -61,9 +65,15 @@ struct RouterArgs {
   int T, E, H, k, W;
 };
 
+// Orders this thread's later generic-proxy accesses to shared memory after
+// earlier async-proxy (bulk copy) writes to the same region.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // NB: 128-expert blocks of W_r (1..4); ST: ring stages.
 template <int NB, int ST>
-__global__ void __launch_bounds__(kRThreads, 1)
+__global__ void __launch_bounds__(kRThreadsTopk, 1)
     router_topk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                        const RouterArgs args) {
   constexpr int kStageBytes = kRTileBytes * (1 + NB);
@@ -139,6 +149,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      const uint64_t adesc0 = make_desc_sw128(smem_u32(smem));
       for (int kt = 0; kt < k_tiles; ++kt) {
         if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
           fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
@@ -146,14 +157,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t st = smem_u32(smem + stage * kStageBytes);
-        const uint64_t adesc = make_desc_sw128(st);
+        // stage descriptors from stage 0's by a constant offset, MMAs unrolled
+        const uint64_t adesc = adesc0 + static_cast<uint64_t>(stage) * (kStageBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < kRKElems / 16; ++kk) {
           const uint32_t acc = (kt | kk) != 0 ? 1u : 0u;
 #pragma unroll
           for (int b = 0; b < NB; b += 2) {
-            const uint64_t bdesc = make_desc_sw128(st + kRTileBytes * (1 + b));
+            const uint64_t bdesc = adesc + (static_cast<uint64_t>(kRTileBytes * (1 + b)) >> 4);
             if (b + 1 < NB)
               tc_mma_bf16(tmem_base + 128 * b, adesc + 2 * kk, bdesc + 2 * kk, idesc_bf16(256), acc);
             else
@@ -170,21 +181,32 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Warps 2..9: quarter q = warp % 4 of the TMEM lanes (rows), half of the
+    // score columns (experts [half E/2, ...)).  Each keeps its row's top 8 of
+    // its half; the second half's lists go through shared memory (the ring
+    // is idle once the accumulator is complete) to the first half's warp,
+    // which merges them, then computes the softmax and writes the row.
     const int q = warp & 3;  // TMEM lane quarter this warp may read
+    const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const int t = m0 + row;
-    if (mbar_wait(acc_bar, 0, abort_flag)) {
-      tc_fence_after();
-      float tv[8];
-      int ti[8];
+    const bool acc_ok = mbar_wait(acc_bar, 0, abort_flag);
+    if (!acc_ok) fail_bits |= MOE_DEVICE_TIMEOUT_EPILOGUE;
+    // this row's top 8 so far as order-preserving keys, largest first; an
+    // empty slot holds key 0, below every score
+    uint32_t tk[8];
+    int ti[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        tv[j] = -INFINITY;
-        ti[j] = 0x7FFFFFFF;
-      }
+    for (int j = 0; j < 8; ++j) {
+      tk[j] = 0u;
+      ti[j] = 0;
+    }
+    if (acc_ok) {
+      tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      const int c0 = half * (NB * 2);
 #pragma unroll 1
-      for (int c = 0; c < NB * 4; ++c) {
+      for (int c = c0; c < c0 + NB * 2; ++c) {
         float v[32];
         tmem_ld32(t_row + 32 * c, v);
         tmem_ld_wait();
@@ -198,25 +220,57 @@ __global__ void __launch_bounds__(kRThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int e = 32 * c + i;
-            // strictly better than the current 8th (an empty slot loses to
-            // anything); experts arrive in ascending order, so an equal score
-            // already held keeps its lower index ahead
-            if (e < args.E && (v[i] > tv[7] || ti[7] == 0x7FFFFFFF)) {
-              tv[7] = v[i];
-              ti[7] = e;
+            const uint32_t key = e < args.E ? logit_key(v[i]) : 0u;
+            // strictly above the current 8th; experts arrive in ascending
+            // order, so an equal score already held keeps its lower index
+            // ahead.  All eight slots are updated at once from the old list
+            // (the comparisons are independent), not by a chain of swaps.
+            if (key > tk[7]) {
+              bool above[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) above[j] = key > tk[j];
 #pragma unroll
               for (int j = 7; j > 0; --j) {
-                if (tv[j] > tv[j - 1] || ti[j - 1] == 0x7FFFFFFF) {
-                  const float fv = tv[j];
-                  tv[j] = tv[j - 1];
-                  tv[j - 1] = fv;
-                  const int fi = ti[j];
-                  ti[j] = ti[j - 1];
-                  ti[j - 1] = fi;
-                }
+                tk[j] = above[j - 1] ? tk[j - 1] : (above[j] ? key : tk[j]);
+                ti[j] = above[j - 1] ? ti[j - 1] : (above[j] ? e : ti[j]);
               }
+              tk[0] = above[0] ? key : tk[0];
+              ti[0] = above[0] ? e : ti[0];
             }
           }
+        }
+      }
+    }
+    uint32_t* xk = reinterpret_cast<uint32_t*>(smem);  // [128 rows][8] keys of the second half
+    int* xi = reinterpret_cast<int*>(smem + kRM * 8 * 4);
+    if (half == 1) {
+      fence_proxy_async_shared();  // the ring last held bulk-copied operands
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        xk[row * 8 + j] = tk[j];
+        xi[row * 8 + j] = ti[j];
+      }
+    }
+    // both warps of the quarter arrive here exactly once, whatever happened
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(64) : "memory");
+    if (half == 0 && acc_ok) {
+      // merge: the second half's experts all have higher indices, so an
+      // equal score goes after the first half's (strictly-above insertion)
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const uint32_t key = xk[row * 8 + jj];
+        const int e = xi[row * 8 + jj];
+        if (key > tk[7]) {
+          bool above[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) above[j] = key > tk[j];
+#pragma unroll
+          for (int j = 7; j > 0; --j) {
+            tk[j] = above[j - 1] ? tk[j - 1] : (above[j] ? key : tk[j]);
+            ti[j] = above[j - 1] ? ti[j - 1] : (above[j] ? e : ti[j]);
+          }
+          tk[0] = above[0] ? key : tk[0];
+          ti[0] = above[0] ? e : ti[0];
         }
       }
       if (t < args.T) {
@@ -224,9 +278,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
         const int k = args.k;
         float ex[8];
         float s = 0.0f;
+        const float top = key_logit(tk[0]);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          ex[j] = (j < k) ? exp_own(__fsub_rn(tv[j], tv[0])) : 0.0f;
+          ex[j] = (j < k) ? exp_own(__fsub_rn(key_logit(tk[j]), top)) : 0.0f;
           if (j == 0) s = ex[0];
           else if (j < k) s = __fadd_rn(s, ex[j]);
         }
@@ -241,8 +296,6 @@ __global__ void __launch_bounds__(kRThreads, 1)
           }
         }
       }
-    } else {
-      fail_bits |= MOE_DEVICE_TIMEOUT_EPILOGUE;
     }
   }
 
@@ -556,7 +609,7 @@ cudaError_t launch_nb(const CUtensorMap& mx, const CUtensorMap& mw, const Router
   });
   if (attr_err != cudaSuccess) return attr_err;
   const dim3 grid(static_cast<unsigned>((a.T + kRM - 1) / kRM));
-  return launch_pdl(router_topk_kernel<NB, ST>, grid, dim3(kRThreads), smem, stream, mx, mw, a);
+  return launch_pdl(router_topk_kernel<NB, ST>, grid, dim3(kRThreadsTopk), smem, stream, mx, mw, a);
 }
 
 template <int NB, int KS>
