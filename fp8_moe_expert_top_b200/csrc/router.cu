@@ -71,6 +71,22 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Insert (key, e) into a row's top 8 (keys largest first), key strictly above
+// tk[7]: all eight slots are updated at once from the old list (independent
+// comparisons, not a chain of swaps); an equal key already held stays ahead.
+__device__ __forceinline__ void topk_insert(uint32_t* tk, int* ti, uint32_t key, int e) {
+  bool above[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) above[j] = key > tk[j];
+#pragma unroll
+  for (int j = 7; j > 0; --j) {
+    tk[j] = above[j - 1] ? tk[j - 1] : (above[j] ? key : tk[j]);
+    ti[j] = above[j - 1] ? ti[j - 1] : (above[j] ? e : ti[j]);
+  }
+  tk[0] = above[0] ? key : tk[0];
+  ti[0] = above[0] ? e : ti[0];
+}
+
 // NB: 128-expert blocks of W_r (1..4); ST: ring stages.
 template <int NB, int ST>
 __global__ void __launch_bounds__(kRThreadsTopk, 1)
@@ -221,22 +237,9 @@ __global__ void __launch_bounds__(kRThreadsTopk, 1)
           for (int i = 0; i < 32; ++i) {
             const int e = 32 * c + i;
             const uint32_t key = e < args.E ? logit_key(v[i]) : 0u;
-            // strictly above the current 8th; experts arrive in ascending
-            // order, so an equal score already held keeps its lower index
-            // ahead.  All eight slots are updated at once from the old list
-            // (the comparisons are independent), not by a chain of swaps.
-            if (key > tk[7]) {
-              bool above[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) above[j] = key > tk[j];
-#pragma unroll
-              for (int j = 7; j > 0; --j) {
-                tk[j] = above[j - 1] ? tk[j - 1] : (above[j] ? key : tk[j]);
-                ti[j] = above[j - 1] ? ti[j - 1] : (above[j] ? e : ti[j]);
-              }
-              tk[0] = above[0] ? key : tk[0];
-              ti[0] = above[0] ? e : ti[0];
-            }
+            // experts arrive in ascending order, so an equal score already
+            // held keeps its lower index ahead
+            if (key > tk[7]) topk_insert(tk, ti, key, e);
           }
         }
       }
@@ -259,19 +262,7 @@ __global__ void __launch_bounds__(kRThreadsTopk, 1)
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
         const uint32_t key = xk[row * 8 + jj];
-        const int e = xi[row * 8 + jj];
-        if (key > tk[7]) {
-          bool above[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) above[j] = key > tk[j];
-#pragma unroll
-          for (int j = 7; j > 0; --j) {
-            tk[j] = above[j - 1] ? tk[j - 1] : (above[j] ? key : tk[j]);
-            ti[j] = above[j - 1] ? ti[j - 1] : (above[j] ? e : ti[j]);
-          }
-          tk[0] = above[0] ? key : tk[0];
-          ti[0] = above[0] ? e : ti[0];
-        }
+        if (key > tk[7]) topk_insert(tk, ti, key, xi[row * 8 + jj]);
       }
       if (t < args.T) {
         // softmax over the k selected scores, as route_topk_kernel computes it
@@ -554,6 +545,253 @@ __global__ void __launch_bounds__(kRThreads, 1)
   }
 }
 
+// Mid-size batches (too many row tiles for the K split, fewer than one per
+// pair of SMs): the experts split over a cluster of two CTAs per 128 tokens.
+// CTA r computes the scores of experts [r NH, (r+1) NH) over all of K (N = NH
+// per MMA, NH = E/2), so each CTA streams half of W_r and no partial scores
+// move.  Its epilogue (two warps per TMEM lane quarter, half of its columns
+// each) keeps each row's top 8 as keys and merges the two halves through its
+// idle ring; after a first cluster barrier CTA 1 sends its lists
+// (st.shared::cluster, 64 bytes per row) into CTA 0's ring, and after a
+// second one CTA 0 merges them (its experts come first, so an equal score
+// keeps the lower index), computes the softmax and writes the row.  Every
+// thread passes both cluster barriers exactly once, whatever happened before.
+template <int NC, int ST>
+__global__ void __launch_bounds__(kRThreadsTopk, 1)
+    router_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                       const RouterArgs args) {
+  constexpr int NH = 32 * NC;                  // experts (MMA N) per CTA
+  constexpr int kWBytes = NH * 128;            // one stage of this CTA's W_r rows
+  constexpr int kStageBytes = kRTileBytes + kWBytes;
+  constexpr uint32_t kTmemCols = NH <= 32 ? 32u : (NH <= 64 ? 64u : (NH <= 128 ? 128u : 256u));
+  static_assert(NC % 2 == 0 && NH <= 256, "two selecting warps per quarter, N <= 256");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + ST * kStageBytes);
+  uint64_t* empty_bar = full_bar + ST;
+  uint64_t* acc_bar = empty_bar + ST;
+  uint64_t* drain_bar = acc_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* drain_failed = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  // exchange areas in the ring, used once every MMA of both CTAs is complete
+  uint32_t* xk = reinterpret_cast<uint32_t*>(smem);             // [128][8] keys, second half of this CTA
+  int* xi = reinterpret_cast<int*>(smem + kRM * 8 * 4);         // [128][8] experts
+  uint32_t* rk = reinterpret_cast<uint32_t*>(smem + kRM * 64);  // [128][8] keys from CTA 1 (CTA 0 only)
+  int* ri = reinterpret_cast<int*>(smem + kRM * 96);            // [128][8] experts from CTA 1
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int m0 = static_cast<int>(blockIdx.x >> 1) * kRM;
+  const int e0 = static_cast<int>(rank) * NH;  // this CTA's first expert
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(acc_bar, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *drain_failed = 0;
+    fence_mbar_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  pdl_wait();
+  pdl_trigger();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int k_tiles = args.H / kRKElems;
+  uint32_t fail_bits = 0;
+  uint32_t armed = 0u, armed_par = 0u;
+  uint32_t tk[8];
+  int ti[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    tk[j] = 0u;
+    ti[j] = 0;
+  }
+  bool acc_ok = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+          fail_bits |= MOE_DEVICE_TIMEOUT_PRODUCER;
+          break;
+        }
+        uint8_t* st = smem + stage * kStageBytes;
+        mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
+        tma_load_2d(st, &tmap_x, kt * kRKElems, m0, &full_bar[stage]);
+        tma_load_2d(st + kRTileBytes, &tmap_w, kt * kRKElems, e0, &full_bar[stage]);
+        armed |= 1u << stage;
+        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == ST) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      const uint64_t adesc0 = make_desc_sw128(smem_u32(smem));
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+          fail_bits |= MOE_DEVICE_TIMEOUT_MMA;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t adesc = adesc0 + static_cast<uint64_t>(stage) * (kStageBytes >> 4);
+        const uint64_t bdesc = adesc + (kRTileBytes >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kRKElems / 16; ++kk)
+          tc_mma_bf16(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, idesc_bf16(NH), (kt | kk) != 0 ? 1u : 0u);
+        tc_commit(&empty_bar[stage]);
+        if (++stage == ST) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) tc_commit(acc_bar);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue: this CTA's top 8 per row
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    const int t = m0 + row;
+    acc_ok = mbar_wait(acc_bar, 0, abort_flag);
+    if (!acc_ok) fail_bits |= MOE_DEVICE_TIMEOUT_EPILOGUE;
+    if (acc_ok) {
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int c = half * (NC / 2); c < (half + 1) * (NC / 2); ++c) {
+        float v[32];
+        tmem_ld32(t_row + 32 * c, v);
+        tmem_ld_wait();
+        if (t < args.T) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int e = e0 + 32 * c + i;
+            if (args.logits_out != nullptr && e < args.E) args.logits_out[static_cast<int64_t>(t) * args.E + e] = v[i];
+            const uint32_t key = e < args.E ? logit_key(v[i]) : 0u;
+            if (key > tk[7]) topk_insert(tk, ti, key, e);
+          }
+        }
+      }
+    }
+    if (half == 1) {
+      fence_proxy_async_shared();  // the ring last held bulk-copied operands
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        xk[row * 8 + j] = tk[j];
+        xi[row * 8 + j] = ti[j];
+      }
+    }
+    // both warps of the quarter arrive here exactly once, whatever happened
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(64) : "memory");
+    if (half == 0 && acc_ok) {
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const uint32_t key = xk[row * 8 + jj];
+        const int e = xi[row * 8 + jj];
+        if (key > tk[7] && e >= 0 && e < args.E) topk_insert(tk, ti, key, e);
+      }
+    }
+  }
+
+  if (fail_bits != 0u && args.status != nullptr) atomicOr(args.status, fail_bits);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (*abort_flag) {
+    // drain what is in flight before the ring is reused and TMEM freed
+    bool drained = true;
+    if (warp == 0 && lane == 0) {
+      for (int st = 0; st < ST; ++st)
+        if ((armed >> st) & 1u) drained = mbar_wait_drain(&full_bar[st], (armed_par >> st) & 1u) && drained;
+    } else if (warp == 1 && lane == 0) {
+      tc_commit(drain_bar);
+      drained = mbar_wait_drain(drain_bar, 0);
+    }
+    if (!drained) *drain_failed = 1;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  const bool ok_cta = !*abort_flag;
+  cluster_sync();  // both CTAs' MMAs are complete: CTA 0's ring may be written
+
+  const bool lister = warp >= 2 && ((warp - 2) >> 2) == 0;  // the half-0 warps hold the lists
+  const int row = (warp & 3) * 32 + lane;
+  if (rank == 1 && lister) {  // also after an abort: empty lists (key 0) merge nothing
+    const uint32_t dk = mapa_shared(smem_u32(rk), 0) + static_cast<uint32_t>(row * 32);
+    const uint32_t di = mapa_shared(smem_u32(ri), 0) + static_cast<uint32_t>(row * 32);
+    st_cluster_v4(dk, __uint_as_float(tk[0]), __uint_as_float(tk[1]), __uint_as_float(tk[2]), __uint_as_float(tk[3]));
+    st_cluster_v4(dk + 16, __uint_as_float(tk[4]), __uint_as_float(tk[5]), __uint_as_float(tk[6]),
+                  __uint_as_float(tk[7]));
+    st_cluster_v4(di, __int_as_float(ti[0]), __int_as_float(ti[1]), __int_as_float(ti[2]), __int_as_float(ti[3]));
+    st_cluster_v4(di + 16, __int_as_float(ti[4]), __int_as_float(ti[5]), __int_as_float(ti[6]), __int_as_float(ti[7]));
+  }
+  cluster_sync();  // CTA 1's lists have arrived
+
+  if (rank == 0 && lister) {
+    // (after an abort in CTA 1 the rows keep CTA 0's experts only; CTA 1's
+    // status bit reports it)
+    const int t = m0 + row;
+    if (ok_cta && t < args.T) {
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        // an expert index outside [0, E) can only come from an aborted
+        // partner's stale ring bytes; it is never taken
+        const uint32_t key = rk[row * 8 + jj];
+        const int e = ri[row * 8 + jj];
+        if (key > tk[7] && e >= 0 && e < args.E) topk_insert(tk, ti, key, e);
+      }
+      // softmax over the k selected scores, as route_topk_kernel computes it
+      const int k = args.k;
+      float ex[8];
+      float s = 0.0f;
+      const float top = key_logit(tk[0]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        ex[j] = (j < k) ? exp_own(__fsub_rn(key_logit(tk[j]), top)) : 0.0f;
+        if (j == 0) s = ex[0];
+        else if (j < k) s = __fadd_rn(s, ex[j]);
+      }
+      const int64_t o = static_cast<int64_t>(t) * k;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < k) {
+          args.topk_ids[o + j] = ti[j];
+          args.topk_w[o + j] = __fdiv_rn(ex[j], s);
+          if (args.bitmap != nullptr)
+            atomicOr(&args.bitmap[static_cast<int64_t>(ti[j]) * args.W + (t >> 5)], 1u << (t & 31));
+        }
+      }
+    }
+  }
+  if (warp == 1 && !*drain_failed) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
 template <int NB>
 constexpr int router_stages() {
   return (kRTileBytes * (1 + NB) * 4 <= 200 * 1024) ? 4 : ((kRTileBytes * (1 + NB) * 3 <= 200 * 1024) ? 3 : 2);
@@ -583,14 +821,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// A [rows][H] bf16 row-major matrix, loaded in boxes of 64 elements x 128
-// rows with the 128-byte swizzle; rows past the end read as zeros.
-bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t H) {
+// A [rows][H] bf16 row-major matrix, loaded in boxes of 64 elements x
+// box_rows rows with the 128-byte swizzle; rows past the end read as zeros.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t H, int box_rows = kRM) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kRKElems), static_cast<cuuint32_t>(kRM)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kRKElems), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t elem[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -610,6 +848,38 @@ cudaError_t launch_nb(const CUtensorMap& mx, const CUtensorMap& mw, const Router
   if (attr_err != cudaSuccess) return attr_err;
   const dim3 grid(static_cast<unsigned>((a.T + kRM - 1) / kRM));
   return launch_pdl(router_topk_kernel<NB, ST>, grid, dim3(kRThreadsTopk), smem, stream, mx, mw, a);
+}
+
+template <int NC>
+constexpr int pair_stages() {
+  return (200 * 1024) / (kRTileBytes + 32 * NC * 128) > 6 ? 6 : (200 * 1024) / (kRTileBytes + 32 * NC * 128);
+}
+template <int NC>
+cudaError_t launch_pair(const CUtensorMap& mx, const CUtensorMap& mw, const RouterArgs& a, cudaStream_t stream) {
+  constexpr int ST = pair_stages<NC>();
+  constexpr size_t smem = 1024 + static_cast<size_t>(ST) * (kRTileBytes + 32 * NC * 128) + (2 * ST + 2) * 8 + 16;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(router_pair_kernel<NC, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem));
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((a.T + kRM - 1) / kRM * 2));
+  cfg.blockDim = dim3(kRThreadsTopk);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, router_pair_kernel<NC, ST>, mx, mw, a);
 }
 
 template <int NB, int KS>
@@ -685,6 +955,21 @@ cudaError_t launch_router_topk(const void* x, const void* w_router, float* logit
   a.W = (T + 31) / 32;
   const int nb = (E + 127) / 128;
   const int ks = router_split(T, H, nb);
+  // Mid-size batches (row tiles too many for the K split but fewer than one
+  // per pair of SMs): the experts split over a two-CTA cluster, each CTA
+  // streaming half of W_r.
+  const int m_tiles = (T + kRM - 1) / kRM;
+  if (ks == 1 && E % 128 == 0 && 2 * m_tiles <= 148) {
+    CUtensorMap mwh;
+    if (!make_map(&mwh, w_router, E, H, E / 2)) return cudaErrorInvalidValue;
+    switch (E / 64) {
+      case 2: return launch_pair<2>(mx, mwh, a, stream);
+      case 4: return launch_pair<4>(mx, mwh, a, stream);
+      case 6: return launch_pair<6>(mx, mwh, a, stream);
+      case 8: return launch_pair<8>(mx, mwh, a, stream);
+      default: break;
+    }
+  }
   switch (nb) {
     case 1: return launch_any<1>(mx, mw, a, ks, stream);
     case 2: return launch_any<2>(mx, mw, a, ks, stream);
