@@ -9,18 +9,25 @@
 // memory (unless the caller asks for a debug copy): the accumulator in TMEM
 // is reduced to the k selected experts by the epilogue.
 //
-// One CTA per 128 tokens:
+// Large batches (router_topk_kernel), one CTA per 128 tokens:
 //   warp 0      producer: TMA tile loads (cp.async.bulk.tensor, 128-byte
 //               swizzle, no multicast) of 64 bf16 of K for the 128 token rows
 //               of x and for all expert rows of W_r, into a ring of stages
 //   warp 1      MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
 //               M = 128, N = 256 and/or 128 per 128-expert block, the
 //               accumulator of all (up to 512) experts in TMEM
-//   warps 2-5   epilogue: one token row per thread: tcgen05.ld 32 scores at
-//               a time, a sorted top-8 kept in registers (strict '>' while
-//               scanning experts in ascending order, so equal scores keep the
-//               lower index), then the same softmax and bitmap update as
-//               route_topk_kernel (bit-identical weights for equal scores).
+//   warps 2-9   epilogue: two warps per TMEM lane quarter, one token row per
+//               thread, half of its scores each: tcgen05.ld 32 scores at a
+//               time, the top 8 kept in registers as order-preserving keys
+//               (strictly-above insertion while scanning experts in
+//               ascending order, so equal scores keep the lower index); the
+//               halves merged through shared memory; then the same softmax
+//               and bitmap update as route_topk_kernel (bit-identical
+//               weights for equal scores).
+// Mid-size batches (router_pair_kernel): the same with the experts split
+// over a cluster of two CTAs per 128 tokens, the two top-8 lists merged
+// through distributed shared memory.  Small batches (router_split_kernel):
+// K split over a cluster of 4 or 8 CTAs per 128 tokens.
 // Every wait is bounded; a wait that runs out raises the CTA's abort flag,
 // the roles stop, work in flight is drained and a status bit is set.
 #include <cstdint>
