@@ -255,7 +255,9 @@ MOE_API moe_status moe_route_topk(const moe_config* cfg, int64_t T, const float*
  * from the exactly rounded sum in its last bits; results do not depend on
  * thread timing.  Batches of up to 37 tiles of 128 tokens (with at most 384
  * experts) split d_model over a cluster of 4 or 8 CTAs per tile and add the
- * partial sums, on chip, in cluster-rank order. */
+ * partial sums, on chip, in cluster-rank order.  Batches of up to 74 tiles
+ * whose num_experts is a multiple of 128 split the experts over a cluster of
+ * two CTAs per tile (each score is still one CTA's full sum). */
 MOE_API moe_status moe_router_topk(const moe_config* cfg, int64_t T, const void* x_bf16, const void* w_router_bf16,
                                    float* logits_out, int32_t* topk_ids, float* topk_w, int32_t* expert_counts,
                                    int32_t* expert_offsets, int32_t* sorted_slots, int32_t* slot_to_row,
