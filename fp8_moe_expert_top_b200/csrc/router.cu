@@ -47,12 +47,11 @@ namespace {
 
 constexpr int kRM = 128;           // tokens per CTA (TMEM lanes)
 constexpr int kRKElems = 64;       // bf16 of K per stage (128 bytes per row)
-constexpr int kREpiWarps = 4;
+// Epilogue warps: two per TMEM lane quarter, each taking half of a row's
+// score columns (one warp per quarter scanning all of them took as long as
+// the MMAs at prefill, and pushed the partial scores half as fast at decode).
+constexpr int kREpiWarps = 8;
 constexpr int kRThreads = 64 + 32 * kREpiWarps;
-// The large-batch kernel's epilogue has two warps per TMEM lane quarter, each
-// selecting over half of a row's scores (one warp per quarter scanning all of
-// them took as long as the MMAs).
-constexpr int kRThreadsTopk = 64 + 32 * 2 * kREpiWarps;
 constexpr int kRTileBytes = kRM * 128;  // one 128-row x 128-byte tile
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* tmap, int c0, int c1, uint64_t* bar) {
@@ -96,7 +95,7 @@ __device__ __forceinline__ void topk_insert(uint32_t* tk, int* ti, uint32_t key,
 
 // NB: 128-expert blocks of W_r (1..4); ST: ring stages.
 template <int NB, int ST>
-__global__ void __launch_bounds__(kRThreadsTopk, 1)
+__global__ void __launch_bounds__(kRThreads, 1)
     router_topk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                        const RouterArgs args) {
   constexpr int kStageBytes = kRTileBytes * (1 + NB);
@@ -479,8 +478,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
   const int t_tile = min(kRM, args.T - m0);
   const int rpo = (t_tile + KS - 1) / KS;
   if (warp >= 2 && acc_ok && (warp & 3) * 32 < t_tile) {
-    // push this CTA's partial scores of each row into the row's owner
+    // push this CTA's partial scores of each row into the row's owner; two
+    // warps per TMEM lane quarter, half of the score columns each
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     // rows past the batch push nothing; their owner is set to this CTA only
     // so that the address below is computed for a rank of the cluster
@@ -490,7 +491,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                          static_cast<uint32_t>(((static_cast<int>(rank) * RPO + r_loc) * EP) * 4);
     const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-    for (int c = 0; c < NB * 4; ++c) {
+    for (int c = half * (NB * 2); c < (half + 1) * (NB * 2); ++c) {
       float v[32];
       tmem_ld32(t_row + 32 * c, v);
       tmem_ld_wait();
@@ -564,7 +565,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
 // keeps the lower index), computes the softmax and writes the row.  Every
 // thread passes both cluster barriers exactly once, whatever happened before.
 template <int NC, int ST>
-__global__ void __launch_bounds__(kRThreadsTopk, 1)
+__global__ void __launch_bounds__(kRThreads, 1)
     router_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                        const RouterArgs args) {
   constexpr int NH = 32 * NC;                  // experts (MMA N) per CTA
@@ -854,7 +855,7 @@ cudaError_t launch_nb(const CUtensorMap& mx, const CUtensorMap& mw, const Router
   });
   if (attr_err != cudaSuccess) return attr_err;
   const dim3 grid(static_cast<unsigned>((a.T + kRM - 1) / kRM));
-  return launch_pdl(router_topk_kernel<NB, ST>, grid, dim3(kRThreadsTopk), smem, stream, mx, mw, a);
+  return launch_pdl(router_topk_kernel<NB, ST>, grid, dim3(kRThreads), smem, stream, mx, mw, a);
 }
 
 template <int NC>
@@ -874,7 +875,7 @@ cudaError_t launch_pair(const CUtensorMap& mx, const CUtensorMap& mw, const Rout
   if (attr_err != cudaSuccess) return attr_err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((a.T + kRM - 1) / kRM * 2));
-  cfg.blockDim = dim3(kRThreadsTopk);
+  cfg.blockDim = dim3(kRThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
