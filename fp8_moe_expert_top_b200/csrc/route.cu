@@ -74,31 +74,6 @@ __global__ void __launch_bounds__(kTopkWarps * 32) route_topk_kernel(const float
   }
 }
 
-// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024).
-__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_sums, int32_t* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int32_t incl = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-    if (lane >= off) incl += o;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int32_t ws = (lane < static_cast<int>(blockDim.x >> 5)) ? warp_sums[lane] : 0;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int32_t o = __shfl_up_sync(0xFFFFFFFFu, ws, off);
-      if (lane >= off) ws += o;
-    }
-    warp_sums[lane] = ws;
-  }
-  __syncthreads();
-  *total = warp_sums[(blockDim.x >> 5) - 1];
-  return incl - v + (warp > 0 ? warp_sums[warp - 1] : 0);
-}
-
 constexpr int kScanThreads = 256;
 constexpr int kScanWordsPerThread = 4;
 
@@ -181,6 +156,7 @@ __global__ void route_scatter_kernel(int T, int E, int k, int W, const int32_t* 
   if (s >= static_cast<int64_t>(T) * k) return;
   const int t = static_cast<int>(s / k);
   const int e = topk_ids[s];
+  if (e < 0 || e >= E) return;  // only after a fused router gave up on a timeout (status word set)
   const int64_t wi = static_cast<int64_t>(e) * W + (t >> 5);
   const int rank = prefix[wi] + __popc(bitmap[wi] & ((1u << (t & 31)) - 1u));
   const int32_t row = expert_offsets[e] + rank;
@@ -203,45 +179,10 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(int T, int E
                                                                     int32_t* __restrict__ slot_to_row) {
   extern __shared__ uint32_t sm_small[];
   __shared__ int32_t warp_sums[32];
-  const int W = (T + 31) >> 5;
-  uint32_t* bm = sm_small;                                    // [E][W] token bitmaps
-  int32_t* pf = reinterpret_cast<int32_t*>(sm_small + E * W);  // [E][W] prefix counts
-  int32_t* off = pf + E * W;                                  // [E] padded offsets
-  const int tid = threadIdx.x;
   pdl_wait();
   pdl_trigger();
-  for (int i = tid; i < E * W; i += blockDim.x) bm[i] = 0u;
-  __syncthreads();
-  const int S = T * k;
-  for (int s = tid; s < S; s += blockDim.x) {
-    const int t = s / k;
-    atomicOr(&bm[topk_ids[s] * W + (t >> 5)], 1u << (t & 31));
-  }
-  __syncthreads();
-  int32_t cnt = 0;
-  if (tid < E) {
-    for (int w = 0; w < W; ++w) {
-      pf[tid * W + w] = cnt;
-      cnt += __popc(bm[tid * W + w]);
-    }
-    expert_counts[tid] = cnt;
-  }
-  int32_t total = 0;
-  const int32_t run = block_exclusive_scan(tid < E ? (cnt + 127) / 128 * 128 : 0, warp_sums, &total);
-  if (tid < E) {
-    expert_offsets[tid] = run;
-    off[tid] = run;
-  }
-  if (tid == 0) expert_offsets[E] = total;
-  for (int64_t r = tid; r < R_max; r += blockDim.x) sorted_slots[r] = -1;
-  __syncthreads();  // the padding marks land before the scatter overwrites the used rows
-  for (int s = tid; s < S; s += blockDim.x) {
-    const int t = s / k, e = topk_ids[s];
-    const int i = e * W + (t >> 5);
-    const int32_t row = off[e] + pf[i] + __popc(bm[i] & ((1u << (t & 31)) - 1u));
-    sorted_slots[row] = s;
-    slot_to_row[s] = row;
-  }
+  small_route_block(T, E, k, R_max, topk_ids, expert_counts, expert_offsets, sorted_slots, slot_to_row, sm_small,
+                    warp_sums);
 }
 
 bool route_small(int T, int E) {

@@ -103,4 +103,92 @@ __device__ __forceinline__ float warp_topk_softmax(float my_v, int k, int lane) 
   return __fdiv_rn(ex, s);
 }
 
+// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024).
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_sums, int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t ws = (lane < static_cast<int>(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xFFFFFFFFu, ws, off);
+      if (lane >= off) ws += o;
+    }
+    warp_sums[lane] = ws;
+  }
+  __syncthreads();
+  *total = warp_sums[(blockDim.x >> 5) - 1];
+  return incl - v + (warp > 0 ? warp_sums[warp - 1] : 0);
+}
+
+// The counting sort of a small batch by one CTA (blockDim.x <= 1024), from
+// topk_ids [T][k]: every expert's token bitmap (E * ceil(T/32) words) and its
+// prefix counts in shared memory (smem: 2 E ceil(T/32) + E words), the slot
+// counts, the 128-padded offsets (exclusive scan in expert order), -1 in
+// every row of sorted_slots, then the scatter: row = offset[e] + (tokens
+// before t that chose e).  An expert index outside [0, E) (possible only if
+// the kernel that wrote topk_ids gave up on a timeout) is skipped, so no
+// access leaves the arrays.
+__device__ __forceinline__ void small_route_block(int T, int E, int k, int64_t R_max,
+                                                  const int32_t* __restrict__ topk_ids,
+                                                  int32_t* __restrict__ expert_counts,
+                                                  int32_t* __restrict__ expert_offsets,
+                                                  int32_t* __restrict__ sorted_slots,
+                                                  int32_t* __restrict__ slot_to_row, uint32_t* smem,
+                                                  int32_t* warp_sums) {
+  const int W = (T + 31) >> 5;
+  uint32_t* bm = smem;                                    // [E][W] token bitmaps
+  int32_t* pf = reinterpret_cast<int32_t*>(smem + E * W);  // [E][W] prefix counts
+  int32_t* off = pf + E * W;                              // [E] padded offsets
+  const int tid = threadIdx.x, nt = blockDim.x;
+  for (int i = tid; i < E * W; i += nt) bm[i] = 0u;
+  __syncthreads();
+  const int S = T * k;
+  for (int s = tid; s < S; s += nt) {
+    const int t = s / k, e = topk_ids[s];
+    if (e >= 0 && e < E) atomicOr(&bm[e * W + (t >> 5)], 1u << (t & 31));
+  }
+  __syncthreads();
+  // experts [tid * per, (tid + 1) * per) per thread, so that the scan runs
+  // in expert order
+  const int per = (E + nt - 1) / nt;
+  const int e_lo = min(E, tid * per), e_hi = min(E, e_lo + per);
+  int32_t mine = 0;
+  for (int e = e_lo; e < e_hi; ++e) {
+    int32_t cnt = 0;
+    for (int w = 0; w < W; ++w) {
+      pf[e * W + w] = cnt;
+      cnt += __popc(bm[e * W + w]);
+    }
+    expert_counts[e] = cnt;
+    mine += (cnt + 127) / 128 * 128;
+  }
+  int32_t total = 0;
+  int32_t run = block_exclusive_scan(mine, warp_sums, &total);
+  for (int e = e_lo; e < e_hi; ++e) {
+    expert_offsets[e] = run;
+    off[e] = run;
+    const int32_t cnt = pf[e * W + W - 1] + __popc(bm[e * W + W - 1]);
+    run += (cnt + 127) / 128 * 128;
+  }
+  if (tid == 0) expert_offsets[E] = total;
+  for (int64_t r = tid; r < R_max; r += nt) sorted_slots[r] = -1;
+  __syncthreads();  // the padding marks land before the scatter overwrites the used rows
+  for (int s = tid; s < S; s += nt) {
+    const int t = s / k, e = topk_ids[s];
+    if (e < 0 || e >= E) continue;
+    const int i = e * W + (t >> 5);
+    const int32_t row = off[e] + pf[i] + __popc(bm[i] & ((1u << (t & 31)) - 1u));
+    sorted_slots[row] = s;
+    slot_to_row[s] = row;
+  }
+}
+
 }  // namespace moe
