@@ -38,12 +38,12 @@ from oracle import route as ort
 # Batches of up to 37 row tiles split K over clusters of 4 or 8 CTAs (the
 # first four cases and 777 tokens: 8; 64 and 129 tokens at d_model 256: 4).
 # Up to 74 row tiles with E a multiple of 128 split the experts over a
-# two-CTA cluster: the 512-expert case (2 tiles), 5000 tokens (40 tiles, 384
-# and 256 experts) and 4900 tokens at 512 experts.  9600 tokens (75 tiles)
+# two-CTA cluster: the 512-expert case (2 tiles), 5000 tokens (40 tiles, 384,
+# 256 and 128 experts) and 4900 tokens at 512 experts.  9600 tokens (75 tiles)
 # take the one-CTA-per-tile kernel, at 384 and at 512 experts (two-stage ring).
 GRID_CASES = [(64, 8, 256, 2), (1, 384, 4096, 8), (777, 384, 4096, 8), (300, 200, 512, 6), (256, 512, 1024, 8),
               (129, 128, 256, 1), (9600, 384, 512, 8), (5000, 384, 512, 8), (5000, 256, 512, 4),
-              (4900, 512, 1024, 8), (9600, 512, 256, 8)]
+              (5000, 128, 256, 2), (4900, 512, 1024, 8), (9600, 512, 256, 8)]
 
 
 def _bufs(cfg, T, E, k, dev):
