@@ -93,6 +93,33 @@ __device__ __forceinline__ void topk_insert(uint32_t* tk, int* ti, uint32_t key,
   ti[0] = above[0] ? e : ti[0];
 }
 
+// Row t's outputs from its top 8 (keys largest first): the softmax over the
+// k selected scores as route_topk_kernel computes it (e_j = exp(l_j - l_0),
+// summed in rank order, one division each), the ids, and the token's bit in
+// each selected expert's bitmap (when the bitmaps are kept).
+__device__ __forceinline__ void write_row_topk(const RouterArgs& args, int t, const uint32_t* tk, const int* ti) {
+  const int k = args.k;
+  float ex[8];
+  float s = 0.0f;
+  const float top = key_logit(tk[0]);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    ex[j] = (j < k) ? exp_own(__fsub_rn(key_logit(tk[j]), top)) : 0.0f;
+    if (j == 0) s = ex[0];
+    else if (j < k) s = __fadd_rn(s, ex[j]);
+  }
+  const int64_t o = static_cast<int64_t>(t) * k;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < k) {
+      args.topk_ids[o + j] = ti[j];
+      args.topk_w[o + j] = __fdiv_rn(ex[j], s);
+      if (args.bitmap != nullptr)
+        atomicOr(&args.bitmap[static_cast<int64_t>(ti[j]) * args.W + (t >> 5)], 1u << (t & 31));
+    }
+  }
+}
+
 // NB: 128-expert blocks of W_r (1..4); ST: ring stages.
 template <int NB, int ST>
 __global__ void __launch_bounds__(kRThreads, 1)
@@ -268,30 +295,11 @@ __global__ void __launch_bounds__(kRThreads, 1)
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
         const uint32_t key = xk[row * 8 + jj];
-        if (key > tk[7]) topk_insert(tk, ti, key, xi[row * 8 + jj]);
+        const int e = xi[row * 8 + jj];
+        if (key > tk[7] && e >= 0 && e < args.E) topk_insert(tk, ti, key, e);
       }
       if (t < args.T) {
-        // softmax over the k selected scores, as route_topk_kernel computes it
-        const int k = args.k;
-        float ex[8];
-        float s = 0.0f;
-        const float top = key_logit(tk[0]);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          ex[j] = (j < k) ? exp_own(__fsub_rn(key_logit(tk[j]), top)) : 0.0f;
-          if (j == 0) s = ex[0];
-          else if (j < k) s = __fadd_rn(s, ex[j]);
-        }
-        const int64_t o = static_cast<int64_t>(t) * k;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j < k) {
-            args.topk_ids[o + j] = ti[j];
-            args.topk_w[o + j] = __fdiv_rn(ex[j], s);
-            if (args.bitmap != nullptr)
-              atomicOr(&args.bitmap[static_cast<int64_t>(ti[j]) * args.W + (t >> 5)], 1u << (t & 31));
-          }
-        }
+        write_row_topk(args, t, tk, ti);
       }
     }
   }
@@ -771,27 +779,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         const int e = ri[row * 8 + jj];
         if (key > tk[7] && e >= 0 && e < args.E) topk_insert(tk, ti, key, e);
       }
-      // softmax over the k selected scores, as route_topk_kernel computes it
-      const int k = args.k;
-      float ex[8];
-      float s = 0.0f;
-      const float top = key_logit(tk[0]);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        ex[j] = (j < k) ? exp_own(__fsub_rn(key_logit(tk[j]), top)) : 0.0f;
-        if (j == 0) s = ex[0];
-        else if (j < k) s = __fadd_rn(s, ex[j]);
-      }
-      const int64_t o = static_cast<int64_t>(t) * k;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j < k) {
-          args.topk_ids[o + j] = ti[j];
-          args.topk_w[o + j] = __fdiv_rn(ex[j], s);
-          if (args.bitmap != nullptr)
-            atomicOr(&args.bitmap[static_cast<int64_t>(ti[j]) * args.W + (t >> 5)], 1u << (t & 31));
-        }
-      }
+      write_row_topk(args, t, tk, ti);
     }
   }
   if (warp == 1 && !*drain_failed) {
