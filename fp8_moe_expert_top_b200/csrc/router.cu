@@ -590,7 +590,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* drain_failed = reinterpret_cast<volatile int*>(tmem_slot + 2);
-  // exchange areas in the ring, used once every MMA of both CTAs is complete
+  // exchange areas in the ring: xk, xi once this CTA's MMAs are complete;
+  // rk, ri once both CTAs' are (after the first cluster barrier)
   uint32_t* xk = reinterpret_cast<uint32_t*>(smem);             // [128][8] keys, second half of this CTA
   int* xi = reinterpret_cast<int*>(smem + kRM * 8 * 4);         // [128][8] experts
   uint32_t* rk = reinterpret_cast<uint32_t*>(smem + kRM * 64);  // [128][8] keys from CTA 1 (CTA 0 only)
